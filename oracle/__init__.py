@@ -1,0 +1,14 @@
+"""fp64 CPU oracle for exact attention (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA library never does.
+Every function is pinned by the ``-m "not gpu"`` tests in
+``tests/test_oracle.py``; no function here is "parity unpinned".
+"""
+from .attention import (  # noqa: F401
+    attention_backward,
+    attention_forward,
+    attention_forward_rows,
+    kv_head,
+    scores,
+)

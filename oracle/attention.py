@@ -1,0 +1,186 @@
+"""CPU fp64 oracle for exact scaled-dot-product attention, forward and backward.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path may import, call or
+link this module: only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` use it.  It shares no code with the CUDA
+library and imports nothing from it.
+
+What it computes
+----------------
+The pages on FlashAttention state that the tiled, IO-aware kernel reaches the
+*same* result as standard attention, up to numerical precision
+("FlashAttention-2" post on t.iss.one/s/quant_prune_distill/56, section
+"Введение"; QbitAI FA1 article on 52ps.vip, section "FlashAttention", "IO
+perceptual precision attention").  Standard attention materialises the full
+score matrix (QbitAI FA2 article on baiyundou.net, section "实验评估", which
+compares against PyTorch standard attention).  So this oracle is that plain
+definition, written out in fp64 with no tiling, no online softmax and no
+deferred rescaling:
+
+    S   = scale * Q_h K_{kv(h)}^T                    [Nq x Nk]
+    S_ij = -inf where causal and j > i               (top-left alignment)
+    LSE_i = m_i + ln sum_j exp(S_ij - m_i),  m_i = max_j S_ij
+    P   = exp(S - LSE)
+    O   = P V_{kv(h)}
+
+and the gradients of L = <O, dO> (the pages only say that the backward pass
+recomputes the attention matrix block by block, same FA2 post, section
+"Введение"; the formulas below are ordinary calculus):
+
+    dV_kv += P^T dO
+    dP     = dO V^T
+    D_i    = sum_j P_ij dP_ij          (equals rowsum(dO * O))
+    dS     = P * (dP - D)
+    dQ     = scale * dS K
+    dK_kv += scale * dS^T Q
+
+Readings where the pages are silent (all listed in the design notes):
+  * GQA/MQA (named on the baiyundou.net FA2 article, section "具体实现",
+    "two small changes") maps query head h to kv head h // (Hq // Hkv).
+  * Causal masking is top-left aligned: key j is visible to query i iff j <= i.
+  * LSE is the natural-log logsumexp of the *scaled* scores.
+
+Rows of the score matrix are independent (FA2 post, section "Параллелизм":
+forward rows are independent), so processing query rows in chunks is exact;
+it only bounds memory.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "kv_head",
+    "scores",
+    "attention_forward",
+    "attention_forward_rows",
+    "attention_backward",
+]
+
+# Rows of S per chunk are chosen so one chunk of S holds at most this many
+# fp64 elements (256 MiB).
+_MAX_CHUNK_ELEMS = 1 << 25
+
+
+def kv_head(h: int, hq: int, hkv: int) -> int:
+    """KV head read by query head ``h``: contiguous groups of Hq/Hkv heads."""
+    if hq % hkv != 0:
+        raise ValueError(f"Hq={hq} is not a multiple of Hkv={hkv}")
+    return h // (hq // hkv)
+
+
+def _as64(x) -> np.ndarray:
+    return np.asarray(x, dtype=np.float64)
+
+
+def scores(q_rows: np.ndarray, k: np.ndarray, scale: float, causal: bool,
+           row_index: np.ndarray) -> np.ndarray:
+    """Scaled, masked score rows S[r, j] for the query rows ``row_index``.
+
+    q_rows: [R, d] (the rows themselves), k: [Nk, d], row_index: [R] absolute
+    query positions (needed for the causal mask)."""
+    s = scale * (q_rows @ k.T)
+    if causal:
+        j = np.arange(k.shape[0])[None, :]
+        s = np.where(j > row_index[:, None], -np.inf, s)
+    return s
+
+
+def _softmax_stats(s: np.ndarray):
+    """Row max-shifted logsumexp and the normalised probabilities."""
+    m = s.max(axis=1)
+    lse = m + np.log(np.exp(s - m[:, None]).sum(axis=1))
+    p = np.exp(s - lse[:, None])
+    return lse, p
+
+
+def _chunk_rows(nq: int, nk: int) -> int:
+    return max(1, min(nq, _MAX_CHUNK_ELEMS // max(1, nk)))
+
+
+def attention_forward(q, k, v, causal: bool, scale: float):
+    """Exact attention forward.
+
+    q: [B, Hq, Nq, d]; k, v: [B, Hkv, Nk, d] (any float dtype; upcast to fp64).
+    Returns (O [B, Hq, Nq, d] fp64, LSE [B, Hq, Nq] fp64)."""
+    q, k, v = _as64(q), _as64(k), _as64(v)
+    b_, hq, nq, d = q.shape
+    hkv, nk = k.shape[1], k.shape[2]
+    o = np.empty((b_, hq, nq, d))
+    lse = np.empty((b_, hq, nq))
+    step = _chunk_rows(nq, nk)
+    for b in range(b_):
+        for h in range(hq):
+            kvh = kv_head(h, hq, hkv)
+            for r0 in range(0, nq, step):
+                rows = np.arange(r0, min(nq, r0 + step))
+                s = scores(q[b, h, rows], k[b, kvh], scale, causal, rows)
+                l_, p = _softmax_stats(s)
+                lse[b, h, rows] = l_
+                o[b, h, rows] = p @ v[b, kvh]
+    return o, lse
+
+
+def attention_forward_rows(q, k, v, causal: bool, scale: float, b: int, h: int,
+                           rows):
+    """O and LSE of selected query rows of one (batch, head).
+
+    Exact for any subset because forward rows are independent.
+    Returns (O [R, d], LSE [R])."""
+    hq, hkv = q.shape[1], k.shape[1]
+    kvh = kv_head(h, hq, hkv)
+    rows = np.asarray(rows, dtype=np.int64)
+    qr = _as64(q[b, h, rows])
+    kk = _as64(k[b, kvh])
+    vv = _as64(v[b, kvh])
+    s = scores(qr, kk, scale, causal, rows)
+    l_, p = _softmax_stats(s)
+    return p @ vv, l_
+
+
+def attention_backward(q, k, v, do, causal: bool, scale: float,
+                       heads=None, return_aux: bool = False):
+    """Exact attention backward by the chain rule on the materialised P.
+
+    q, do: [B, Hq, Nq, d]; k, v: [B, Hkv, Nk, d].
+    ``heads`` optionally restricts the work to a list of (b, kv_head) groups;
+    gradients of the other groups are left as NaN.
+    Returns (dQ, dK, dV) in fp64, plus (O, LSE, D) when ``return_aux``."""
+    q, k, v, do = _as64(q), _as64(k), _as64(v), _as64(do)
+    b_, hq, nq, d = q.shape
+    hkv, nk = k.shape[1], k.shape[2]
+    g = hq // hkv
+    if hq % hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    dq = np.full(q.shape, np.nan)
+    dk = np.full(k.shape, np.nan)
+    dv = np.full(v.shape, np.nan)
+    o = np.full(q.shape, np.nan)
+    lse = np.full((b_, hq, nq), np.nan)
+    dd = np.full((b_, hq, nq), np.nan)
+    groups = heads if heads is not None else [(b, j) for b in range(b_)
+                                              for j in range(hkv)]
+    step = _chunk_rows(nq, nk)
+    for (b, kvh) in groups:
+        kk, vv = k[b, kvh], v[b, kvh]
+        dk_acc = np.zeros((nk, d))
+        dv_acc = np.zeros((nk, d))
+        for h in range(kvh * g, (kvh + 1) * g):
+            for r0 in range(0, nq, step):
+                rows = np.arange(r0, min(nq, r0 + step))
+                qh, doh = q[b, h, rows], do[b, h, rows]
+                s = scores(qh, kk, scale, causal, rows)
+                l_, p = _softmax_stats(s)
+                dv_acc += p.T @ doh
+                dp = doh @ vv.T
+                d_row = (p * dp).sum(axis=1)
+                ds = p * (dp - d_row[:, None])
+                dq[b, h, rows] = scale * (ds @ kk)
+                dk_acc += scale * (ds.T @ qh)
+                o[b, h, rows] = p @ vv
+                lse[b, h, rows] = l_
+                dd[b, h, rows] = d_row
+        dk[b, kvh] = dk_acc
+        dv[b, kvh] = dv_acc
+    if return_aux:
+        return dq, dk, dv, (o, lse, dd)
+    return dq, dk, dv
