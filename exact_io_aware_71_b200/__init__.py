@@ -1,0 +1,18 @@
+"""Exact IO-aware tiled attention for NVIDIA B200 (sm_100a).
+
+The compute lives in ``libfa.so`` (hand-written CUDA, C ABI in
+``include/fa.h``); this package is its ctypes binding plus the seeded input
+generators used by the tests and the benchmark.
+"""
+from .binding import (  # noqa: F401
+    FA_OK,
+    FaError,
+    backward,
+    fa_bwd,
+    fa_bwd_workspace_size,
+    fa_device_status,
+    fa_fwd,
+    fa_status_string,
+    forward,
+    load,
+)

@@ -1,0 +1,129 @@
+"""ctypes binding of libfa's C ABI (include/fa.h).
+
+Argument marshalling only: every step of the attention computation runs in
+the CUDA kernels behind these calls.  There is no fallback; if the shared
+library is missing, loading fails with an error that says how to build it.
+The functions named like the C entry points take raw device pointers (ints);
+``forward`` / ``backward`` accept contiguous torch CUDA tensors, allocate the
+outputs with torch (device memory only) and call the same entry points on
+torch's current stream.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libfa.so")
+
+FA_OK = 0
+STATUS_NAMES = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED",
+                3: "FA_ERR_MISALIGNED", 4: "FA_ERR_WORKSPACE", 5: "FA_ERR_CUDA",
+                6: "FA_ERR_DEVICE_TIMEOUT"}
+
+# Exported symbols declared in include/fa.h.
+SYMBOLS = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_status_string",
+           "fa_device_status")
+
+
+class FaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what} failed: {STATUS_NAMES.get(status, status)}")
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libfa.so (once) and declare the C signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with "
+                          "`python exact_io_aware_71_b200/build.py` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(path)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, vp]
+    lib.fa_fwd.restype = i
+    lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, vp, sz, vp]
+    lib.fa_bwd.restype = i
+    lib.fa_bwd_workspace_size.argtypes = [i, i, i, i, i, i, i]
+    lib.fa_bwd_workspace_size.restype = sz
+    lib.fa_status_string.argtypes = [i]
+    lib.fa_status_string.restype = ctypes.c_char_p
+    lib.fa_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
+    lib.fa_device_status.restype = i
+    _lib = lib
+    return lib
+
+
+# ------------------------------------------------------------ raw C entry points
+def fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, stream) -> int:
+    return load().fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, int(causal), float(scale),
+                         stream)
+
+
+def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, causal, scale,
+           workspace, workspace_bytes, stream) -> int:
+    return load().fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, int(causal),
+                         float(scale), workspace, workspace_bytes, stream)
+
+
+def fa_bwd_workspace_size(B, Hq, Hkv, Nq, Nk, d, causal) -> int:
+    return load().fa_bwd_workspace_size(B, Hq, Hkv, Nq, Nk, d, int(causal))
+
+
+def fa_status_string(status: int) -> str:
+    return load().fa_status_string(status).decode()
+
+
+def fa_device_status(stream=None):
+    where = ctypes.c_int(0)
+    st = load().fa_device_status(stream, ctypes.byref(where))
+    return st, where.value
+
+
+# ------------------------------------------------------------ torch convenience
+def _stream_handle():
+    import torch
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _dims(q, k):
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    return B, Hq, Hkv, Nq, Nk, d
+
+
+def forward(q, k, v, causal: bool, scale: float, out=None, lse=None):
+    """O, LSE for contiguous bf16 CUDA tensors q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d]."""
+    import torch
+    B, Hq, Hkv, Nq, Nk, d = _dims(q, k)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(B, Hq, Nq, dtype=torch.float32, device=q.device)
+    st = fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                B, Hq, Hkv, Nq, Nk, d, causal, scale, _stream_handle())
+    if st != FA_OK:
+        raise FaError(st, "fa_fwd")
+    return out, lse
+
+
+def backward(q, k, v, o, lse, do, causal: bool, scale: float, workspace=None):
+    """dQ, dK, dV (bf16) for the forward inputs/outputs and dO."""
+    import torch
+    B, Hq, Hkv, Nq, Nk, d = _dims(q, k)
+    need = fa_bwd_workspace_size(B, Hq, Hkv, Nq, Nk, d, causal)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    st = fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                B, Hq, Hkv, Nq, Nk, d, causal, scale, workspace.data_ptr(), workspace.numel(),
+                _stream_handle())
+    if st != FA_OK:
+        raise FaError(st, "fa_bwd")
+    return dq, dk, dv

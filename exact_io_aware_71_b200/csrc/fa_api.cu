@@ -1,0 +1,192 @@
+// C ABI of libfa: argument checks, TMA descriptor encoding and kernel launch.
+// Every step of the attention computation runs in the kernels included here;
+// this file only validates, describes the tensors to the TMA unit and launches.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include "fa.h"
+#include "fa_fwd.cuh"
+#include "fa_bwd.cuh"
+
+namespace {
+
+using namespace fa;
+
+__device__ DevStatus g_status;   // one status word per device (module global)
+
+// ---------------------------------------------------------------- checks
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+int check_sizes(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  // Grid and index arithmetic use 32-bit ints for (batch*head) and rows.
+  const int64_t bhq = int64_t(B) * Hq;
+  const int64_t tiles = bhq * ((int64_t(Nq) + 127) / 128);
+  if (bhq > (int64_t(1) << 24) || tiles >= (int64_t(1) << 31)) return FA_ERR_UNSUPPORTED;
+  if (int64_t(B) * Hkv * ((int64_t(Nk) + 127) / 128) * 2 >= (int64_t(1) << 31))
+    return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+// ---------------------------------------------------------------- TMA maps
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// A [heads, rows, d] bf16 tensor seen as 3-D for TMA, 64-element (128-byte)
+// inner boxes with the 128-byte swizzle; rows outside [0, rows) read as zero.
+bool make_map_bf16(CUtensorMap* m, const void* base, int d, int rows, int64_t heads,
+                   int box_rows) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(rows), cuuint64_t(heads)};
+  cuuint64_t strides[2] = {cuuint64_t(d) * 2, cuuint64_t(rows) * cuuint64_t(d) * 2};
+  cuuint32_t box[3] = {64u, cuuint32_t(box_rows), 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// The same for fp32 [heads, rows, d] with 32-element (128-byte) inner boxes.
+bool make_map_f32(CUtensorMap* m, const void* base, int d, int rows, int64_t heads,
+                  int box_rows) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(rows), cuuint64_t(heads)};
+  cuuint64_t strides[2] = {cuuint64_t(d) * 4, cuuint64_t(rows) * cuuint64_t(d) * 4};
+  cuuint32_t box[3] = {32u, cuuint32_t(box_rows), 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+DevStatus* status_ptr() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
+  return static_cast<DevStatus*>(p);
+}
+
+// ---------------------------------------------------------------- forward
+template <int D, bool CAUSAL>
+int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+               const CUtensorMap& mo, const FwdParams& p, cudaStream_t stream) {
+  using C = FwdCfg<D>;
+  auto kern = fa_fwd_kernel<D, CAUSAL>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+      cudaSuccess)
+    return FA_ERR_CUDA;
+  const unsigned grid = unsigned(p.n_qblocks) * unsigned(p.B * p.Hq);
+  kern<<<grid, C::NTHREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fa_status_string(int s) {
+  switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_MISALIGNED: return "FA_ERR_MISALIGNED";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_DEVICE_TIMEOUT: return "FA_ERR_DEVICE_TIMEOUT";
+    default: return "FA_ERR_UNKNOWN";
+  }
+}
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+           int Hkv, int Nq, int Nk, int d, int causal, float scale, cudaStream_t stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  int st = check_sizes(B, Hq, Hkv, Nq, Nk, d, causal, scale);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(lse))
+    return FA_ERR_MISALIGNED;
+
+  const int bc = (d == 256) ? 64 : 128;
+  CUtensorMap mq, mk, mv, mo;
+  if (!make_map_bf16(&mq, q, d, Nq, int64_t(B) * Hq, 128) ||
+      !make_map_bf16(&mk, k, d, Nk, int64_t(B) * Hkv, bc) ||
+      !make_map_bf16(&mv, v, d, Nk, int64_t(B) * Hkv, bc) ||
+      !make_map_bf16(&mo, o, d, Nq, int64_t(B) * Hq, 32))
+    return FA_ERR_CUDA;
+
+  FwdParams p;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Nq = Nq; p.Nk = Nk;
+  p.group = Hq / Hkv;
+  p.n_qblocks = (Nq + 127) / 128;
+  p.causal = causal;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.lse = lse;
+  p.status = status_ptr();
+  if (!p.status) return FA_ERR_CUDA;
+
+  if (d == 64) return causal ? launch_fwd<64, true>(mq, mk, mv, mo, p, stream)
+                             : launch_fwd<64, false>(mq, mk, mv, mo, p, stream);
+  if (d == 128) return causal ? launch_fwd<128, true>(mq, mk, mv, mo, p, stream)
+                              : launch_fwd<128, false>(mq, mk, mv, mo, p, stream);
+  return causal ? launch_fwd<256, true>(mq, mk, mv, mo, p, stream)
+                : launch_fwd<256, false>(mq, mk, mv, mo, p, stream);
+}
+
+size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal) {
+  if (check_sizes(B, Hq, Hkv, Nq, Nk, d, causal, 1.0f) != FA_OK) return 0;
+  return bwd_workspace_bytes(B, Hq, Hkv, Nq, Nk, d);
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dO, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nk,
+           int d, int causal, float scale, void* workspace, size_t workspace_bytes,
+           cudaStream_t stream) {
+  if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  int st = check_sizes(B, Hq, Hkv, Nq, Nk, d, causal, scale);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(lse) ||
+      !aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_MISALIGNED;
+  const size_t need = bwd_workspace_bytes(B, Hq, Hkv, Nq, Nk, d);
+  if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
+  DevStatus* sp = status_ptr();
+  if (!sp) return FA_ERR_CUDA;
+  return launch_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, causal, scale,
+                    workspace, sp, stream);
+}
+
+int fa_device_status(cudaStream_t stream, int* where) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return FA_ERR_CUDA;
+  DevStatus h{0u, 0u}, zero{0u, 0u};
+  if (cudaMemcpyFromSymbol(&h, g_status, sizeof(h)) != cudaSuccess) return FA_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return FA_ERR_CUDA;
+  if (where) *where = int(h.where);
+  return h.timeout ? FA_ERR_DEVICE_TIMEOUT : FA_OK;
+}
+
+}  // extern "C"

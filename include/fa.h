@@ -1,0 +1,101 @@
+/*
+ * libfa: exact, IO-aware tiled attention for one NVIDIA B200 (sm_100a).
+ *
+ * What it computes.  Exact softmax(scale * Q K^T) V and its gradients, the
+ * same result as standard attention up to rounding ("FlashAttention-2" post,
+ * t.iss.one/s/quant_prune_distill/56, section "Введение"; QbitAI FA1
+ * article, 52ps.vip, section "FlashAttention").  Q, K and V are streamed
+ * tile by tile from HBM into on-chip memory and the N x N score matrix is
+ * never written to HBM (same FA1 article, section "FlashAttention", figure
+ * caption; QbitAI FA2 article, baiyundou.net, section "具体实现").  The
+ * backward pass recomputes the probabilities block by block from Q, K, V and
+ * the saved log-sum-exp (FA1 article, section "FlashAttention": "recalculate
+ * attention in backward").
+ *
+ * Conventions shared by every entry point.
+ *  - Element types: q, k, v, o, dO, dq, dk, dv are bf16; lse is fp32.
+ *  - Layout: contiguous row-major [B, H, N, d]; H = Hq for q, o, dO, dq and
+ *    H = Hkv for k, v, dk, dv.  lse is [B, Hq, Nq].
+ *  - GQA / MQA (FA2 article, section "具体实现", second small change): Hkv
+ *    divides Hq and query head h reads kv head h / (Hq / Hkv).
+ *  - Causal masking is top-left aligned: key j is visible to query i iff
+ *    j <= i.  Key blocks that lie wholly above the diagonal are skipped, not
+ *    computed and zeroed (FA2 post, section "Алгоритм вычисления").
+ *  - lse[i] = ln sum_j exp(scale * q_i . k_j) over the visible keys.
+ *  - Head dims d in {64, 128, 256} (FA2 article: head dimension up to 256).
+ *  - Every pointer is a device pointer owned by the caller; the library
+ *    allocates and frees nothing.  q, k, v, o, dO, dq, dk, dv and the
+ *    workspace must be 16-byte aligned (TMA); lse 4-byte aligned.
+ *  - Calls are asynchronous on `stream` (0 = legacy default stream) and never
+ *    synchronise.  Arguments are checked before anything is launched; a
+ *    failed check returns a status and launches nothing.
+ *  - A kernel whose internal pipeline wait exceeds its time limit records an
+ *    error on the device and returns instead of hanging; fa_device_status()
+ *    reports it.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1,    /* null pointer, size < 1, Hq % Hkv != 0, bad scale */
+  FA_ERR_UNSUPPORTED = 2,    /* d not in {64, 128, 256}, or sizes beyond int range */
+  FA_ERR_MISALIGNED = 3,     /* a pointer breaks the alignment rule above */
+  FA_ERR_WORKSPACE = 4,      /* workspace null or smaller than fa_bwd_workspace_size() */
+  FA_ERR_CUDA = 5,           /* a CUDA runtime/driver call or launch failed */
+  FA_ERR_DEVICE_TIMEOUT = 6  /* a kernel gave up on a pipeline wait (see fa_device_status) */
+} fa_status;
+
+/*
+ * Forward pass.  O = softmax(scale * Q K^T [masked]) V and the per-row
+ * natural-log log-sum-exp.
+ *   q   [B, Hq, Nq, d] bf16 (in)      k, v [B, Hkv, Nk, d] bf16 (in)
+ *   o   [B, Hq, Nq, d] bf16 (out)     lse  [B, Hq, Nq] fp32 (out)
+ *   causal: 0 or 1.   scale: finite, > 0 (usually 1/sqrt(d)).
+ * Returns FA_OK or an fa_status code.
+ */
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+           int Hkv, int Nq, int Nk, int d, int causal, float scale, cudaStream_t stream);
+
+/*
+ * Bytes of caller-owned device workspace fa_bwd needs for these sizes (the
+ * fp32 dQ accumulator, the fp32 row terms D = rowsum(dO * O), and fp32
+ * dK/dV partials when a kv head's query group is split across CTAs).
+ * Returns 0 for invalid sizes.
+ */
+size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal);
+
+/*
+ * Backward pass.  Given the forward inputs, its outputs o and lse, and dO,
+ * writes dq [B, Hq, Nq, d], dk and dv [B, Hkv, Nk, d] (all bf16).  For GQA
+ * dk/dv sum over the query heads of each group.  `workspace` must hold
+ * fa_bwd_workspace_size(...) bytes; its contents need not be initialised
+ * and are clobbered.  The same `scale` and `causal` as the forward pass.
+ */
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dO, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nk,
+           int d, int causal, float scale, void* workspace, size_t workspace_bytes,
+           cudaStream_t stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* fa_status_string(int status);
+
+/*
+ * Synchronises `stream`, then reads and clears the current device's kernel
+ * status word.  Returns FA_OK, FA_ERR_DEVICE_TIMEOUT (a kernel gave up on a
+ * pipeline wait; *where, if non-NULL, receives the code of the wait) or
+ * FA_ERR_CUDA.
+ */
+int fa_device_status(cudaStream_t stream, int* where);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FA_H_ */

@@ -1,0 +1,94 @@
+"""The C ABI on the CPU: the library loads, exports every symbol the header
+declares, and rejects bad arguments with a status code before launching
+anything (these calls never reach the GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import exact_io_aware_71_b200 as fa
+from exact_io_aware_71_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa.h")
+
+A = 0x7F0000000000   # a 16-byte-aligned fake device address: never dereferenced
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = fa.load()
+    names = declared_functions()
+    assert set(names) == set(binding.SYMBOLS)
+    for n in names:
+        assert hasattr(lib, n), n
+        assert ctypes.cast(getattr(lib, n), ctypes.c_void_p).value
+
+
+def test_status_strings():
+    for code, name in binding.STATUS_NAMES.items():
+        assert fa.fa_status_string(code) == name
+    assert fa.fa_status_string(99) == "FA_ERR_UNKNOWN"
+
+
+def fwd(**kw):
+    a = dict(q=A, k=A, v=A, o=A, lse=A, B=1, Hq=2, Hkv=2, Nq=128, Nk=128, d=64, causal=0,
+             scale=0.125, stream=None)
+    a.update(kw)
+    return fa.fa_fwd(**a)
+
+
+def bwd(**kw):
+    a = dict(q=A, k=A, v=A, o=A, lse=A, dO=A, dq=A, dk=A, dv=A, B=1, Hq=2, Hkv=2, Nq=128,
+             Nk=128, d=64, causal=0, scale=0.125, workspace=A, workspace_bytes=1 << 40,
+             stream=None)
+    a.update(kw)
+    return fa.fa_bwd(**a)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), 1), (dict(lse=None), 1), (dict(B=0), 1), (dict(Nq=0), 1), (dict(Nk=0), 1),
+    (dict(Hq=3, Hkv=2), 1), (dict(Hkv=0), 1), (dict(scale=0.0), 1), (dict(scale=-1.0), 1),
+    (dict(scale=float("nan")), 1), (dict(scale=float("inf")), 1), (dict(causal=2), 1),
+    (dict(d=32), 2), (dict(d=96), 2), (dict(d=512), 2),
+    (dict(q=A + 8), 3), (dict(o=A + 2), 3), (dict(v=A + 4), 3), (dict(lse=A + 2), 3),
+    (dict(B=1 << 20, Hq=1 << 10, Hkv=1 << 10), 2),
+])
+def test_fwd_rejects_bad_arguments(kw, status):
+    assert fwd(**kw) == status
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dO=None), 1), (dict(dq=None), 1), (dict(Hq=4, Hkv=3), 1), (dict(d=48), 2),
+    (dict(dk=A + 8), 3), (dict(workspace=None), 4), (dict(workspace_bytes=16), 4),
+    (dict(workspace=A + 4), 3),
+])
+def test_bwd_rejects_bad_arguments(kw, status):
+    assert bwd(**kw) == status
+
+
+def test_workspace_size():
+    assert fa.fa_bwd_workspace_size(1, 2, 2, 128, 128, 64, 0) > 0
+    assert fa.fa_bwd_workspace_size(0, 2, 2, 128, 128, 64, 0) == 0
+    assert fa.fa_bwd_workspace_size(1, 3, 2, 128, 128, 64, 0) == 0
+    assert fa.fa_bwd_workspace_size(1, 2, 2, 128, 128, 80, 0) == 0
+    # grows with the problem
+    a = fa.fa_bwd_workspace_size(1, 2, 2, 128, 128, 128, 0)
+    b = fa.fa_bwd_workspace_size(2, 2, 2, 128, 128, 128, 0)
+    assert b >= 2 * a - 4096
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    saved = binding._lib
+    binding._lib = None
+    try:
+        with pytest.raises(ImportError):
+            binding.load(str(tmp_path / "nope.so"))
+    finally:
+        binding._lib = saved
