@@ -1,0 +1,436 @@
+#!/usr/bin/env python
+"""Throughput of exact attention forward + backward on B200 through libfa.
+
+One *step* is one pass of the whole hot path on one batch: fa_fwd (tiled
+forward, O and LSE) followed by the three backward stages (preprocess, main,
+dQ convert), on the standard training shape B=8, H=16, N=2048, d=128,
+non-causal, bf16 inputs iid N(0, 1) drawn from a fixed seed.
+
+Prints ONE JSON line (rank 0).  ``value`` is whole-job attention TFLOP/s over
+all ranks, with the nominal FLOP count 3.5 * 4*B*H*N^2*d per step (forward
+4*B*H*N^2*d, backward 2.5x that).  Timing: W untimed warm-up steps, then K
+steps between a barrier + synchronize on both sides, CUDA events on the
+launching stream, max over ranks.  Inputs (448 MiB read per step) exceed
+the 126 MB L2, so no flush is needed between steps.
+
+``--impl reference`` times the fp64 CPU oracle instead (the only other place
+this script runs it), on a bounded sample of the same workload.
+Multi-GPU (torchrun): every rank runs an independent batch of the same shape
+(weak scaling, no collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+DEFAULT_WORKLOAD = "train_b8h16n2048d128_full"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["exact_io_aware_71_b200/csrc/sm100.cuh", "exact_io_aware_71_b200/csrc/fa_fwd.cuh",
+                  "exact_io_aware_71_b200/csrc/fa_bwd.cuh"]
+METRIC = "attention fwd / fwd+bwd TFLOP/s (bf16, 1×B200) and % of dense BF16 peak"
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU work for the oracle baseline sample")
+    return ap.parse_args(argv)
+
+
+# ----------------------------------------------------------------- host logic
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return {k: float(pk[k]) for k in FALLBACK_PEAKS}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    for r in rec.get("entries", []):
+        if (r.get("kernel") == kernel and r.get("workload") == workload
+                and r.get("src_sha") == kernel_source_hash()):
+            return r.get("dram_bytes_per_launch")
+    return None
+
+
+def aggregate(local_ms: float, local_units: float, world: int, reduce_max=None):
+    """Whole-job throughput: units processed by all ranks over the slowest
+    rank's time.  ``reduce_max`` maps a local float to the max over ranks."""
+    t = reduce_max(local_ms) if reduce_max else local_ms
+    return t, local_units * world / (t / 1e3)
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        self.proc.wait()
+        return parse_clock_samples(open(self.path).read())
+
+
+def parse_clock_samples(text: str):
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    sm, mx, reasons, power = [], [], set(), []
+    for line in text.strip().splitlines():
+        parts = [p.strip() for p in line.split(",")]
+        if len(parts) < 9:
+            continue
+        try:
+            sm.append(float(parts[1]))
+            mx.append(float(parts[2]))
+            power.append(float(parts[3]))
+        except ValueError:
+            continue
+        for n, v in zip(names, parts[5:9]):
+            if v.lower().startswith("active"):
+                reasons.add(n)
+    if not sm:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+    return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+            "samples": len(sm), "power_w_max": max(power)}
+
+
+# ----------------------------------------------------------------- oracle timing
+_INPUT_CACHE = {}
+
+
+def time_oracle(wl, seconds: float, max_groups=None):
+    """fp64 oracle forward + backward on whole (batch, kv-head) groups of the
+    workload, as many as fit in about `seconds`; returns (TFLOP/s, cores,
+    sample description).  Work is exact per group, so the rate scales."""
+    from threadpoolctl import threadpool_limits
+
+    import oracle
+    from exact_io_aware_71_b200.inputs import make_inputs
+
+    cores = len(os.sched_getaffinity(0))
+    if wl.name not in _INPUT_CACHE:
+        _INPUT_CACHE.clear()
+        _INPUT_CACHE[wl.name] = make_inputs(wl)
+    q, k, v, do = _INPUT_CACHE[wl.name]
+    g = wl.Hq // wl.Hkv
+    groups = [(b, j) for b in range(wl.B) for j in range(wl.Hkv)]
+    per_group_flops = 3.5 * wl.fwd_flops() / len(groups)
+    done, t_total = 0, 0.0
+    with threadpool_limits(limits=cores):
+        for (b, j) in groups:
+            if max_groups is not None and done >= max_groups:
+                break
+            qs = q[b:b + 1, j * g:(j + 1) * g].double().numpy()
+            dos = do[b:b + 1, j * g:(j + 1) * g].double().numpy()
+            ks = k[b:b + 1, j:j + 1].double().numpy()
+            vs = v[b:b + 1, j:j + 1].double().numpy()
+            t0 = time.perf_counter()
+            oracle.attention_backward(qs, ks, vs, dos, wl.causal, wl.scale, return_aux=True)
+            t_total += time.perf_counter() - t0
+            done += 1
+            if max_groups is None and t_total >= seconds and done >= 2:
+                break
+    tflops = done * per_group_flops / t_total / 1e12
+    sample = (f"fp64 NumPy oracle fwd+bwd on {done} of {len(groups)} (batch, kv-head) groups "
+              f"({g} query head(s) each) of {wl.name}; {t_total:.1f} s of CPU work; "
+              f"rate scaled exactly by FLOPs")
+    return tflops, cores, sample, t_total, done * per_group_flops
+
+
+# ----------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+
+    from exact_io_aware_71_b200 import binding as fa
+    from exact_io_aware_71_b200.inputs import make_inputs, workloads
+
+    wl = workloads()[args.workload]
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    fa.load()
+    seed_wl = wl.with_(seed=wl.seed + 1000 * rank) if world > 1 else wl
+    q, k, v, do = (t.to(dev) for t in make_inputs(seed_wl))
+    o = torch.empty_like(q)
+    lse = torch.empty(wl.B, wl.Hq, wl.Nq, dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    wsb = fa.fa_bwd_workspace_size(wl.B, wl.Hq, wl.Hkv, wl.Nq, wl.Nk, wl.d, wl.causal)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    dims = (wl.B, wl.Hq, wl.Hkv, wl.Nq, wl.Nk, wl.d, int(wl.causal), wl.scale)
+    bwd_args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr()) + dims
+
+    names = ["fa_fwd_kernel", "fa_bwd_pre_kernel", "fa_bwd_main_kernel", "fa_bwd_dq_kernel"]
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        st = fa.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                       *dims, sh)
+        if st:
+            raise fa.FaError(st, "fa_fwd")
+        for i, stage in enumerate((fa.FA_BWD_PRE, fa.FA_BWD_MAIN, fa.FA_BWD_DQ)):
+            if evs:
+                evs[i + 1].record(stream)
+            st = fa.fa_bwd_stage(stage, *bwd_args, ws.data_ptr(), wsb, sh)
+            if st:
+                raise fa.FaError(st, "fa_bwd_stage")
+        if evs:
+            evs[4].record(stream)
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def reduce_max(x):
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    st, where = fa.fa_device_status(sh)
+    if st:
+        raise RuntimeError(f"device status {st} at wait {where} during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    e0.record(stream)
+    for s in range(args.steps):
+        step(evs[s])
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop()
+    local_ms = e0.elapsed_time(e1)
+    per_kernel_ms = [sum(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(args.steps))
+                     / args.steps for i in range(4)]
+    st, where = fa.fa_device_status(sh)
+    if st:
+        raise RuntimeError(f"device status {st} at wait {where} in the timed region")
+
+    flops_step = 3.5 * wl.fwd_flops()
+    t_ms, flops_per_s = aggregate(local_ms, args.steps * flops_step, world, reduce_max)
+    value = flops_per_s / 1e12
+
+    # ---- roofline of the dominant kernel (largest share of the step)
+    peaks, peak_src = load_peaks()
+    dom = max(range(4), key=lambda i: per_kernel_ms[i])
+    algo_flops = [wl.fwd_flops(), None, wl.bwd_flops(), None]
+    if algo_flops[dom] is not None:
+        achieved = algo_flops[dom] / (per_kernel_ms[dom] / 1e3) / 1e12
+        roof = {"bound": "tensor", "kernel": names[dom], "achieved": round(achieved, 2),
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(achieved / peaks["bf16_tflops"], 4),
+                "peak_source": f"{peak_src} bf16 cuBLAS burst (MEASURED_PEAKS.json)"
+                if peak_src == "measured" else "fallback 1.59 PFLOP/s",
+                "traffic": recorded_traffic(names[dom], wl.name)}
+    else:
+        roof = {"bound": "hbm", "kernel": names[dom], "achieved": None, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": None, "traffic": None}
+    fwd_tflops = wl.fwd_flops() / (per_kernel_ms[0] / 1e3) / 1e12
+    bwd_ms = sum(per_kernel_ms[1:])
+    bwd_tflops = wl.bwd_flops() / (bwd_ms / 1e3) / 1e12
+
+    # ---- end to end through the public API with host buffers
+    e2e = run_e2e(args, wl, dev, stream, fa, q, k, v, do, reduce_max, world)
+
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": round(t_ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded iid N(0,1), bf16)",
+        "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "Nq": wl.Nq,
+                   "Nk": wl.Nk, "d": wl.d, "causal": wl.causal,
+                   "step": "fa_fwd + fa_bwd (pre, main, dq)",
+                   "parallelism": f"{world} independent replica(s), no collective",
+                   "l2": "inputs larger than L2 (448 MiB read per step), no flush"},
+        "fwd_tflops": round(fwd_tflops, 2), "bwd_tflops": round(bwd_tflops, 2),
+        "fwd_frac_of_peak": round(fwd_tflops / peaks["bf16_tflops"], 4),
+        "bwd_frac_of_peak": round(bwd_tflops / peaks["bf16_tflops"], 4),
+        "per_kernel_ms": {n: round(t, 4) for n, t in zip(names, per_kernel_ms)},
+        "roofline": roof, "e2e": e2e, "clocks": clk, "gpu_launches": 4 * args.steps,
+    }
+    return out
+
+
+def run_e2e(args, wl, dev, stream, fa, q, k, v, do, reduce_max, world):
+    """Same metric through the public torch-level binding with host buffers:
+    each step copies q, k, v, dO from pinned host memory, runs fa_fwd and
+    fa_bwd, and reads o, lse, dq, dk, dv back to pinned host memory."""
+    import torch
+
+    hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, do))
+    dq_, dk_, dv_ = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    o_ = torch.empty_like(q)
+    lse_ = torch.empty(wl.B, wl.Hq, wl.Nq, dtype=torch.float32, device=dev)
+    outs_h = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (o_, lse_, dq_, dk_, dv_)]
+    dev_in = [torch.empty_like(t) for t in (q, k, v, do)]
+    wsb = fa.fa_bwd_workspace_size(wl.B, wl.Hq, wl.Hkv, wl.Nq, wl.Nk, wl.d, wl.causal)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+
+    def step():
+        for dst, src in zip(dev_in, (hq, hk, hv, hdo)):
+            dst.copy_(src, non_blocking=True)
+        fa.forward(dev_in[0], dev_in[1], dev_in[2], wl.causal, wl.scale, out=o_, lse=lse_)
+        g = fa.backward(dev_in[0], dev_in[1], dev_in[2], o_, lse_, dev_in[3], wl.causal,
+                        wl.scale, workspace=ws)
+        for dst, src in zip(outs_h, (o_, lse_) + g):
+            dst.copy_(src, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    t_ms, fps = aggregate(e0.elapsed_time(e1), args.e2e_steps * 3.5 * wl.fwd_flops(), world,
+                          reduce_max)
+    bi = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
+    bo = sum(t.numel() * t.element_size() for t in outs_h)
+    return {"value": round(fps / 1e12, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": bi,
+            "d2h_bytes_per_step": bo, "steps": args.e2e_steps,
+            "ms_per_step": round(t_ms / args.e2e_steps, 3)}
+
+
+# ----------------------------------------------------------------- reference arm
+def run_reference(args):
+    from exact_io_aware_71_b200.inputs import workloads
+    wl = workloads()[args.workload]
+    for _ in range(args.warmup):
+        time_oracle(wl, 0.0, max_groups=1)
+    t_all, f_all = 0.0, 0.0
+    cores = len(os.sched_getaffinity(0))
+    for _ in range(args.steps):
+        _, cores, sample, t, f = time_oracle(wl, 0.0, max_groups=1)
+        t_all += t
+        f_all += f
+    value = f_all / t_all / 1e12
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * t_all / args.steps, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded iid N(0,1), bf16 inputs upcast to fp64)",
+        "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "Nq": wl.Nq,
+                   "Nk": wl.Nk, "d": wl.d, "causal": wl.causal,
+                   "step": "oracle fwd+bwd on one (batch, kv-head) group of the workload"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args)), flush=True)
+        return 0
+
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        out = run_ours(args, rank, world, local_rank)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            from exact_io_aware_71_b200.inputs import workloads
+            tf, cores, sample, _, _ = time_oracle(workloads()[args.workload], args.cpu_seconds)
+            out["cpu_baseline"] = {"value": round(tf, 6), "unit": "TFLOP/s", "cores": cores,
+                                   "kind": "oracle", "sample": sample}
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -9,6 +9,7 @@ from .binding import (  # noqa: F401
     FaError,
     backward,
     fa_bwd,
+    fa_bwd_stage,
     fa_bwd_workspace_size,
     fa_device_status,
     fa_fwd,

@@ -22,8 +22,10 @@ STATUS_NAMES = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED",
                 6: "FA_ERR_DEVICE_TIMEOUT"}
 
 # Exported symbols declared in include/fa.h.
-SYMBOLS = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_status_string",
+SYMBOLS = ("fa_fwd", "fa_bwd", "fa_bwd_stage", "fa_bwd_workspace_size", "fa_status_string",
            "fa_device_status")
+
+FA_BWD_ALL, FA_BWD_PRE, FA_BWD_MAIN, FA_BWD_DQ = 0, 1, 2, 3
 
 
 class FaError(RuntimeError):
@@ -49,6 +51,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fa_fwd.restype = i
     lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, vp, sz, vp]
     lib.fa_bwd.restype = i
+    lib.fa_bwd_stage.argtypes = [i] + lib.fa_bwd.argtypes
+    lib.fa_bwd_stage.restype = i
     lib.fa_bwd_workspace_size.argtypes = [i, i, i, i, i, i, i]
     lib.fa_bwd_workspace_size.restype = sz
     lib.fa_status_string.argtypes = [i]
@@ -69,6 +73,12 @@ def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, causal, scale
            workspace, workspace_bytes, stream) -> int:
     return load().fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, int(causal),
                          float(scale), workspace, workspace_bytes, stream)
+
+
+def fa_bwd_stage(stage, q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, causal, scale,
+                 workspace, workspace_bytes, stream) -> int:
+    return load().fa_bwd_stage(stage, q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d,
+                               int(causal), float(scale), workspace, workspace_bytes, stream)
 
 
 def fa_bwd_workspace_size(B, Hq, Hkv, Nq, Nk, d, causal) -> int:

@@ -5,6 +5,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <algorithm>
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -12,13 +13,20 @@
 
 #include "fa.h"
 #include "fa_fwd.cuh"
+
+namespace fa {
+bool make_map_bf16(CUtensorMap* m, const void* base, int d, int rows, int64_t heads,
+                   int box_rows);
+}
 #include "fa_bwd.cuh"
+
+namespace fa {
+__device__ DevStatus g_status;   // one status word per device (module global)
+}
 
 namespace {
 
 using namespace fa;
-
-__device__ DevStatus g_status;   // one status word per device (module global)
 
 // ---------------------------------------------------------------- checks
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -54,9 +62,11 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+}  // namespace
+
 // A [heads, rows, d] bf16 tensor seen as 3-D for TMA, 64-element (128-byte)
 // inner boxes with the 128-byte swizzle; rows outside [0, rows) read as zero.
-bool make_map_bf16(CUtensorMap* m, const void* base, int d, int rows, int64_t heads,
+bool fa::make_map_bf16(CUtensorMap* m, const void* base, int d, int rows, int64_t heads,
                    int box_rows) {
   auto enc = encode_fn();
   if (!enc) return false;
@@ -70,20 +80,7 @@ bool make_map_bf16(CUtensorMap* m, const void* base, int d, int rows, int64_t he
   return r == CUDA_SUCCESS;
 }
 
-// The same for fp32 [heads, rows, d] with 32-element (128-byte) inner boxes.
-bool make_map_f32(CUtensorMap* m, const void* base, int d, int rows, int64_t heads,
-                  int box_rows) {
-  auto enc = encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(rows), cuuint64_t(heads)};
-  cuuint64_t strides[2] = {cuuint64_t(d) * 4, cuuint64_t(rows) * cuuint64_t(d) * 4};
-  cuuint32_t box[3] = {32u, cuuint32_t(box_rows), 1u};
-  cuuint32_t estr[3] = {1u, 1u, 1u};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
+namespace {
 
 DevStatus* status_ptr() {
   void* p = nullptr;
@@ -161,10 +158,18 @@ size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int 
   return bwd_workspace_bytes(B, Hq, Hkv, Nq, Nk, d);
 }
 
-int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
-           const void* dO, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nk,
-           int d, int causal, float scale, void* workspace, size_t workspace_bytes,
-           cudaStream_t stream) {
+int fa_bwd_stage(int stage, const void* q, const void* k, const void* v, const void* o,
+                 const float* lse, const void* dO, void* dq, void* dk, void* dv, int B, int Hq,
+                 int Hkv, int Nq, int Nk, int d, int causal, float scale, void* workspace,
+                 size_t workspace_bytes, cudaStream_t stream) {
+  int stages;
+  switch (stage) {
+    case FA_BWD_ALL: stages = 7; break;
+    case FA_BWD_PRE: stages = 1; break;
+    case FA_BWD_MAIN: stages = 2; break;
+    case FA_BWD_DQ: stages = 4; break;
+    default: return FA_ERR_INVALID_ARG;
+  }
   if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
   int st = check_sizes(B, Hq, Hkv, Nq, Nk, d, causal, scale);
   if (st != FA_OK) return st;
@@ -176,8 +181,16 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
   if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
   DevStatus* sp = status_ptr();
   if (!sp) return FA_ERR_CUDA;
-  return launch_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, causal, scale,
-                    workspace, sp, stream);
+  return launch_bwd(stages, q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, causal,
+                    scale, workspace, sp, stream);
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dO, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nk,
+           int d, int causal, float scale, void* workspace, size_t workspace_bytes,
+           cudaStream_t stream) {
+  return fa_bwd_stage(FA_BWD_ALL, q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, causal,
+                      scale, workspace, workspace_bytes, stream);
 }
 
 int fa_device_status(cudaStream_t stream, int* where) {

@@ -1,14 +1,599 @@
-// Backward pass (placeholder until the kernels land).
+// Backward pass of exact tiled attention on sm_100a.
+//
+// The backward pass recomputes the probabilities block by block from Q, K
+// and the saved log-sum-exp instead of storing them (QbitAI FA1 article,
+// section "FlashAttention": recalculation in the backward pass), and it is
+// parallel over key blocks, whose gradients are independent (FA2 post,
+// section "Параллелизм": in the backward pass the columns are independent).
+//
+// Three kernels:
+//   fa_bwd_pre      D_i = sum_c dO_ic * O_ic and LSE_i * log2(e) into padded
+//                   fp32 rows, and dQacc <- 0            (HBM-bound)
+//   fa_bwd_main     one CTA per (batch, kv head, 128-key block[, d half]):
+//                   K_j, V_j stay in shared memory; for every query head of
+//                   the kv group and every query block i at or below the
+//                   diagonal:
+//                     S^T  = K_j Q_i^T           (TMEM, lanes = keys)
+//                     P^T  = exp2(S^T * scale*log2e - LSE_i*log2e)
+//                     dV_j += P^T dO_i           (P^T read from TMEM)
+//                     dP^T = V_j dO_i^T
+//                     dS^T = P^T o (dP^T - D_i)
+//                     dK_j += dS^T Q_i           (dS^T read from TMEM)
+//                     dQ_i^T = K_j^T dS^T  -> fp32 reduce-add into dQacc
+//                   then dK_j * scale and dV_j are written as bf16
+//   fa_bwd_dq       dq = bf16(scale * dQacc)              (HBM-bound)
+//
+// TMEM (512 columns): S^T | dP^T | dQ^T | dK | dV; P^T and dS^T overwrite S^T
+// and dP^T in place as packed bf16.  For d = 256 the dK / dV accumulators
+// alone would fill TMEM, so two CTAs share a key block, each owning one
+// 128-wide half of d for dK, dV and dQ (both recompute S and dP).
 #pragma once
 #include "sm100.cuh"
+
 namespace fa {
+
+template <int D>
+struct BwdCfg {
+  static constexpr int BC = 128;                        // keys per CTA (TMEM lanes)
+  static constexpr int BR = (D == 64) ? 128 : 64;       // query rows per step
+  static constexpr int DH = (D == 256) ? 128 : D;       // d columns owned by a CTA
+  static constexpr int NSPLIT = D / DH;                 // CTAs per key block
+  static constexpr int KCH = D / 64;
+  static constexpr int QS = (D == 256) ? 1 : 3;         // Q/dO pipeline stages
+  static constexpr int K_BYTES = BC * D * 2;
+  static constexpr int QT_BYTES = BR * D * 2;           // one Q or dO tile
+  static constexpr int STAGE_BYTES = 2 * QT_BYTES + 2 * BR * 4;
+  static constexpr int STAGE_STRIDE = (STAGE_BYTES + 1023) / 1024 * 1024;
+  static constexpr int DS_BYTES = BC * BR * 2;
+  static constexpr int TM_S = 0, TM_DP = BR, TM_DQ = 2 * BR, TM_DK = 3 * BR, TM_DV = 3 * BR + DH;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int NTHREADS = 192;
+  static constexpr int SMEM_BYTES = 2 * K_BYTES + QS * STAGE_STRIDE + DS_BYTES + 1024 + 1024;
+  static_assert(TM_DV + DH <= TMEM_COLS, "TMEM budget");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+  static_assert(QS * STAGE_STRIDE >= 2 * BC * DH * 2, "dK/dV staging fits in the Q/dO stages");
+};
+
+inline int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+// Workspace: dQacc fp32 [B*Hq, Nq, d] | Dpad fp32 [B*Hq, Nq_pad] | Lpad fp32 [B*Hq, Nq_pad]
+struct BwdWorkspace {
+  size_t dq_off, d_off, l_off, total;
+};
+inline BwdWorkspace bwd_workspace_layout(int B, int Hq, int Nq, int d) {
+  const size_t bh = size_t(B) * Hq;
+  const size_t nq_pad = size_t(round_up(Nq, 128));
+  BwdWorkspace w;
+  w.dq_off = 0;
+  w.d_off = (bh * Nq * d * 4 + 255) / 256 * 256;
+  w.l_off = w.d_off + (bh * nq_pad * 4 + 255) / 256 * 256;
+  w.total = w.l_off + (bh * nq_pad * 4 + 255) / 256 * 256;
+  return w;
+}
 inline size_t bwd_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d) {
   (void)Hkv; (void)Nk;
-  return size_t(B) * Hq * Nq * (size_t(d) + 1) * 4;
+  return bwd_workspace_layout(B, Hq, Nq, d).total;
 }
-inline int launch_bwd(const void*, const void*, const void*, const void*, const float*,
-                      const void*, void*, void*, void*, int, int, int, int, int, int, int, float,
-                      void*, DevStatus*, cudaStream_t) {
+
+// ------------------------------------------------------------------ pre
+// One group of D/8 threads per row; each thread handles 8 consecutive
+// elements (16 bytes) of O and dO and zeroes 8 floats of dQacc.
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_pre_kernel(
+    const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
+    const float* __restrict__ lse, float* __restrict__ dqacc, float* __restrict__ Dpad,
+    float* __restrict__ Lpad, int rows_bh, int Nq, int Nq_pad) {
+  constexpr int TPR = D / 8;                       // threads per row
+  constexpr int RPB = 256 / TPR;                   // rows per block pass
+  const int sub = threadIdx.x % TPR;
+  const int rlocal = threadIdx.x / TPR;
+  const long long total = (long long)rows_bh * Nq_pad;
+  for (long long r = (long long)blockIdx.x * RPB + rlocal; r < total;
+       r += (long long)gridDim.x * RPB) {
+    const long long bh = r / Nq_pad;
+    const int q = int(r - bh * Nq_pad);
+    float acc = 0.f;
+    const bool valid = q < Nq;
+    if (valid) {
+      const size_t e = (size_t(bh) * Nq + q) * D + sub * 8;
+      const uint4 ov = *reinterpret_cast<const uint4*>(o + e);
+      const uint4 dv = *reinterpret_cast<const uint4*>(dO + e);
+      const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
+      const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 a = __bfloat1622float2(o2[i]);
+        const float2 b = __bfloat1622float2(d2[i]);
+        acc = fmaf(a.x, b.x, acc);
+        acc = fmaf(a.y, b.y, acc);
+      }
+      float4* z = reinterpret_cast<float4*>(dqacc + e);
+      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (sub == 0) {
+      const size_t pi = size_t(bh) * Nq_pad + q;
+      Dpad[pi] = valid ? acc : 0.f;
+      Lpad[pi] = valid ? lse[size_t(bh) * Nq + q] * 1.4426950408889634f : INFINITY;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ dq convert
+__global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const float* __restrict__ dqacc,
+                                                        __nv_bfloat16* __restrict__ dq,
+                                                        long long n8, float scale) {
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
+       i += (long long)gridDim.x * blockDim.x) {
+    const float4 a = reinterpret_cast<const float4*>(dqacc)[2 * i];
+    const float4 b = reinterpret_cast<const float4*>(dqacc)[2 * i + 1];
+    uint4 out;
+    out.x = pack_bf16(a.x * scale, a.y * scale);
+    out.y = pack_bf16(a.z * scale, a.w * scale);
+    out.z = pack_bf16(b.x * scale, b.y * scale);
+    out.w = pack_bf16(b.z * scale, b.w * scale);
+    reinterpret_cast<uint4*>(dq)[i] = out;
+  }
+}
+
+// ------------------------------------------------------------------ main
+struct BwdParams {
+  int B, Hq, Hkv, Nq, Nk, Nq_pad;
+  int group;          // Hq / Hkv
+  int n_kblocks;      // ceil(Nk / 128)
+  int n_qblocks;      // ceil(Nq / BR)
+  float scale;
+  float scale_log2;
+  const float* Dpad;
+  const float* Lpad;
+  float* dqacc;
+  DevStatus* status;
+};
+
+enum : unsigned { WB_KV = 16, WB_QEMPTY, WB_QFULL, WB_S, WB_DP, WB_P, WB_DS, WB_DQFULL,
+                  WB_DQEMPTY, WB_FINAL, WB_DRAIN };
+
+__device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_t bytes,
+                                             uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
+    fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ,
+                       const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV,
+                       const __grid_constant__ CUtensorMap tmdO,
+                       const __grid_constant__ CUtensorMap tmdK,
+                       const __grid_constant__ CUtensorMap tmdV, const BwdParams p) {
+  using C = BwdCfg<D>;
+  constexpr int BR = C::BR, BC = C::BC, DH = C::DH, QS = C::QS;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sK = smem;                                   // [KCH][BC][128B]
+  uint8_t* sV = sK + C::K_BYTES;
+  uint8_t* sStage = sV + C::K_BYTES;                    // QS x {Q | dO | L | D}
+  uint8_t* sdS = sStage + QS * C::STAGE_STRIDE;         // [BR/64][BC][128B] dS^T
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sdS + C::DS_BYTES);
+  uint64_t* bar_kv = bars + 0;
+  uint64_t* bar_qfull = bars + 1;                       // [QS]
+  uint64_t* bar_qempty = bars + 1 + QS;                 // [QS]
+  uint64_t* bar_s = bars + 1 + 2 * QS;
+  uint64_t* bar_dp = bars + 2 + 2 * QS;
+  uint64_t* bar_p = bars + 3 + 2 * QS;
+  uint64_t* bar_ds = bars + 4 + 2 * QS;
+  uint64_t* bar_dqfull = bars + 5 + 2 * QS;
+  uint64_t* bar_dqempty = bars + 6 + 2 * QS;
+  uint64_t* bar_final = bars + 7 + 2 * QS;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 8 + 2 * QS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // Work unit: (batch, kv head, key block, d half).  Key blocks near the
+  // start see the most query blocks under the causal mask; they go first.
+  const int split = blockIdx.x % C::NSPLIT;
+  const int rest = blockIdx.x / C::NSPLIT;
+  const int kb = rest % p.n_kblocks;
+  const int bkv = rest / p.n_kblocks;
+  const int b = bkv / p.Hkv;
+  const int hkv = bkv - b * p.Hkv;
+  const int key0 = kb * BC;
+  const int i0 = CAUSAL ? (key0 / BR) : 0;              // first query block that sees key0
+  const int n_i = max(0, p.n_qblocks - i0);
+  const int n_steps = p.group * n_i;
+  const int dcol0 = split * DH;                         // first d column owned here
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_kv, 1);
+    for (int i = 0; i < QS; ++i) {
+      mbar_init(bar_qfull + i, 1);
+      mbar_init(bar_qempty + i, 1);
+    }
+    mbar_init(bar_s, 1);
+    mbar_init(bar_dp, 1);
+    mbar_init(bar_p, 128);
+    mbar_init(bar_ds, 128);
+    mbar_init(bar_dqfull, 1);
+    mbar_init(bar_dqempty, 128);
+    mbar_init(bar_final, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_holder, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && n_steps > 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmdO);
+      mbar_arrive_expect_tx(bar_kv, 2 * C::K_BYTES);
+      for (int c = 0; c < C::KCH; ++c) {
+        tma_load_3d(sK + c * BC * 128, &tmK, bar_kv, c * 64, key0, bkv);
+        tma_load_3d(sV + c * BC * 128, &tmV, bar_kv, c * 64, key0, bkv);
+      }
+      int issued = 0;
+      for (int t = 0; t < n_steps; ++t) {
+        const int hh = t / n_i;
+        const int qi = i0 + (t - hh * n_i);
+        const int bh = b * p.Hq + hkv * p.group + hh;
+        const int st = t % QS;
+        if (!mbar_wait(bar_qempty + st, ((t / QS) & 1) ^ 1, abort_flag, p.status, WB_QEMPTY))
+          break;
+        uint8_t* sq = sStage + st * C::STAGE_STRIDE;
+        uint8_t* sdo = sq + C::QT_BYTES;
+        float* sl = reinterpret_cast<float*>(sdo + C::QT_BYTES);
+        float* sd = sl + BR;
+        mbar_arrive_expect_tx(bar_qfull + st, C::STAGE_BYTES);
+        for (int c = 0; c < C::KCH; ++c) {
+          tma_load_3d(sq + c * BR * 128, &tmQ, bar_qfull + st, c * 64, qi * BR, bh);
+          tma_load_3d(sdo + c * BR * 128, &tmdO, bar_qfull + st, c * 64, qi * BR, bh);
+        }
+        const size_t ro = size_t(bh) * p.Nq_pad + size_t(qi) * BR;
+        bulk_load_1d(sl, p.Lpad + ro, BR * 4, bar_qfull + st);
+        bulk_load_1d(sd, p.Dpad + ro, BR * 4, bar_qfull + st);
+        ++issued;
+      }
+      if (issued < n_steps) {
+        for (int t = issued - 1; t >= 0 && t >= issued - QS; --t) {
+          volatile int no_abort = 0;
+          mbar_wait(bar_qfull + (t % QS), (t / QS) & 1, &no_abort, nullptr, WB_DRAIN);
+        }
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n_steps > 0) {
+      constexpr uint32_t ID_S = idesc_bf16_f32(128, BR, 0, 0);    // S^T, dP^T: K-major both
+      constexpr uint32_t ID_KV = idesc_bf16_f32(128, DH, 0, 1);   // dV, dK: B MN-major
+      constexpr uint32_t ID_DQ = idesc_bf16_f32(128, BR, 1, 1);   // dQ^T: A, B MN-major
+      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aS0 = smem_u32(sStage);
+      const uint32_t adS = smem_u32(sdS);
+      bool ok = mbar_wait(bar_kv, 0, abort_flag, p.status, WB_KV);
+      tc_fence_after();
+      for (int t = 0; t < n_steps && ok; ++t) {
+        const int st = t % QS;
+        const uint32_t aQ = aS0 + st * C::STAGE_STRIDE;
+        const uint32_t adO = aQ + C::QT_BYTES;
+        if (!(ok = mbar_wait(bar_qfull + st, (t / QS) & 1, abort_flag, p.status, WB_QFULL)))
+          break;
+        tc_fence_after();
+        // S^T = K Q^T and dP^T = V dO^T  (M = 128 keys, N = BR queries, K = d)
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ko = (kk >> 2) * BC * 128 + (kk & 3) * 32;
+          const uint32_t qo = (kk >> 2) * BR * 128 + (kk & 3) * 32;
+          umma_ss(tmem + C::TM_S, sdesc_sw128(aK + ko, 16, 1024), sdesc_sw128(aQ + qo, 16, 1024),
+                  ID_S, kk > 0);
+        }
+        umma_commit(bar_s);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ko = (kk >> 2) * BC * 128 + (kk & 3) * 32;
+          const uint32_t qo = (kk >> 2) * BR * 128 + (kk & 3) * 32;
+          umma_ss(tmem + C::TM_DP, sdesc_sw128(aV + ko, 16, 1024),
+                  sdesc_sw128(adO + qo, 16, 1024), ID_S, kk > 0);
+        }
+        umma_commit(bar_dp);
+        // dV += P^T dO  (A = P^T in TMEM, B = dO[:, dcol0:dcol0+DH] MN-major)
+        if (!(ok = mbar_wait(bar_p, t & 1, abort_flag, p.status, WB_P))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BR / 16; ++kk) {
+          const uint32_t bo = (dcol0 / 64) * BR * 128 + kk * 2048;
+          umma_ts(tmem + C::TM_DV, tmem + C::TM_S + kk * 8, sdesc_sw128(adO + bo, BR * 128, 1024),
+                  ID_KV, (t > 0 || kk > 0) ? 1u : 0u);
+        }
+        // dK += dS^T Q
+        if (!(ok = mbar_wait(bar_ds, t & 1, abort_flag, p.status, WB_DS))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BR / 16; ++kk) {
+          const uint32_t bo = (dcol0 / 64) * BR * 128 + kk * 2048;
+          umma_ts(tmem + C::TM_DK, tmem + C::TM_DP + kk * 8, sdesc_sw128(aQ + bo, BR * 128, 1024),
+                  ID_KV, (t > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(bar_qempty + st);
+        // dQ^T = K^T dS^T  (M = 128 rows of d, N = BR queries, K = 128 keys).
+        // For d = 64 the upper 64 rows of M read the V tile and are ignored.
+        if (!(ok = mbar_wait(bar_dqempty, (t & 1) ^ 1, abort_flag, p.status, WB_DQEMPTY))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BC / 16; ++kk) {
+          const uint32_t ao = (dcol0 / 64) * BC * 128 + kk * 2048;
+          umma_ss(tmem + C::TM_DQ, sdesc_sw128(aK + ao, BC * 128, 1024),
+                  sdesc_sw128(adS + kk * 2048, BC * 128, 1024), ID_DQ, kk > 0);
+        }
+        umma_commit(bar_dqfull);
+      }
+      umma_commit(bar_final);
+      volatile int no_abort = 0;
+      mbar_wait(bar_final, 0, &no_abort, nullptr, WB_DRAIN);
+    }
+  } else {
+    // ------------------------------------------------------------ compute warps
+    const int r = threadIdx.x;                     // key row == TMEM lane
+    const uint32_t tl = tmem + (uint32_t(warp * 32) << 16);
+    const int key = key0 + r;
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+    for (int t = 0; t < n_steps; ++t) {
+      const int hh = t / n_i;
+      const int qi = i0 + (t - hh * n_i);
+      const int bh = b * p.Hq + hkv * p.group + hh;
+      const int st = t % QS;
+      const float* sl = reinterpret_cast<const float*>(sStage + st * C::STAGE_STRIDE +
+                                                       2 * C::QT_BYTES);
+      const float* sd = sl + BR;
+      const int q0 = qi * BR;
+      // Queries visible to this key: q >= key (causal); columns c < cstart
+      // are masked.  Padding keys (>= Nk) are masked in every column.
+      const bool need_mask = (CAUSAL && (key0 + BC - 1 > q0)) || (key0 + BC > p.Nk);
+      const int cstart = key >= p.Nk ? BR : (CAUSAL ? key - q0 : 0);
+
+      ok = mbar_wait(bar_qfull + st, (t / QS) & 1, abort_flag, p.status, WB_QFULL) &&
+           mbar_wait(bar_s, t & 1, abort_flag, p.status, WB_S);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      tc_fence_after();
+      float P[BR];
+#pragma unroll
+      for (int c = 0; c < BR / 32; ++c) {
+        uint32_t u[32];
+        FA_TMEM_LD32(tl + C::TM_S + c * 32, u);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const int cc = c * 32 + i;
+          float p0 = ex2(fmaf(__uint_as_float(u[i]), sl2, -sl[cc]));
+          float p1 = ex2(fmaf(__uint_as_float(u[i + 1]), sl2, -sl[cc + 1]));
+          if (need_mask) {
+            if (cc < cstart) p0 = 0.f;
+            if (cc + 1 < cstart) p1 = 0.f;
+          }
+          P[cc] = p0;
+          P[cc + 1] = p1;
+          pk[i / 2] = pack_bf16(p0, p1);
+        }
+        FA_TMEM_ST16(tl + C::TM_S + c * 16, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar_p);
+
+      ok = mbar_wait(bar_dp, t & 1, abort_flag, p.status, WB_DP);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < BR / 32; ++c) {
+        uint32_t u[32];
+        FA_TMEM_LD32(tl + C::TM_DP + c * 32, u);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const int cc = c * 32 + i;
+          const float d0 = P[cc] * (__uint_as_float(u[i]) - sd[cc]);
+          const float d1 = P[cc + 1] * (__uint_as_float(u[i + 1]) - sd[cc + 1]);
+          pk[i / 2] = pack_bf16(d0, d1);
+        }
+        FA_TMEM_ST16(tl + C::TM_DP + c * 16, pk);
+        // dS^T row r, queries c*32 .. c*32+31: half of a 128-byte swizzled row
+        uint8_t* row = sdS + (c >> 1) * BC * 128 + r * 128;
+#pragma unroll
+        for (int u4 = 0; u4 < 4; ++u4) {
+          const int unit = (c & 1) * 4 + u4;
+          *reinterpret_cast<uint4*>(row + ((unit ^ (r & 7)) * 16)) =
+              make_uint4(pk[4 * u4], pk[4 * u4 + 1], pk[4 * u4 + 2], pk[4 * u4 + 3]);
+        }
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar_ds);
+
+      // dQ^T for this step: lane r holds d column dcol0 + r for BR queries.
+      ok = mbar_wait(bar_dqfull, t & 1, abort_flag, p.status, WB_DQFULL);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      tc_fence_after();
+      if (r < DH) {
+        float* dst = p.dqacc + (size_t(bh) * p.Nq + q0) * D + dcol0 + r;
+        const int nvalid = min(BR, p.Nq - q0);
+#pragma unroll
+        for (int c = 0; c < BR / 32; ++c) {
+          uint32_t u[32];
+          FA_TMEM_LD32(tl + C::TM_DQ + c * 32, u);
+          tmem_wait_ld();
+          if (c == BR / 32 - 1) {
+            tc_fence_before();
+            mbar_arrive(bar_dqempty);
+          }
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (c * 32 + i < nvalid) atomicAdd(dst + size_t(c * 32 + i) * D, __uint_as_float(u[i]));
+        }
+      } else {
+        tc_fence_before();
+        mbar_arrive(bar_dqempty);
+      }
+    }
+
+    // ---- epilogue: dK = scale * dK_acc and dV, bf16, through shared memory
+    if (ok && n_steps > 0) {
+      ok = mbar_wait(bar_final, 0, abort_flag, p.status, WB_FINAL);
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok) tc_fence_after();
+    }
+    if (ok) {
+      // The Q/dO stages are free now: stage dK then dV (each [DH/64][128][128B]).
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const int tcol = which == 0 ? C::TM_DK : C::TM_DV;
+        const float mul = which == 0 ? p.scale : 1.f;
+        uint8_t* stage = sStage + which * (BC * DH * 2);
+#pragma unroll
+        for (int c = 0; c < DH / 32; ++c) {
+          uint32_t u[32];
+          if (n_steps > 0) {
+            FA_TMEM_LD32(tl + tcol + c * 32, u);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) u[i] = 0u;
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack_bf16(__uint_as_float(u[2 * i]) * mul, __uint_as_float(u[2 * i + 1]) * mul);
+          uint8_t* box = stage + ((c >> 1) * 4 + warp) * 4096 + lane * 128;
+#pragma unroll
+          for (int u4 = 0; u4 < 4; ++u4) {
+            const int unit = (c & 1) * 4 + u4;
+            *reinterpret_cast<uint4*>(box + ((unit ^ (lane & 7)) * 16)) =
+                make_uint4(pk[4 * u4], pk[4 * u4 + 1], pk[4 * u4 + 2], pk[4 * u4 + 3]);
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && key0 + warp * 32 < p.Nk) {
+        for (int which = 0; which < 2; ++which) {
+          const CUtensorMap* tm = which == 0 ? &tmdK : &tmdV;
+          const uint8_t* stage = sStage + which * (BC * DH * 2);
+          for (int c = 0; c < DH / 64; ++c)
+            tma_store_3d(tm, stage + (c * 4 + warp) * 4096, dcol0 + c * 64, key0 + warp * 32, bkv);
+        }
+        bulk_commit();
+        bulk_wait0();
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ launch
+bool make_map_bf16(CUtensorMap* m, const void* base, int d, int rows, int64_t heads, int box_rows);
+
+template <int D, bool CAUSAL>
+int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const void* o,
+                 const float* lse, const void* dO, void* dq, void* dk, void* dv, int B, int Hq,
+                 int Hkv, int Nq, int Nk, float scale, void* workspace, DevStatus* status,
+                 cudaStream_t stream) {
+  using C = BwdCfg<D>;
+  const BwdWorkspace w = bwd_workspace_layout(B, Hq, Nq, D);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* dqacc = reinterpret_cast<float*>(ws + w.dq_off);
+  float* Dpad = reinterpret_cast<float*>(ws + w.d_off);
+  float* Lpad = reinterpret_cast<float*>(ws + w.l_off);
+  const int Nq_pad = round_up(Nq, 128);
+  const int bhq = B * Hq;
+
+  CUtensorMap mq, mk, mv, mdo, mdk, mdv;
+  if ((stages & 2) && (!make_map_bf16(&mq, q, D, Nq, int64_t(bhq), C::BR) ||
+      !make_map_bf16(&mk, k, D, Nk, int64_t(B) * Hkv, C::BC) ||
+      !make_map_bf16(&mv, v, D, Nk, int64_t(B) * Hkv, C::BC) ||
+      !make_map_bf16(&mdo, dO, D, Nq, int64_t(bhq), C::BR) ||
+      !make_map_bf16(&mdk, dk, D, Nk, int64_t(B) * Hkv, 32) ||
+      !make_map_bf16(&mdv, dv, D, Nk, int64_t(B) * Hkv, 32)))
+    return 5;
+
+  if (stages & 1) {
+    constexpr int RPB = 256 / (D / 8);
+    const long long rows = (long long)bhq * Nq_pad;
+    const long long blocks = std::min<long long>((rows + RPB - 1) / RPB, 148LL * 16);
+    fa_bwd_pre_kernel<D><<<unsigned(blocks), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, dqacc,
+        Dpad, Lpad, bhq, Nq, Nq_pad);
+    if (cudaGetLastError() != cudaSuccess) return 5;
+  }
+  if (stages & 2) {
+    auto kern = fa_bwd_main_kernel<D, CAUSAL>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+        cudaSuccess)
+      return 5;
+    BwdParams p;
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Nq = Nq; p.Nk = Nk; p.Nq_pad = Nq_pad;
+    p.group = Hq / Hkv;
+    p.n_kblocks = (Nk + C::BC - 1) / C::BC;
+    p.n_qblocks = (Nq + C::BR - 1) / C::BR;
+    p.scale = scale;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.Dpad = Dpad;
+    p.Lpad = Lpad;
+    p.dqacc = dqacc;
+    p.status = status;
+    const unsigned grid = unsigned(p.n_kblocks) * unsigned(B * Hkv) * C::NSPLIT;
+    kern<<<grid, C::NTHREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdk, mdv, p);
+    if (cudaGetLastError() != cudaSuccess) return 5;
+  }
+  if (stages & 4) {
+    const long long n8 = (long long)bhq * Nq * D / 8;
+    const long long blocks = std::min<long long>((n8 + 255) / 256, 148LL * 16);
+    fa_bwd_dq_kernel<<<unsigned(blocks), 256, 0, stream>>>(
+        dqacc, static_cast<__nv_bfloat16*>(dq), n8, scale);
+    if (cudaGetLastError() != cudaSuccess) return 5;
+  }
+  return 0;
+}
+
+// stages: bit 0 = preprocess, bit 1 = main, bit 2 = dq convert.
+inline int launch_bwd(int stages, const void* q, const void* k, const void* v, const void* o,
+                      const float* lse, const void* dO, void* dq, void* dk, void* dv, int B,
+                      int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale,
+                      void* workspace, DevStatus* status, cudaStream_t stream) {
+#define FA_BWD_CASE(DD)                                                                        \
+  if (d == DD)                                                                                 \
+    return causal ? launch_bwd_t<DD, true>(stages, q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, \
+                                           Nq, Nk, scale, workspace, status, stream)           \
+                  : launch_bwd_t<DD, false>(stages, q, k, v, o, lse, dO, dq, dk, dv, B, Hq,    \
+                                            Hkv, Nq, Nk, scale, workspace, status, stream);
+  FA_BWD_CASE(64)
+  FA_BWD_CASE(128)
+  FA_BWD_CASE(256)
+#undef FA_BWD_CASE
   return 2;
 }
+
 }  // namespace fa

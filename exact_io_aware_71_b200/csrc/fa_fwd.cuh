@@ -22,6 +22,12 @@
 #pragma once
 #include "sm100.cuh"
 
+// A row's O and l are rescaled only when its running max (log2 units) grows
+// by more than this; in between, probabilities reach at most 2^threshold.
+#ifndef FA_RESCALE_LOG2_THRESHOLD
+#define FA_RESCALE_LOG2_THRESHOLD 8.0f
+#endif
+
 namespace fa {
 
 template <int D>
@@ -73,8 +79,11 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
   uint64_t* bar_kv_empty = bars + 1 + NS;
   uint64_t* bar_s_full = bars + 1 + 2 * NS;      // [2]
   uint64_t* bar_p_full = bars + 3 + 2 * NS;      // [2]
-  uint64_t* bar_o_done = bars + 5 + 2 * NS;
-  uint64_t* bar_drain = bars + 6 + 2 * NS;
+  // O-done barriers alternate by key-block parity: softmax warps may drift one
+  // block apart, and with a single barrier a warp already at block j+1 could
+  // mistake the completion of P_{j-1} V_{j-1} (same parity) for P_j V_j.
+  uint64_t* bar_o_done = bars + 5 + 2 * NS;      // [2]
+  uint64_t* bar_drain = bars + 7 + 2 * NS;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 8 + 2 * NS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -103,7 +112,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
       mbar_init(bar_s_full + i, 1);
       mbar_init(bar_p_full + i, BR);
     }
-    mbar_init(bar_o_done, 1);
+    mbar_init(bar_o_done + 0, 1);
+    mbar_init(bar_o_done + 1, 1);
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -205,7 +215,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
           const uint64_t bd = sdesc_sw128(vbase + kk * 16 * 128, BC * 128, 1024);
           umma_ts(tmem + C::TM_O, a_tm + kk * 8, bd, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(bar_o_done);
+        umma_commit(bar_o_done + (j & 1));
         release(slot);
       };
       if (ok) mma_s(0);
@@ -257,11 +267,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
       if (j == 0) {
         m = mc;
       } else {
-        const bool need = mc > m + 8.0f;
+        const bool need = mc > m + FA_RESCALE_LOG2_THRESHOLD;
         if (__any_sync(0xffffffffu, need)) {
           const float mn = need ? mc : m;
           const float alpha = ex2(m - mn);
-          ok = mbar_wait(bar_o_done, (j - 1) & 1, abort_flag, p.status, W_O_DONE);
+          ok = mbar_wait(bar_o_done + ((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag, p.status,
+                         W_O_DONE);
           if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
@@ -299,7 +310,9 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
       tc_fence_before();
       mbar_arrive(bar_p_full + (j & 1));
     }
-    if (ok) ok = mbar_wait(bar_o_done, (n_blocks - 1) & 1, abort_flag, p.status, W_O_DONE);
+    if (ok)
+      ok = mbar_wait(bar_o_done + ((n_blocks - 1) & 1), ((n_blocks - 1) >> 1) & 1, abort_flag,
+                     p.status, W_O_DONE);
     if (__all_sync(0xffffffffu, ok)) {
       tc_fence_after();
       const float inv = 1.0f / lr;

@@ -65,9 +65,9 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
            int Hkv, int Nq, int Nk, int d, int causal, float scale, cudaStream_t stream);
 
 /*
- * Bytes of caller-owned device workspace fa_bwd needs for these sizes (the
- * fp32 dQ accumulator, the fp32 row terms D = rowsum(dO * O), and fp32
- * dK/dV partials when a kv head's query group is split across CTAs).
+ * Bytes of caller-owned device workspace fa_bwd needs for these sizes: the
+ * fp32 dQ accumulator [B, Hq, Nq, d] and two fp32 row vectors (D =
+ * rowsum(dO * O) and LSE * log2 e) padded to 128 rows per head.
  * Returns 0 for invalid sizes.
  */
 size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal);
@@ -83,6 +83,25 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
            const void* dO, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nk,
            int d, int causal, float scale, void* workspace, size_t workspace_bytes,
            cudaStream_t stream);
+
+/* Stages of fa_bwd, for callers that time or schedule them separately. */
+typedef enum {
+  FA_BWD_ALL = 0,   /* the whole backward pass (same as fa_bwd) */
+  FA_BWD_PRE = 1,   /* D = rowsum(dO * O), LSE copy, dQ accumulator := 0 (in the workspace) */
+  FA_BWD_MAIN = 2,  /* dK, dV written; dQ accumulated into the workspace */
+  FA_BWD_DQ = 3     /* dq = scale * dQ accumulator, as bf16 */
+} fa_bwd_stage_t;
+
+/*
+ * One stage of the backward pass, same arguments and checks as fa_bwd.
+ * Issuing FA_BWD_PRE, FA_BWD_MAIN and FA_BWD_DQ in that order on one stream
+ * (with the same workspace, untouched in between) is exactly fa_bwd.
+ * Returns FA_ERR_INVALID_ARG for an unknown stage.
+ */
+int fa_bwd_stage(int stage, const void* q, const void* k, const void* v, const void* o,
+                 const float* lse, const void* dO, void* dq, void* dk, void* dv, int B, int Hq,
+                 int Hkv, int Nq, int Nk, int d, int causal, float scale, void* workspace,
+                 size_t workspace_bytes, cudaStream_t stream);
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* fa_status_string(int status);

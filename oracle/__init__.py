@@ -7,6 +7,7 @@ Every function is pinned by the ``-m "not gpu"`` tests in
 """
 from .attention import (  # noqa: F401
     attention_backward,
+    attention_backward_dq_rows,
     attention_forward,
     attention_forward_rows,
     kv_head,

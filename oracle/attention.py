@@ -54,6 +54,7 @@ __all__ = [
     "attention_forward",
     "attention_forward_rows",
     "attention_backward",
+    "attention_backward_dq_rows",
 ]
 
 # Rows of S per chunk are chosen so one chunk of S holds at most this many
@@ -184,3 +185,22 @@ def attention_backward(q, k, v, do, causal: bool, scale: float,
     if return_aux:
         return dq, dk, dv, (o, lse, dd)
     return dq, dk, dv
+
+
+def attention_backward_dq_rows(q, k, v, do, causal: bool, scale: float, b: int, h: int,
+                               rows):
+    """dQ of selected query rows of one (batch, head).
+
+    Row i of dQ needs only row i of P and dP (D_i is a sum over that row), so
+    any subset of rows is exact on its own.  Returns dQ [R, d] in fp64."""
+    hq, hkv = q.shape[1], k.shape[1]
+    kvh = kv_head(h, hq, hkv)
+    rows = np.asarray(rows, dtype=np.int64)
+    qr, dor = _as64(q[b, h, rows]), _as64(do[b, h, rows])
+    kk, vv = _as64(k[b, kvh]), _as64(v[b, kvh])
+    s = scores(qr, kk, scale, causal, rows)
+    _, p = _softmax_stats(s)
+    dp = dor @ vv.T
+    d_row = (p * dp).sum(axis=1)
+    ds = p * (dp - d_row[:, None])
+    return scale * (ds @ kk)

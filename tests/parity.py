@@ -44,29 +44,41 @@ def report(name, got, ref):
             f"relfro={relfro(got, ref):.3e}")
 
 
-def check_fwd(o, lse, o_ref, lse_ref, representable=False):
-    """The acceptance bar on O and LSE.  With ``representable`` (stress inputs
-    outside the named workloads, whose outputs reach |O| >= 4 where half a
-    bf16 ulp alone exceeds 1e-2) the O bound per element becomes
-    1e-2 + half_ulp_bf16(ref)."""
-    msg = report("O", o, o_ref) + "; " + report("LSE", lse, lse_ref)
+def bound(ref, tol):
+    """Per-element error bound: ``tol`` wherever half a bf16 ulp of the
+    reference is below ``tol``; where it is not (|O| >= 4 for tol = 1e-2,
+    |grad| >= 8 for tol = 2e-2) no bf16 output can meet ``tol`` and the bound
+    is half_ulp(ref) + tol.  Returns (bound array, number of relaxed elements)."""
+    hu = half_ulp_bf16(ref)
+    relaxed = hu >= tol
+    return np.where(relaxed, hu + tol, tol), int(relaxed.sum())
+
+
+def _check_bounded(name, got, ref, tol):
+    b, nrel = bound(ref, tol)
+    err = np.abs(np.asarray(got, np.float64) - np.asarray(ref, np.float64))
+    msg = report(name, got, ref) + f", relaxed={nrel}"
+    assert np.isfinite(got).all(), msg
+    assert (err <= b).all(), msg + f", worst excess={float((err - b).max()):.3e}"
+    return msg
+
+
+def check_fwd(o, lse, o_ref, lse_ref):
+    """O: per element within 1e-2 (see ``bound``) and relative Frobenius
+    <= 5e-3; LSE: max-abs <= 1e-3."""
+    msg = _check_bounded("O", o, o_ref, TOL_O_MAXABS) + "; " + report("LSE", lse, lse_ref)
     print(msg)
-    if representable:
-        excess = np.abs(np.asarray(o, np.float64) - o_ref) - half_ulp_bf16(o_ref)
-        assert excess.max() <= TOL_O_MAXABS, msg
-    else:
-        assert maxabs(o, o_ref) <= TOL_O_MAXABS, msg
     assert relfro(o, o_ref) <= TOL_O_RELFRO, msg
     assert maxabs(lse, lse_ref) <= TOL_LSE_MAXABS, msg
     return msg
 
 
-def check_grads(grads, refs):
-    msgs = [report(n, g, r) for n, g, r in zip(("dQ", "dK", "dV"), grads, refs)]
+def check_grads(grads, refs, names=("dQ", "dK", "dV")):
+    """Each gradient per element within 2e-2 (see ``bound``)."""
+    msgs = []
+    for n, g, r in zip(names, grads, refs):
+        msgs.append(_check_bounded(n, g, r, TOL_GRAD_MAXABS))
     print("; ".join(msgs))
-    for g, r, m in zip(grads, refs, msgs):
-        assert np.isfinite(g).all(), m
-        assert maxabs(g, r) <= TOL_GRAD_MAXABS, "; ".join(msgs)
     return "; ".join(msgs)
 
 

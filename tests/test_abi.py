@@ -73,6 +73,14 @@ def test_bwd_rejects_bad_arguments(kw, status):
     assert bwd(**kw) == status
 
 
+@pytest.mark.parametrize("stage", [-1, 4, 99])
+def test_bwd_stage_rejects_unknown_stage(stage):
+    a = dict(q=A, k=A, v=A, o=A, lse=A, dO=A, dq=A, dk=A, dv=A, B=1, Hq=2, Hkv=2, Nq=128,
+             Nk=128, d=64, causal=0, scale=0.125, workspace=A, workspace_bytes=1 << 40,
+             stream=None)
+    assert fa.fa_bwd_stage(stage, **a) == 1
+
+
 def test_workspace_size():
     assert fa.fa_bwd_workspace_size(1, 2, 2, 128, 128, 64, 0) > 0
     assert fa.fa_bwd_workspace_size(0, 2, 2, 128, 128, 64, 0) == 0

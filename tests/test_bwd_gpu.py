@@ -1,0 +1,134 @@
+"""GPU parity of fa_bwd (with fa_fwd's O and LSE) against the fp64 oracle,
+through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_io_aware_71_b200 import binding as fa
+from exact_io_aware_71_b200.inputs import Workload, make_inputs, workloads
+from tests.parity import check_grads, sample_rows, to64
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def run(wl, qmul=1.0):
+    q, k, v, do = make_inputs(wl)
+    if qmul != 1.0:
+        q = (q.float() * qmul).to(torch.bfloat16)
+    qd, kd, vd, dod = q.to(DEV), k.to(DEV), v.to(DEV), do.to(DEV)
+    o, lse = fa.forward(qd, kd, vd, wl.causal, wl.scale)
+    dq, dk, dv = fa.backward(qd, kd, vd, o, lse, dod, wl.causal, wl.scale)
+    torch.cuda.synchronize()
+    st, where = fa.fa_device_status(None)
+    assert st == 0, f"device status {st} at wait {where}"
+    return (q, k, v, do), (to64(dq), to64(dk), to64(dv))
+
+
+def full_check(wl, qmul=1.0):
+    (q, k, v, do), got = run(wl, qmul)
+    ref = oracle.attention_backward(to64(q), to64(k), to64(v), to64(do), wl.causal, wl.scale)
+    return check_grads(got, ref)
+
+
+def W(B, Hq, Hkv, Nq, Nk, d, causal, seed=21):
+    return Workload(f"b{B}_{Hq}_{Hkv}_{Nq}_{Nk}_{d}_{int(causal)}", B, Hq, Hkv, Nq, Nk, d,
+                    causal, seed)
+
+
+@pytest.mark.parametrize("name", ["tiny_b1h2n128d64_full", "tiny_b1h2n128d64_causal"])
+def test_tiny_workload(name):
+    full_check(workloads()[name])
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("hq,hkv", [(4, 4), (4, 2), (4, 1)])
+def test_head_dims_and_gqa(d, causal, hq, hkv):
+    full_check(W(2, hq, hkv, 384, 384, d, causal))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("n", [1, 17, 127, 129, 1000])
+def test_ragged_lengths(n, d, causal):
+    full_check(W(1, 2, 2, n, n, d, causal, seed=n))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("nq,nk", [(200, 333), (333, 200), (64, 1024), (1024, 64)])
+def test_unequal_lengths(nq, nk, causal):
+    """Includes key blocks no query can see (causal, Nk > Nq): dK = dV = 0."""
+    full_check(W(1, 2, 1, nq, nk, 128, causal, seed=nq + nk))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_mqa_wide_group(causal):
+    """32 query heads on one kv head: the per-CTA loop over the group."""
+    full_check(W(1, 32, 1, 1024, 1024, 128, causal, seed=3))
+
+
+@pytest.mark.parametrize("qmul", [2.0, 4.0])
+def test_large_magnitude_scores(qmul):
+    full_check(W(1, 2, 2, 512, 512, 64, True, seed=9), qmul=qmul)
+
+
+def test_backward_repeatable_within_tolerance():
+    """dQ is accumulated with unordered fp32 atomics, so runs may differ in
+    the last bits; dK and dV are accumulated in a fixed order."""
+    wl = W(1, 4, 2, 640, 640, 128, True)
+    _, g1 = run(wl)
+    _, g2 = run(wl)
+    assert np.array_equal(g1[1], g2[1]) and np.array_equal(g1[2], g2[2])
+    assert np.abs(g1[0] - g2[0]).max() <= 2e-2
+
+
+# --------------------------------------------------------------- full-size workloads
+BWD_WORKLOADS = [n for n, w in workloads().items()
+                 if "bwd" in w.directions and not n.startswith("tiny")]
+
+
+@pytest.mark.parametrize("name", BWD_WORKLOADS)
+def test_full_size(name):
+    """Full-size backward on the GPU.  The oracle runs the complete backward
+    on sampled (batch, kv head) groups whose query group is at most 4 heads
+    (dK/dV need every query row of the group), and dQ on sampled rows of
+    sampled heads for every workload (each dQ row is exact on its own)."""
+    wl = workloads()[name]
+    (q, k, v, do), (dq, dk, dv) = run(wl)
+    for g in (dq, dk, dv):
+        assert np.isfinite(g).all()
+    q, k, v, do = to64(q), to64(k), to64(v), to64(do)
+    g = wl.Hq // wl.Hkv
+    rng = np.random.default_rng(1)
+    if g <= 4:
+        groups = sorted({(0, 0), (wl.B - 1, wl.Hkv - 1),
+                         (int(rng.integers(wl.B)), int(rng.integers(wl.Hkv)))})[:2]
+        ref = oracle.attention_backward(q, k, v, do, wl.causal, wl.scale, heads=groups)
+        sel_q = [(b, h) for (b, j) in groups for h in range(j * g, (j + 1) * g)]
+        got = (np.stack([dq[b, h] for b, h in sel_q]), np.stack([dk[b, j] for b, j in groups]),
+               np.stack([dv[b, j] for b, j in groups]))
+        exp = (np.stack([ref[0][b, h] for b, h in sel_q]),
+               np.stack([ref[1][b, j] for b, j in groups]),
+               np.stack([ref[2][b, j] for b, j in groups]))
+        check_grads(got, exp)
+    heads = [(int(rng.integers(wl.B)), int(rng.integers(wl.Hq))) for _ in range(6)]
+    heads += [(0, 0), (wl.B - 1, wl.Hq - 1)]
+    got, exp = [], []
+    for (b, h) in heads:
+        rows = sample_rows(wl.Nq, 32, seed=7 * b + h)
+        exp.append(oracle.attention_backward_dq_rows(q, k, v, do, wl.causal, wl.scale, b, h,
+                                                     rows))
+        got.append(dq[b, h, rows])
+    check_grads([np.concatenate(got)], [np.concatenate(exp)], names=("dQ rows",))
+    if g > 4:
+        # Sums that hold at any size: rows of dS sum to zero, so the key
+        # gradients of each kv head sum to zero; rows of P sum to one, so the
+        # value gradients sum to the summed output gradients of the group.
+        dv_sum = dv.sum(axis=2)
+        do_sum = do.reshape(wl.B, wl.Hkv, g, wl.Nq, wl.d).sum(axis=(2, 3))
+        scale = np.abs(do_sum).max()
+        assert np.abs(dv_sum - do_sum).max() <= 2e-3 * scale
+        assert np.abs(dk.sum(axis=2)).max() <= 2e-3 * np.abs(dk).sum(axis=2).max()

@@ -303,6 +303,18 @@ def test_gradient_invariants(causal):
     np.testing.assert_allclose(lse, l2, atol=1e-14)
 
 
+def test_dq_rows_match_full_backward():
+    q = rnd((2, 4, 21, 8), 60)
+    k = rnd((2, 2, 21, 8), 61)
+    v = rnd((2, 2, 21, 8), 62)
+    do = rnd((2, 4, 21, 8), 63)
+    for causal in (False, True):
+        dq = oracle.attention_backward(q, k, v, do, causal, 0.4)[0]
+        rows = [0, 1, 7, 20]
+        got = oracle.attention_backward_dq_rows(q, k, v, do, causal, 0.4, 1, 3, rows)
+        np.testing.assert_allclose(got, dq[1, 3, rows], atol=1e-14)
+
+
 def test_backward_group_subset():
     q = rnd((2, 4, 10, 4), 43)
     k = rnd((2, 2, 10, 4), 44)
