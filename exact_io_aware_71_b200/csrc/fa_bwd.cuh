@@ -15,7 +15,7 @@
 //                   diagonal:
 //                     S^T  = K_j Q_i^T           (TMEM, lanes = keys)
 //                     P^T  = exp2(S^T * scale*log2e - LSE_i*log2e)
-//                     dV_j += P^T dO_i           (P^T read from TMEM)
+//                     dV_j += P^T dO_i           (P^T read from TMEM as bf16 hi + lo)
 //                     dP^T = V_j dO_i^T
 //                     dS^T = P^T o (dP^T - D_i)
 //                     dK_j += dS^T Q_i           (dS^T read from TMEM)
@@ -315,11 +315,14 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
         if (!(ok = mbar_wait(bar_p, t & 1, abort_flag, p.status, WB_P))) break;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < BR / 16; ++kk) {
-          const uint32_t bo = (dcol0 / 64) * BR * 128 + kk * 2048;
-          umma_ts(tmem + C::TM_DV, tmem + C::TM_S + kk * 8, sdesc_sw128(adO + bo, BR * 128, 1024),
-                  ID_KV, (t > 0 || kk > 0) ? 1u : 0u);
-        }
+        for (int half = 0; half < 2; ++half)
+#pragma unroll
+          for (int kk = 0; kk < BR / 16; ++kk) {
+            const uint32_t bo = (dcol0 / 64) * BR * 128 + kk * 2048;
+            umma_ts(tmem + C::TM_DV, tmem + C::TM_S + half * (BR / 2) + kk * 8,
+                    sdesc_sw128(adO + bo, BR * 128, 1024), ID_KV,
+                    (t > 0 || kk > 0 || half > 0) ? 1u : 0u);
+          }
         // dK += dS^T Q
         if (!(ok = mbar_wait(bar_ds, t & 1, abort_flag, p.status, WB_DS))) break;
         tc_fence_after();
@@ -371,27 +374,37 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
            mbar_wait(bar_s, t & 1, abort_flag, p.status, WB_S);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
+      // P^T for this key row, kept in registers for dS.  It goes back to TMEM
+      // (over S^T) as two bf16 halves, hi = bf16(P) in columns [0, BR/2) and
+      // lo = bf16(P - hi) in [BR/2, BR): dV accumulates P_hi^T dO + P_lo^T dO,
+      // so the rounding of P to bf16 does not pile up across the many query
+      // rows (and query heads of a GQA group) that feed one dV row.
       float P[BR];
 #pragma unroll
       for (int c = 0; c < BR / 32; ++c) {
         uint32_t u[32];
         FA_TMEM_LD32(tl + C::TM_S + c * 32, u);
         tmem_wait_ld();
-        uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
+        for (int i = 0; i < 32; ++i) {
           const int cc = c * 32 + i;
-          float p0 = ex2(fmaf(__uint_as_float(u[i]), sl2, -sl[cc]));
-          float p1 = ex2(fmaf(__uint_as_float(u[i + 1]), sl2, -sl[cc + 1]));
-          if (need_mask) {
-            if (cc < cstart) p0 = 0.f;
-            if (cc + 1 < cstart) p1 = 0.f;
-          }
-          P[cc] = p0;
-          P[cc + 1] = p1;
-          pk[i / 2] = pack_bf16(p0, p1);
+          float pv = ex2(fmaf(__uint_as_float(u[i]), sl2, -sl[cc]));
+          if (need_mask && cc < cstart) pv = 0.f;
+          P[cc] = pv;
         }
-        FA_TMEM_ST16(tl + C::TM_S + c * 16, pk);
+      }
+#pragma unroll
+      for (int c = 0; c < BR / 32; ++c) {
+        uint32_t hi[16], lo[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = P[c * 32 + 2 * i], p1 = P[c * 32 + 2 * i + 1];
+          const uint32_t h = pack_bf16(p0, p1);
+          hi[i] = h;
+          lo[i] = pack_bf16(p0 - __uint_as_float(h << 16), p1 - __uint_as_float(h & 0xFFFF0000u));
+        }
+        FA_TMEM_ST16(tl + C::TM_S + c * 16, hi);
+        FA_TMEM_ST16(tl + C::TM_S + BR / 2 + c * 16, lo);
       }
       tmem_wait_st();
       tc_fence_before();

