@@ -19,11 +19,14 @@ LIB_PATH = os.path.join(HERE, "libfa.so")
 FA_OK = 0
 STATUS_NAMES = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED",
                 3: "FA_ERR_MISALIGNED", 4: "FA_ERR_WORKSPACE", 5: "FA_ERR_CUDA",
-                6: "FA_ERR_DEVICE_TIMEOUT"}
+                6: "FA_ERR_DEVICE_TIMEOUT", 7: "FA_ERR_TOO_LARGE"}
 
 # Exported symbols declared in include/fa.h.
 SYMBOLS = ("fa_fwd", "fa_bwd", "fa_bwd_stage", "fa_bwd_workspace_size", "fa_status_string",
-           "fa_device_status")
+           "fa_device_status", "fa_bwd_noalloc")
+
+# Bytes of the built-in scratch behind fa_bwd_noalloc (FA_NOALLOC_SCRATCH_BYTES).
+NOALLOC_SCRATCH_BYTES = 64 << 20
 
 FA_BWD_ALL, FA_BWD_PRE, FA_BWD_MAIN, FA_BWD_DQ = 0, 1, 2, 3
 
@@ -53,6 +56,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fa_bwd.restype = i
     lib.fa_bwd_stage.argtypes = [i] + lib.fa_bwd.argtypes
     lib.fa_bwd_stage.restype = i
+    lib.fa_bwd_noalloc.argtypes = lib.fa_bwd.argtypes[:17] + [vp]
+    lib.fa_bwd_noalloc.restype = i
     lib.fa_bwd_workspace_size.argtypes = [i, i, i, i, i, i, i]
     lib.fa_bwd_workspace_size.restype = sz
     lib.fa_status_string.argtypes = [i]
@@ -79,6 +84,14 @@ def fa_bwd_stage(stage, q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, 
                  workspace, workspace_bytes, stream) -> int:
     return load().fa_bwd_stage(stage, q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d,
                                int(causal), float(scale), workspace, workspace_bytes, stream)
+
+
+def fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, causal, scale,
+                   stream) -> int:
+    """fa_bwd without a caller workspace: scratch is the library's built-in
+    device array (for callers that cannot allocate device memory)."""
+    return load().fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d,
+                                 int(causal), float(scale), stream)
 
 
 def fa_bwd_workspace_size(B, Hq, Hkv, Nq, Nk, d, causal) -> int:

@@ -82,6 +82,25 @@ bool fa::make_map_bf16(CUtensorMap* m, const void* base, int d, int rows, int64_
 
 namespace {
 
+// Scratch of fa_bwd_noalloc (see fa.h).  In host code this name is only a
+// host-side stand-in for the array; its device address comes from
+// cudaGetSymbolAddress, looked up once per device with that device current.
+__device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
+
+void* noalloc_scratch() {
+  static std::mutex mu;
+  static void* addr[128] = {};
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    addr[dev] = p;
+  }
+  return addr[dev];
+}
+
 DevStatus* status_ptr() {
   void* p = nullptr;
   if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
@@ -115,6 +134,7 @@ const char* fa_status_string(int s) {
     case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE";
     case FA_ERR_CUDA: return "FA_ERR_CUDA";
     case FA_ERR_DEVICE_TIMEOUT: return "FA_ERR_DEVICE_TIMEOUT";
+    case FA_ERR_TOO_LARGE: return "FA_ERR_TOO_LARGE";
     default: return "FA_ERR_UNKNOWN";
   }
 }
@@ -191,6 +211,20 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
            cudaStream_t stream) {
   return fa_bwd_stage(FA_BWD_ALL, q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, causal,
                       scale, workspace, workspace_bytes, stream);
+}
+
+int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                   const void* dO, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq,
+                   int Nk, int d, int causal, float scale, cudaStream_t stream) {
+  if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  int st = check_sizes(B, Hq, Hkv, Nq, Nk, d, causal, scale);
+  if (st != FA_OK) return st;
+  if (bwd_workspace_bytes(B, Hq, Hkv, Nq, Nk, d) > FA_NOALLOC_SCRATCH_BYTES)
+    return FA_ERR_TOO_LARGE;
+  void* scratch = noalloc_scratch();
+  if (!scratch) return FA_ERR_CUDA;
+  return fa_bwd_stage(FA_BWD_ALL, q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, causal,
+                      scale, scratch, FA_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 int fa_device_status(cudaStream_t stream, int* where) {

@@ -50,7 +50,8 @@ typedef enum {
   FA_ERR_MISALIGNED = 3,     /* a pointer breaks the alignment rule above */
   FA_ERR_WORKSPACE = 4,      /* workspace null or smaller than fa_bwd_workspace_size() */
   FA_ERR_CUDA = 5,           /* a CUDA runtime/driver call or launch failed */
-  FA_ERR_DEVICE_TIMEOUT = 6  /* a kernel gave up on a pipeline wait (see fa_device_status) */
+  FA_ERR_DEVICE_TIMEOUT = 6, /* a kernel gave up on a pipeline wait (see fa_device_status) */
+  FA_ERR_TOO_LARGE = 7       /* fa_bwd_noalloc: the problem needs more than its built-in scratch */
 } fa_status;
 
 /*
@@ -102,6 +103,37 @@ int fa_bwd_stage(int stage, const void* q, const void* k, const void* v, const v
                  const float* lse, const void* dO, void* dq, void* dk, void* dv, int B, int Hq,
                  int Hkv, int Nq, int Nk, int d, int causal, float scale, void* workspace,
                  size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Size of the scratch area built into the library for fa_bwd_noalloc: a
+ * file-scope device array of this many bytes, which every GPU that loads the
+ * library holds until the process exits.
+ */
+#define FA_NOALLOC_SCRATCH_BYTES (64ull << 20)
+
+/*
+ * Backward pass for callers that cannot allocate device memory.  The pages
+ * have no counterpart to this entry point; it exists for callers that may
+ * not call cudaMalloc themselves, for instance a plug-in inside a host
+ * application that owns every device allocation, or code on a
+ * latency-critical path where cudaMalloc (which may synchronise the device)
+ * is not acceptable.  Same arguments and results as fa_bwd without the
+ * workspace: its scratch (the fp32 dQ accumulator and the two fp32 row
+ * vectors) lives in the library's built-in array of FA_NOALLOC_SCRATCH_BYTES
+ * instead.  The call allocates nothing and calls no allocating routine.
+ *  - Problems whose fa_bwd_workspace_size() exceeds FA_NOALLOC_SCRATCH_BYTES
+ *    are rejected with FA_ERR_TOO_LARGE before anything is launched.
+ *  - The first call on a device looks up the array's device address (with
+ *    that device current) and caches it; make that first call before any
+ *    stream capture.
+ *  - Every call shares the one array per device, and it keeps the last
+ *    call's contents; the call re-initialises every part it reads.  Calls
+ *    whose kernels overlap on the GPU (e.g. on two streams, or from two host
+ *    threads) race on the array: serialise them.
+ */
+int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                   const void* dO, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq,
+                   int Nk, int d, int causal, float scale, cudaStream_t stream);
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* fa_status_string(int status);
