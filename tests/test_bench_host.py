@@ -1,0 +1,85 @@
+"""Host logic of bench.py on the CPU: whole-job aggregation over ranks
+(gloo, world size 2), clock-sample parsing, and the traffic record gate."""
+import json
+import os
+import socket
+
+import pytest
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, times, out):
+    import torch
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        def reduce_max(x):
+            t = torch.tensor([x], dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            return float(t.item())
+        t, rate = bench.aggregate(times[rank], 1e12, world, reduce_max)
+        out[rank] = (t, rate)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_aggregate_takes_the_slowest_rank_over_gloo():
+    times = [100.0, 250.0]
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_worker, args=(2, _free_port(), times, out), nprocs=2, join=True)
+        res = dict(out)
+    for r in (0, 1):
+        t, rate = res[r]
+        assert t == 250.0
+        assert rate == pytest.approx(2 * 1e12 / 0.25)
+
+
+def test_aggregate_single_rank():
+    t, rate = bench.aggregate(50.0, 3e12, 1)
+    assert t == 50.0 and rate == pytest.approx(6e13)
+
+
+def test_parse_clock_samples():
+    text = ("0, 1965, 1965, 400.1, 0x0, Not Active, Not Active, Not Active, Not Active\n"
+            "0, 1800, 1965, 990.0, 0x4, Not Active, Not Active, Not Active, Active\n"
+            "0, 1965, 1965, 500.0, 0x0, Not Active, Not Active, Not Active, Not Active\n")
+    c = bench.parse_clock_samples(text)
+    assert c["sm_mhz"] == 1965 and c["sm_max_mhz"] == 1965
+    assert c["reasons"] == ["sw_power_cap"] and c["samples"] == 3
+    assert bench.parse_clock_samples("")["sm_mhz"] is None
+
+
+def test_traffic_is_reported_only_for_current_sources(tmp_path, monkeypatch):
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    for rel in bench.KERNEL_SOURCES:
+        p = tmp_path / rel
+        p.parent.mkdir(parents=True, exist_ok=True)
+        p.write_text("kernel " + rel)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    sha = bench.kernel_source_hash()
+    rec = {"entries": [{"kernel": "k", "workload": "w", "src_sha": sha,
+                        "dram_bytes_per_launch": 123}]}
+    (prof / "traffic.json").write_text(json.dumps(rec))
+    assert bench.recorded_traffic("k", "w") == 123
+    assert bench.recorded_traffic("k", "other") is None
+    (tmp_path / bench.KERNEL_SOURCES[0]).write_text("changed")
+    assert bench.recorded_traffic("k", "w") is None
+
+
+def test_peaks_fallback(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    pk, src = bench.load_peaks()
+    assert src == "fallback" and pk["bf16_tflops"] == 1590.0
