@@ -108,17 +108,42 @@ DevStatus* status_ptr() {
 }
 
 // ---------------------------------------------------------------- forward
-template <int D, bool CAUSAL>
-int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-               const CUtensorMap& mo, const FwdParams& p, cudaStream_t stream) {
-  using C = FwdCfg<D>;
-  auto kern = fa_fwd_kernel<D, CAUSAL>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+template <class KernelT>
+int launch_kernel(KernelT kern, int smem, int threads, unsigned grid, const CUtensorMap& mq,
+                  const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
+                  const FwdParams& p, cudaStream_t stream) {
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
     return FA_ERR_CUDA;
-  const unsigned grid = unsigned(p.n_qblocks) * unsigned(p.B * p.Hq);
-  kern<<<grid, C::NTHREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
+  kern<<<grid, threads, smem, stream>>>(mq, mk, mv, mo, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// d = 64 / 128: two query tiles per CTA; d = 256: one.
+template <int D, bool CAUSAL>
+int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+               const CUtensorMap& mo, FwdParams p, cudaStream_t stream) {
+  if constexpr (D == 256) {
+    using C = FwdCfg<D>;
+    p.n_units = p.n_qblocks;
+    return launch_kernel(fa_fwd_kernel<D, CAUSAL>, C::SMEM_BYTES, C::NTHREADS,
+                         unsigned(p.n_units) * unsigned(p.B * p.Hq), mq, mk, mv, mo, p, stream);
+  } else {
+    using C = FwdPairCfg<D>;
+    // The warpgroups' register split must fit in what the block is launched
+    // with, or the setmaxnreg.inc would wait forever: refuse to launch.
+    static int regs = -1;
+    if (regs < 0) {
+      cudaFuncAttributes fattr;
+      if (cudaFuncGetAttributes(&fattr, fa_fwd_pair_kernel<D, CAUSAL>) != cudaSuccess)
+        return FA_ERR_CUDA;
+      regs = fattr.numRegs;
+    }
+    if (regs * C::NTHREADS < C::REGS_NEEDED) return FA_ERR_UNSUPPORTED;
+    p.n_units = (p.n_qblocks + 1) / 2;
+    return launch_kernel(fa_fwd_pair_kernel<D, CAUSAL>, C::SMEM_BYTES, C::NTHREADS,
+                         unsigned(p.n_units) * unsigned(p.B * p.Hq), mq, mk, mv, mo, p, stream);
+  }
 }
 
 }  // namespace

@@ -1,35 +1,458 @@
 // Forward pass of exact tiled attention on sm_100a.
 //
-// One CTA computes one tile: 128 query rows of one (batch, query head).
-// Warp roles (192 threads):
-//   warps 0-3  softmax: thread t owns query row t of the tile, reads its row of
-//              S from TMEM, keeps the running max m and running sum l, writes
-//              P (bf16) back into TMEM, rescales O lazily, and finally writes
-//              O / l and the log-sum-exp;
-//   warp 4     TMA producer: Q once, then K_j / V_j through an NS-slot ring;
-//   warp 5     MMA issuer (one thread) and TMEM owner.
-// Per key block j the tensor cores compute S_j = Q K_j^T into one of two TMEM
-// S buffers and O += P_j V_j with P_j read straight from TMEM, so softmax on
-// block j overlaps S_{j+1} and P_{j-1} V_{j-1}.  The score matrix stays on
-// chip; only O and the log-sum-exp reach HBM (QbitAI FA2 article, section
-// "具体实现"; FA1 article, section "FlashAttention").  The online softmax
-// keeps a running max and sum and defers the division by l to the end
-// (FA2 article, section "具体实现", first improvement: fewer rescaling
-// operations without changing the output); O is rescaled only when a row's
-// max grows by more than 2^8, which is exact because O and l always carry the
-// same (possibly stale) max.  Causal key blocks wholly above the diagonal
-// are never loaded or computed (FA2 post, section "Алгоритм вычисления").
+// The score matrix stays on chip: only O and the log-sum-exp reach HBM
+// (QbitAI FA2 article, section "具体实现"; FA1 article, section
+// "FlashAttention").  Per key block j the tensor cores compute S_j = Q K_j^T
+// into TMEM and O += P_j V_j with P_j read straight from TMEM.  The online
+// softmax keeps a running max and sum and defers the division by the sum to
+// the end (FA2 article, section "具体实现", first improvement: fewer
+// rescaling operations without changing the output); O is rescaled only when
+// a row's max grows by more than 2^8, which is exact because O and the sums
+// always carry the same (possibly stale) max.  Causal key blocks wholly above
+// the diagonal are never loaded or computed (FA2 post, section "Алгоритм
+// вычисления").  Forward rows are independent (FA2 post, section
+// "Параллелизм"), so the grid runs over (batch, head, query tile).
+//
+// Thread t of a softmax warpgroup owns query row t of its tile (TMEM lane t):
+// the row max and sums never leave the thread.
+//
+// Two kernels:
+//  * fa_fwd_pair_kernel (d = 64, 128): a CTA owns two 128-row query tiles of
+//    one head and streams K/V once for both.  Warps 0-3 and 4-7 are the two
+//    tiles' softmax warpgroups; in the third warpgroup warp 8 is the TMA
+//    producer, warp 9 the MMA issuer (10, 11 idle).  TMEM holds S and O of
+//    each tile (2 x (128 + d) columns); while one warpgroup exponentiates its
+//    S, the tensor pipe works on the other tile, and two softmax warps share
+//    each SM sub-partition.  The softmax warpgroups take 216 registers per
+//    thread from the third warpgroup's share (setmaxnreg).
+//  * fa_fwd_kernel (d = 256): one 128-row tile per CTA with two S buffers
+//    (O alone takes 256 TMEM columns), warps 0-3 softmax, 4 producer, 5 MMA.
 #pragma once
 #include "sm100.cuh"
 
-// A row's O and l are rescaled only when its running max (log2 units) grows
-// by more than this; in between, probabilities reach at most 2^threshold.
+// A row's O and sums are rescaled only when its running max (log2 units)
+// grows by more than this; in between, probabilities reach at most 2^threshold.
 #ifndef FA_RESCALE_LOG2_THRESHOLD
 #define FA_RESCALE_LOG2_THRESHOLD 8.0f
 #endif
 
 namespace fa {
 
+struct FwdParams {
+  int B, Hq, Hkv, Nq, Nk;
+  int group;          // Hq / Hkv
+  int n_qblocks;      // ceil(Nq / 128)
+  int n_units;        // query units per head: tiles (one-tile kernel) or tile pairs
+  int causal;
+  float scale_log2;   // scale * log2(e)
+  float* lse;         // [B, Hq, Nq]
+  DevStatus* status;
+};
+
+// Wait codes recorded on a timeout.
+enum : unsigned { W_Q = 1, W_KV_EMPTY, W_KV_FULL, W_S_FULL, W_P_FULL, W_O_DONE, W_DRAIN };
+
+// ------------------------------------------------------------------ softmax
+// Running state of one query row, held by the thread that owns the row.
+// l: fp32 sum of the probabilities (for the log-sum-exp); lr: the same
+// probabilities after rounding to bf16, i.e. the weights that actually
+// multiply V, so that O = sum(p~ v) / sum(p~) stays a convex combination
+// even when one key dominates a row.
+struct RowState {
+  float m, l, lr;
+};
+
+// One key block of the online softmax for this thread's row.
+//   tS     TMEM address (this warp's lanes) of the block's BC fp32 scores;
+//          P is written back over them as packed bf16 (BC/2 columns)
+//   tO     the row's O accumulator (D fp32 columns)
+//   j      block index within the tile's sequence; key0 = j * BC
+//   q_tile first query row of the tile, grow this thread's query row
+//   o_done the two barriers that complete after P V of even / odd blocks
+// The caller has waited for S; the function waits for P_{j-1} V_{j-1} only
+// if it has to rescale O.  Returns false if that wait gave up.
+template <int BC, int D, bool CAUSAL>
+__device__ __forceinline__ bool softmax_block(RowState& st, uint32_t tS, uint32_t tO, int j,
+                                              int q_tile, int grow, int Nk, float sl2,
+                                              uint64_t* o_done, volatile int* abort,
+                                              DevStatus* status) {
+  float s[BC];
+  {
+    uint32_t* r = reinterpret_cast<uint32_t*>(s);
+#pragma unroll
+    for (int c = 0; c < BC / 32; ++c) FA_TMEM_LD32(tS + c * 32, (r + c * 32));
+    tmem_wait_ld();
+  }
+  const int key0 = j * BC;
+  if ((key0 + BC > Nk) || (CAUSAL && key0 + BC - 1 > q_tile)) {
+    const int lim = CAUSAL ? min(Nk - key0, grow - key0 + 1) : (Nk - key0);
+#pragma unroll
+    for (int c = 0; c < BC; ++c)
+      if (c >= lim) s[c] = -INFINITY;
+  }
+  // Row max as four independent three-input max chains.
+  float mx;
+  {
+    float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+    for (int c = 0; c < BC; c += 8) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) m4[q] = fmax3(m4[q], s[c + 2 * q], s[c + 2 * q + 1]);
+    }
+    mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+  }
+  const float mc = mx * sl2;
+  if (j == 0) {
+    st.m = mc;
+  } else {
+    const bool need = mc > st.m + FA_RESCALE_LOG2_THRESHOLD;
+    if (__any_sync(0xffffffffu, need)) {
+      const float mn = need ? mc : st.m;
+      const float alpha = ex2(st.m - mn);
+      // O must hold every block up to j-1 before it is rescaled.  The
+      // barriers alternate by block parity: warps of a warpgroup may be one
+      // block apart, and one barrier would let a warp at block j+1 take
+      // P_{j-1}V_{j-1}'s completion (same parity) for P_j V_j's.
+      bool ok = mbar_wait(o_done + ((j - 1) & 1), ((j - 1) >> 1) & 1, abort, status, W_O_DONE);
+      if (!__all_sync(0xffffffffu, ok)) return false;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        FA_TMEM_LD32(tO + c * 32, r);
+        tmem_wait_ld();
+        float2* r2 = reinterpret_cast<float2*>(r);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) r2[i] = fmul2(r2[i], make_float2(alpha, alpha));
+        FA_TMEM_ST32(tO + c * 32, r);
+      }
+      tmem_wait_st();
+      st.l *= alpha;
+      st.lr *= alpha;
+      st.m = mn;
+    }
+  }
+  const float neg = (st.m == -INFINITY) ? 0.f : -st.m;
+  // p = 2^(s*scale*log2e - m): packed FMA, MUFU ex2, both sums in four packed
+  // accumulator pairs; P is stored to TMEM 32 columns at a time.
+  float2 al[4], ar[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) al[q] = ar[q] = make_float2(0.f, 0.f);
+  const float2 sl22 = make_float2(sl2, sl2), neg2 = make_float2(neg, neg);
+#pragma unroll
+  for (int c = 0; c < BC / 32; ++c) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int e = c * 32 + 2 * i;
+      const float2 t = ffma2(make_float2(s[e], s[e + 1]), sl22, neg2);
+      const float2 pp = make_float2(ex2(t.x), ex2(t.y));
+      al[i & 3] = fadd2(al[i & 3], pp);
+      const uint32_t pr = pack_bf16(pp.x, pp.y);
+      ar[i & 3] = fadd2(ar[i & 3], make_float2(__uint_as_float(pr << 16),
+                                               __uint_as_float(pr & 0xFFFF0000u)));
+      pk[i] = pr;
+    }
+    FA_TMEM_ST16(tS + c * 16, pk);
+  }
+  const float2 la = fadd2(fadd2(al[0], al[1]), fadd2(al[2], al[3]));
+  const float2 lb = fadd2(fadd2(ar[0], ar[1]), fadd2(ar[2], ar[3]));
+  st.l += la.x + la.y;
+  st.lr += lb.x + lb.y;
+  tmem_wait_st();
+  tc_fence_before();
+  return true;
+}
+
+// After the tile's last P V: O / lr to bf16, staged in `stage` (the tile's
+// free Q buffer) in the 128-byte swizzled layout, one 4 KiB box per warp and
+// 64 columns, TMA-stored by lane 0 of each warp; then the log-sum-exp.
+template <int D>
+__device__ __forceinline__ void softmax_finish(const RowState& st, uint32_t tO, uint8_t* stage,
+                                               int w, int lane, const CUtensorMap* tmO,
+                                               int q_tile, int Nq, int bh, float* lse,
+                                               int grow) {
+  const float inv = 1.0f / st.lr;
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t r[32];
+    FA_TMEM_LD32(tO + c * 32, r);
+    tmem_wait_ld();
+    uint32_t pk2[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      pk2[i] = pack_bf16(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
+    uint8_t* box = stage + ((c >> 1) * 4 + w) * 4096 + lane * 128;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int unit = (c & 1) * 4 + u;
+      *reinterpret_cast<uint4*>(box + ((unit ^ (lane & 7)) * 16)) =
+          make_uint4(pk2[4 * u], pk2[4 * u + 1], pk2[4 * u + 2], pk2[4 * u + 3]);
+    }
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0 && q_tile + w * 32 < Nq) {
+    for (int c = 0; c < D / 64; ++c)
+      tma_store_3d(tmO, stage + (c * 4 + w) * 4096, c * 64, q_tile + w * 32, bh);
+    bulk_commit();
+    bulk_wait0();
+  }
+  if (grow < Nq) lse[size_t(bh) * Nq + grow] = (st.m + __log2f(st.l)) * 0.69314718055994531f;
+}
+
+// ------------------------------------------------------------------ tile pairs (d = 64, 128)
+template <int D>
+struct FwdPairCfg {
+  static constexpr int BR = 128;                    // query rows per tile (two tiles per CTA)
+  static constexpr int BC = 128;                    // keys per block
+  static constexpr int KCH = D / 64;                // 128-byte chunks along d
+  static constexpr int Q_BYTES = BR * D * 2;        // one tile
+  static constexpr int KV_BYTES = BC * D * 2;
+  static constexpr int NS = (D == 64) ? 8 : 5;      // K/V ring slots
+  static constexpr int TM_TILE = 256;               // tile t: S at t*256, O at t*256 + 128
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int NTHREADS = 384;
+  static constexpr int REGS_SOFTMAX = 216;          // per thread, warpgroups 0 and 1
+  static constexpr int REGS_OTHER = 72;             // per thread, warpgroup 2
+  static constexpr int REGS_NEEDED = 256 * REGS_SOFTMAX + 128 * REGS_OTHER;
+  static constexpr int SMEM_BYTES = 2 * Q_BYTES + NS * KV_BYTES + 1024 + 1024;
+  static_assert(128 + D <= TM_TILE, "TMEM budget");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+};
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
+    fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
+                       const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV,
+                       const __grid_constant__ CUtensorMap tmO, const FwdParams p) {
+  using C = FwdPairCfg<D>;
+  constexpr int BR = C::BR, BC = C::BC, NS = C::NS;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sQ = smem;                          // 2 tiles of [KCH][BR][128B]; O staging later
+  uint8_t* sKV = smem + 2 * C::Q_BYTES;        // NS slots of [KCH][BC][128B]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + NS * C::KV_BYTES);
+  uint64_t* bar_q = bars + 0;                  // [2]
+  uint64_t* bar_kv_full = bars + 2;            // [NS]
+  uint64_t* bar_kv_empty = bars + 2 + NS;      // [NS]
+  uint64_t* bar_s_full = bars + 2 + 2 * NS;    // [2] per tile
+  uint64_t* bar_p_full = bars + 4 + 2 * NS;    // [2] per tile
+  uint64_t* bar_o_done = bars + 6 + 2 * NS;    // [2 tiles][2 parities]
+  uint64_t* bar_drain = bars + 10 + 2 * NS;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 12 + 2 * NS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // Unit = (batch, head, tile pair).  Consecutive CTAs share a head so that
+  // its K/V stay hot in L2; causal pairs run longest first within a head.
+  const int bh = blockIdx.x / p.n_units;
+  int pu = blockIdx.x - bh * p.n_units;
+  if (CAUSAL) pu = p.n_units - 1 - pu;
+  const int b = bh / p.Hq;
+  const int h = bh - b * p.Hq;
+  const int bkv = b * p.Hkv + h / p.group;
+  const int q0 = pu * 2 * BR;
+  int nt[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int qt = q0 + t * BR;
+    const int kv_end = CAUSAL ? min(p.Nk, qt + BR) : p.Nk;
+    nt[t] = (qt < p.Nq) ? (kv_end + BC - 1) / BC : 0;   // tile 1 may lie past Nq
+  }
+  const int nmax = max(nt[0], nt[1]);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_q + i, 1);
+      mbar_init(bar_s_full + i, 1);
+      mbar_init(bar_p_full + i, BR);
+    }
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(bar_kv_full + i, 1);
+      mbar_init(bar_kv_empty + i, 1);
+    }
+    for (int i = 0; i < 4; ++i) mbar_init(bar_o_done + i, 1);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_holder, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp >= 8) {
+    regs_dec<C::REGS_OTHER>();
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      for (int t = 0; t < 2; ++t) {
+        if (nt[t] == 0) continue;
+        mbar_arrive_expect_tx(bar_q + t, C::Q_BYTES);
+        for (int c = 0; c < C::KCH; ++c)
+          tma_load_3d(sQ + t * C::Q_BYTES + c * BR * 128, &tmQ, bar_q + t, c * 64, q0 + t * BR,
+                      bh);
+      }
+      // Ring order = MMA consumption order: K0, V0, K1, V1, ...
+      int cnt = 0;
+      bool ok = true;
+      for (int j = 0; j < nmax && ok; ++j) {
+        for (int kv = 0; kv < 2 && ok; ++kv) {
+          const int slot = cnt % NS;
+          if (!mbar_wait(bar_kv_empty + slot, ((cnt / NS) & 1) ^ 1, abort_flag, p.status,
+                         W_KV_EMPTY)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar_kv_full + slot, C::KV_BYTES);
+          uint8_t* dst = sKV + slot * C::KV_BYTES;
+          const CUtensorMap* tm = kv == 0 ? &tmK : &tmV;
+          for (int c = 0; c < C::KCH; ++c)
+            tma_load_3d(dst + c * BC * 128, tm, bar_kv_full + slot, c * 64, j * BC, bkv);
+          ++cnt;
+        }
+      }
+      if (!ok) {
+        for (int i = cnt - 1; i >= 0 && i >= cnt - NS; --i) {
+          volatile int no_abort = 0;
+          mbar_wait(bar_kv_full + (i % NS), (i / NS) & 1, &no_abort, nullptr, W_DRAIN);
+        }
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(BR, BC, 0, 0);
+      constexpr uint32_t IDESC_O = idesc_bf16_f32(BR, D, 0, 1);
+      const uint32_t sQ_addr = smem_u32(sQ);
+      const uint32_t sKV_addr = smem_u32(sKV);
+      int cnt = 0;
+      bool ok = true;
+      auto acquire = [&](int& slot) -> bool {
+        slot = cnt % NS;
+        if (!mbar_wait(bar_kv_full + slot, (cnt / NS) & 1, abort_flag, p.status, W_KV_FULL))
+          return false;
+        tc_fence_after();
+        ++cnt;
+        return true;
+      };
+      auto mma_s = [&](int t, int slot) {
+        const uint32_t qbase = sQ_addr + t * C::Q_BYTES;
+        const uint32_t kbase = sKV_addr + slot * C::KV_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t a = sdesc_sw128(qbase + (kk >> 2) * BR * 128 + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(kbase + (kk >> 2) * BC * 128 + (kk & 3) * 32, 16, 1024);
+          umma_ss(tmem + t * C::TM_TILE, a, bd, IDESC_S, kk > 0);
+        }
+        umma_commit(bar_s_full + t);
+      };
+      auto mma_pv = [&](int t, int j, int slot) -> bool {
+        if (!mbar_wait(bar_p_full + t, j & 1, abort_flag, p.status, W_P_FULL)) return false;
+        tc_fence_after();
+        const uint32_t vbase = sKV_addr + slot * C::KV_BYTES;
+        const uint32_t tt = tmem + t * C::TM_TILE;
+#pragma unroll
+        for (int kk = 0; kk < BC / 16; ++kk) {
+          const uint64_t bd = sdesc_sw128(vbase + kk * 16 * 128, BC * 128, 1024);
+          umma_ts(tt + 128, tt + kk * 8, bd, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(bar_o_done + t * 2 + (j & 1));
+        return true;
+      };
+      int sK = 0, sV = 0;
+      ok = acquire(sK);
+      if (ok) ok = mbar_wait(bar_q + 0, 0, abort_flag, p.status, W_Q);
+      if (ok) {
+        tc_fence_after();
+        mma_s(0, sK);
+        if (nt[1] > 0) {
+          ok = mbar_wait(bar_q + 1, 0, abort_flag, p.status, W_Q);
+          if (ok) {
+            tc_fence_after();
+            mma_s(1, sK);
+          }
+        }
+        umma_commit(bar_kv_empty + sK);
+      }
+      // Per block j: P0 V_j, then S0_{j+1} (it overwrites P0_j in TMEM, so it
+      // must follow P0_j V_j; tcgen05 MMAs run in issue order), then the
+      // same for tile 1.  Each K/V slot is released after its last reader.
+      for (int j = 0; j < nmax && ok; ++j) {
+        if (!(ok = acquire(sV))) break;
+        if (j < nt[0] && !(ok = mma_pv(0, j, sV))) break;
+        const bool next = j + 1 < nmax;
+        if (next) {
+          if (!(ok = acquire(sK))) break;
+          if (j + 1 < nt[0]) mma_s(0, sK);
+        }
+        if (j < nt[1] && !(ok = mma_pv(1, j, sV))) break;
+        umma_commit(bar_kv_empty + sV);
+        if (next) {
+          if (j + 1 < nt[1]) mma_s(1, sK);
+          umma_commit(bar_kv_empty + sK);
+        }
+      }
+      umma_commit(bar_drain);
+      volatile int no_abort = 0;
+      mbar_wait(bar_drain, 0, &no_abort, nullptr, W_DRAIN);
+    }
+  }
+    // warps 10 and 11 have no role
+  } else {
+    regs_inc<C::REGS_SOFTMAX>();
+    // ------------------------------------------------------------ softmax (tile = warp / 4)
+    const int t = warp >> 2;                        // 0 or 1 (warps 0..7)
+    const int w = warp & 3;                         // TMEM lane quarter
+    const int row = w * 32 + lane;
+    const int q_tile = q0 + t * BR;
+    const int grow = q_tile + row;
+    const uint32_t tl = tmem + t * C::TM_TILE + (uint32_t(w * 32) << 16);
+    uint64_t* o_done = bar_o_done + t * 2;
+    RowState st{-INFINITY, 0.f, 0.f};
+    bool ok = nt[t] > 0;
+    for (int j = 0; j < nt[t] && ok; ++j) {
+      ok = mbar_wait(bar_s_full + t, j & 1, abort_flag, p.status, W_S_FULL);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      tc_fence_after();
+      ok = softmax_block<BC, D, CAUSAL>(st, tl, tl + 128, j, q_tile, grow, p.Nk, p.scale_log2,
+                                        o_done, abort_flag, p.status);
+      if (!ok) break;
+      mbar_arrive(bar_p_full + t);
+    }
+    if (ok) {
+      const int jl = nt[t] - 1;
+      ok = mbar_wait(o_done + (jl & 1), (jl >> 1) & 1, abort_flag, p.status, W_O_DONE);
+      if (__all_sync(0xffffffffu, ok)) {
+        tc_fence_after();
+        softmax_finish<D>(st, tl + 128, sQ + t * C::Q_BYTES, w, lane, &tmO, q_tile, p.Nq, bh,
+                          p.lse, grow);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ one tile (d = 256)
 template <int D>
 struct FwdCfg {
   static constexpr int BR = 128;                       // query rows per tile
@@ -46,19 +469,6 @@ struct FwdCfg {
   static_assert(TM_O + D <= TMEM_COLS, "TMEM budget");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
-
-struct FwdParams {
-  int B, Hq, Hkv, Nq, Nk;
-  int group;          // Hq / Hkv
-  int n_qblocks;      // ceil(Nq / 128)
-  int causal;
-  float scale_log2;   // scale * log2(e)
-  float* lse;         // [B, Hq, Nq]
-  DevStatus* status;
-};
-
-// Wait codes recorded on a timeout.
-enum : unsigned { W_Q = 1, W_KV_EMPTY, W_KV_FULL, W_S_FULL, W_P_FULL, W_O_DONE, W_DRAIN };
 
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
@@ -79,10 +489,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
   uint64_t* bar_kv_empty = bars + 1 + NS;
   uint64_t* bar_s_full = bars + 1 + 2 * NS;      // [2]
   uint64_t* bar_p_full = bars + 3 + 2 * NS;      // [2]
-  // O-done barriers alternate by key-block parity: softmax warps may drift one
-  // block apart, and with a single barrier a warp already at block j+1 could
-  // mistake the completion of P_{j-1} V_{j-1} (same parity) for P_j V_j.
-  uint64_t* bar_o_done = bars + 5 + 2 * NS;      // [2]
+  uint64_t* bar_o_done = bars + 5 + 2 * NS;      // [2] by block parity
   uint64_t* bar_drain = bars + 7 + 2 * NS;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 8 + 2 * NS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
@@ -90,11 +497,9 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // Tile coordinates: consecutive CTAs share a (batch, head) so that its K/V
-  // stay hot in L2; within a head causal tiles run longest first.
-  const int bh = blockIdx.x / p.n_qblocks;
-  int qb = blockIdx.x - bh * p.n_qblocks;
-  if (CAUSAL) qb = p.n_qblocks - 1 - qb;
+  const int bh = blockIdx.x / p.n_units;
+  int qb = blockIdx.x - bh * p.n_units;
+  if (CAUSAL) qb = p.n_units - 1 - qb;
   const int b = bh / p.Hq;
   const int h = bh - b * p.Hq;
   const int bkv = b * p.Hkv + h / p.group;
@@ -111,9 +516,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar_s_full + i, 1);
       mbar_init(bar_p_full + i, BR);
+      mbar_init(bar_o_done + i, 1);
     }
-    mbar_init(bar_o_done + 0, 1);
-    mbar_init(bar_o_done + 1, 1);
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -151,6 +555,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
           tma_load_3d(dst + c * BC * 128, tm, bar_kv_full + slot, c * 64, j * BC, bkv);
         ++cnt;
       };
+      // Ring order = MMA consumption order: K0, K1, V0, K2, V1, ...
       load(&tmK, 0);
       for (int j = 1; j < n_blocks && ok; ++j) {
         load(&tmK, j);
@@ -218,6 +623,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
         umma_commit(bar_o_done + (j & 1));
         release(slot);
       };
+      // S_{j+1} is issued before P_j V_j so that softmax on block j+1 can
+      // start as soon as P_j is handed over (two S buffers).
       if (ok) mma_s(0);
       for (int j = 1; j < n_blocks && ok; ++j) {
         mma_s(j);
@@ -234,116 +641,25 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
     const int row = threadIdx.x;                       // 0..127 == TMEM lane
     const uint32_t tl = tmem + (uint32_t(warp * 32) << 16);
     const int grow = q_row0 + row;
-    const float sl2 = p.scale_log2;
-    // l: fp32 sum of the probabilities (for the log-sum-exp); lr: sum of the
-    // same probabilities after rounding to bf16, i.e. of the weights that
-    // actually multiply V, so that O = sum(p~ v) / sum(p~) is a convex
-    // combination even when one key dominates a row.
-    float m = -INFINITY, l = 0.f, lr = 0.f;
+    RowState st{-INFINITY, 0.f, 0.f};
     bool ok = true;
-    for (int j = 0; j < n_blocks; ++j) {
+    for (int j = 0; j < n_blocks && ok; ++j) {
       ok = mbar_wait(bar_s_full + (j & 1), (j >> 1) & 1, abort_flag, p.status, W_S_FULL);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
-      float s[BC];
-      {
-        uint32_t* r = reinterpret_cast<uint32_t*>(s);
-#pragma unroll
-        for (int c = 0; c < BC / 32; ++c) FA_TMEM_LD32(tl + C::TM_S + (j & 1) * BC + c * 32, (r + c * 32));
-        tmem_wait_ld();
-      }
-      const int key0 = j * BC;
-      const bool need_mask = (key0 + BC > p.Nk) || (CAUSAL && key0 + BC - 1 > q_row0);
-      if (need_mask) {
-        const int lim = CAUSAL ? min(p.Nk - key0, grow - key0 + 1) : (p.Nk - key0);
-#pragma unroll
-        for (int c = 0; c < BC; ++c)
-          if (c >= lim) s[c] = -INFINITY;
-      }
-      float mx = s[0];
-#pragma unroll
-      for (int c = 1; c < BC; ++c) mx = fmaxf(mx, s[c]);
-      const float mc = mx * sl2;
-      if (j == 0) {
-        m = mc;
-      } else {
-        const bool need = mc > m + FA_RESCALE_LOG2_THRESHOLD;
-        if (__any_sync(0xffffffffu, need)) {
-          const float mn = need ? mc : m;
-          const float alpha = ex2(m - mn);
-          ok = mbar_wait(bar_o_done + ((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag, p.status,
-                         W_O_DONE);
-          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t r[32];
-            FA_TMEM_LD32(tl + C::TM_O + c * 32, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            FA_TMEM_ST32(tl + C::TM_O + c * 32, r);
-          }
-          tmem_wait_st();
-          l *= alpha;
-          lr *= alpha;
-          m = mn;
-        }
-      }
-      const float neg = (m == -INFINITY) ? 0.f : -m;
-      uint32_t pk[BC / 2];
-      float ls = 0.f, lrs = 0.f;
-#pragma unroll
-      for (int c = 0; c < BC; c += 2) {
-        const float p0 = ex2(fmaf(s[c], sl2, neg));
-        const float p1 = ex2(fmaf(s[c + 1], sl2, neg));
-        ls += p0 + p1;
-        const uint32_t pr = pack_bf16(p0, p1);
-        lrs += __uint_as_float(pr << 16) + __uint_as_float(pr & 0xFFFF0000u);
-        pk[c / 2] = pr;
-      }
-      l += ls;
-      lr += lrs;
-#pragma unroll
-      for (int c = 0; c < BC / 64; ++c) FA_TMEM_ST32(tl + C::TM_S + (j & 1) * BC + c * 32, (pk + c * 32));
-      tmem_wait_st();
-      tc_fence_before();
+      ok = softmax_block<BC, D, CAUSAL>(st, tl + C::TM_S + (j & 1) * BC, tl + C::TM_O, j, q_row0,
+                                        grow, p.Nk, p.scale_log2, bar_o_done, abort_flag,
+                                        p.status);
+      if (!ok) break;
       mbar_arrive(bar_p_full + (j & 1));
     }
-    if (ok)
-      ok = mbar_wait(bar_o_done + ((n_blocks - 1) & 1), ((n_blocks - 1) >> 1) & 1, abort_flag,
-                     p.status, W_O_DONE);
-    if (__all_sync(0xffffffffu, ok)) {
-      tc_fence_after();
-      const float inv = 1.0f / lr;
-      // Stage this warp's 32 rows of O (bf16) in the Q buffer in the 128-byte
-      // swizzled layout the TMA store expects, one 4 KiB box per 64 columns.
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t r[32];
-        FA_TMEM_LD32(tl + C::TM_O + c * 32, r);
-        tmem_wait_ld();
-        uint32_t pk2[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pk2[i] = pack_bf16(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
-        uint8_t* box = sQ + ((c >> 1) * 4 + warp) * 4096 + lane * 128;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int unit = (c & 1) * 4 + u;
-          *reinterpret_cast<uint4*>(box + ((unit ^ (lane & 7)) * 16)) =
-              make_uint4(pk2[4 * u], pk2[4 * u + 1], pk2[4 * u + 2], pk2[4 * u + 3]);
-        }
+    if (ok) {
+      const int jl = n_blocks - 1;
+      ok = mbar_wait(bar_o_done + (jl & 1), (jl >> 1) & 1, abort_flag, p.status, W_O_DONE);
+      if (__all_sync(0xffffffffu, ok)) {
+        tc_fence_after();
+        softmax_finish<D>(st, tl + C::TM_O, sQ, warp, lane, &tmO, q_row0, p.Nq, bh, p.lse, grow);
       }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0 && q_row0 + warp * 32 < p.Nq) {
-        for (int c = 0; c < C::KCH; ++c)
-          tma_store_3d(&tmO, sQ + (c * 4 + warp) * 4096, c * 64, q_row0 + warp * 32, bh);
-        bulk_commit();
-        bulk_wait0();
-      }
-      if (grow < p.Nq) p.lse[size_t(bh) * p.Nq + grow] = (m + __log2f(l)) * 0.69314718055994531f;
     }
   }
 
