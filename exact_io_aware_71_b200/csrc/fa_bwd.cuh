@@ -11,8 +11,8 @@
 //                   fp32 rows, and dQacc <- 0            (HBM-bound)
 //   fa_bwd_main     one CTA per (batch, kv head, 128-key block[, d half]):
 //                   K_j, V_j stay in shared memory; for every query head of
-//                   the kv group and every query block i at or below the
-//                   diagonal:
+//                   the kv group and every 64-row query block i at or below
+//                   the diagonal ("step" t):
 //                     S^T  = K_j Q_i^T           (TMEM, lanes = keys)
 //                     P^T  = exp2(S^T * scale*log2e - LSE_i*log2e)
 //                     dV_j += P^T dO_i           (P^T read from TMEM as bf16 hi + lo)
@@ -23,10 +23,17 @@
 //                   then dK_j * scale and dV_j are written as bf16
 //   fa_bwd_dq       dq = bf16(scale * dQacc)              (HBM-bound)
 //
-// TMEM (512 columns): S^T | dP^T | dQ^T | dK | dV; P^T and dS^T overwrite S^T
-// and dP^T in place as packed bf16.  For d = 256 the dK / dV accumulators
-// alone would fill TMEM, so two CTAs share a key block, each owning one
-// 128-wide half of d for dK, dV and dQ (both recompute S and dP).
+// fa_bwd_main roles (384 threads): warpgroups 0 and 1 are compute warps
+// (TMEM lane = key row); warpgroup w owns query columns [32w, 32w+32) of
+// every step, and writes its P^T (hi, lo) and dS^T only over its own S^T /
+// dP^T columns, so neither group can overwrite scores the other has not yet
+// read.  Warp 8 issues the TMA loads, warp 9 the MMAs (10, 11 idle).
+// TMEM (512 columns): S^T x2 | dP^T | dQ^T | dK | dV.  S^T is double-buffered
+// so S^T of step t+1 is computed while step t's dS is formed; per step the
+// MMA order is dV_t, S_{t+1}, dK_t, dQ_t, dP_{t+1}, and the compute warps
+// read out dQ_{t-1} between P_t and dS_t.  For d = 256 the dK / dV
+// accumulators alone would fill TMEM, so two CTAs share a key block, each
+// owning one 128-wide half of d for dK, dV and dQ (both recompute S and dP).
 #pragma once
 #include "sm100.cuh"
 
@@ -35,7 +42,7 @@ namespace fa {
 template <int D>
 struct BwdCfg {
   static constexpr int BC = 128;                        // keys per CTA (TMEM lanes)
-  static constexpr int BR = (D == 64) ? 128 : 64;       // query rows per step
+  static constexpr int BR = 64;                         // query rows per step
   static constexpr int DH = (D == 256) ? 128 : D;       // d columns owned by a CTA
   static constexpr int NSPLIT = D / DH;                 // CTAs per key block
   static constexpr int KCH = D / 64;
@@ -44,10 +51,14 @@ struct BwdCfg {
   static constexpr int QT_BYTES = BR * D * 2;           // one Q or dO tile
   static constexpr int STAGE_BYTES = 2 * QT_BYTES + 2 * BR * 4;
   static constexpr int STAGE_STRIDE = (STAGE_BYTES + 1023) / 1024 * 1024;
-  static constexpr int DS_BYTES = BC * BR * 2;
-  static constexpr int TM_S = 0, TM_DP = BR, TM_DQ = 2 * BR, TM_DK = 3 * BR, TM_DV = 3 * BR + DH;
+  static constexpr int DS_BYTES = BC * BR * 2;          // dS^T: [BC keys][BR queries] bf16
+  static constexpr int TM_S = 0;                        // two S^T buffers of BR columns
+  static constexpr int TM_DP = 2 * BR;
+  static constexpr int TM_DQ = 3 * BR;
+  static constexpr int TM_DK = 4 * BR;
+  static constexpr int TM_DV = 4 * BR + DH;
   static constexpr int TMEM_COLS = 512;
-  static constexpr int NTHREADS = 192;
+  static constexpr int NTHREADS = 384;
   static constexpr int SMEM_BYTES = 2 * K_BYTES + QS * STAGE_STRIDE + DS_BYTES + 1024 + 1024;
   static_assert(TM_DV + DH <= TMEM_COLS, "TMEM budget");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
@@ -181,19 +192,19 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
   uint8_t* sK = smem;                                   // [KCH][BC][128B]
   uint8_t* sV = sK + C::K_BYTES;
   uint8_t* sStage = sV + C::K_BYTES;                    // QS x {Q | dO | L | D}
-  uint8_t* sdS = sStage + QS * C::STAGE_STRIDE;         // [BR/64][BC][128B] dS^T
+  uint8_t* sdS = sStage + QS * C::STAGE_STRIDE;         // [BC][128B] dS^T, 64 queries per row
   uint64_t* bars = reinterpret_cast<uint64_t*>(sdS + C::DS_BYTES);
   uint64_t* bar_kv = bars + 0;
   uint64_t* bar_qfull = bars + 1;                       // [QS]
   uint64_t* bar_qempty = bars + 1 + QS;                 // [QS]
-  uint64_t* bar_s = bars + 1 + 2 * QS;
-  uint64_t* bar_dp = bars + 2 + 2 * QS;
-  uint64_t* bar_p = bars + 3 + 2 * QS;
-  uint64_t* bar_ds = bars + 4 + 2 * QS;
-  uint64_t* bar_dqfull = bars + 5 + 2 * QS;
-  uint64_t* bar_dqempty = bars + 6 + 2 * QS;
-  uint64_t* bar_final = bars + 7 + 2 * QS;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 8 + 2 * QS);
+  uint64_t* bar_s = bars + 1 + 2 * QS;                  // [2] per S^T buffer
+  uint64_t* bar_dp = bars + 3 + 2 * QS;
+  uint64_t* bar_p = bars + 4 + 2 * QS;
+  uint64_t* bar_ds = bars + 5 + 2 * QS;
+  uint64_t* bar_dqfull = bars + 6 + 2 * QS;
+  uint64_t* bar_dqempty = bars + 7 + 2 * QS;
+  uint64_t* bar_final = bars + 8 + 2 * QS;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 9 + 2 * QS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -219,17 +230,18 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
       mbar_init(bar_qfull + i, 1);
       mbar_init(bar_qempty + i, 1);
     }
-    mbar_init(bar_s, 1);
+    mbar_init(bar_s + 0, 1);
+    mbar_init(bar_s + 1, 1);
     mbar_init(bar_dp, 1);
-    mbar_init(bar_p, 128);
-    mbar_init(bar_ds, 128);
+    mbar_init(bar_p, 256);
+    mbar_init(bar_ds, 256);
     mbar_init(bar_dqfull, 1);
-    mbar_init(bar_dqempty, 128);
+    mbar_init(bar_dqempty, 256);
     mbar_init(bar_final, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_holder, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -238,7 +250,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && n_steps > 0) {
       prefetch_tmap(&tmQ);
@@ -277,7 +289,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
         }
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && n_steps > 0) {
       constexpr uint32_t ID_S = idesc_bf16_f32(128, BR, 0, 0);    // S^T, dP^T: K-major both
@@ -285,33 +297,34 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
       constexpr uint32_t ID_DQ = idesc_bf16_f32(128, BR, 1, 1);   // dQ^T: A, B MN-major
       const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aS0 = smem_u32(sStage);
       const uint32_t adS = smem_u32(sdS);
-      bool ok = mbar_wait(bar_kv, 0, abort_flag, p.status, WB_KV);
-      tc_fence_after();
-      for (int t = 0; t < n_steps && ok; ++t) {
-        const int st = t % QS;
-        const uint32_t aQ = aS0 + st * C::STAGE_STRIDE;
-        const uint32_t adO = aQ + C::QT_BYTES;
-        if (!(ok = mbar_wait(bar_qfull + st, (t / QS) & 1, abort_flag, p.status, WB_QFULL)))
-          break;
-        tc_fence_after();
-        // S^T = K Q^T and dP^T = V dO^T  (M = 128 keys, N = BR queries, K = d)
+      // A-operand column (within a P^T / dS^T buffer) of k-step kk: compute
+      // group kk/2 wrote queries [32(kk/2), +32) packed into its own columns.
+      auto pcol = [](int kk) { return uint32_t((kk >> 1) * 32 + (kk & 1) * 8); };
+      auto mma_sdp = [&](uint32_t d_tm, uint32_t a_base, uint32_t b_base) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ko = (kk >> 2) * BC * 128 + (kk & 3) * 32;
           const uint32_t qo = (kk >> 2) * BR * 128 + (kk & 3) * 32;
-          umma_ss(tmem + C::TM_S, sdesc_sw128(aK + ko, 16, 1024), sdesc_sw128(aQ + qo, 16, 1024),
+          umma_ss(d_tm, sdesc_sw128(a_base + ko, 16, 1024), sdesc_sw128(b_base + qo, 16, 1024),
                   ID_S, kk > 0);
         }
-        umma_commit(bar_s);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ko = (kk >> 2) * BC * 128 + (kk & 3) * 32;
-          const uint32_t qo = (kk >> 2) * BR * 128 + (kk & 3) * 32;
-          umma_ss(tmem + C::TM_DP, sdesc_sw128(aV + ko, 16, 1024),
-                  sdesc_sw128(adO + qo, 16, 1024), ID_S, kk > 0);
-        }
+      };
+      auto stage_q = [&](int t) { return aS0 + (t % QS) * C::STAGE_STRIDE; };
+      bool ok = mbar_wait(bar_kv, 0, abort_flag, p.status, WB_KV) &&
+                mbar_wait(bar_qfull + 0, 0, abort_flag, p.status, WB_QFULL);
+      tc_fence_after();
+      if (ok) {
+        mma_sdp(tmem + C::TM_S, aK, stage_q(0));
+        umma_commit(bar_s + 0);
+        mma_sdp(tmem + C::TM_DP, aV, stage_q(0) + C::QT_BYTES);
         umma_commit(bar_dp);
-        // dV += P^T dO  (A = P^T in TMEM, B = dO[:, dcol0:dcol0+DH] MN-major)
+      }
+      for (int t = 0; t < n_steps && ok; ++t) {
+        const int st = t % QS;
+        const uint32_t aQ = stage_q(t);
+        const uint32_t adO = aQ + C::QT_BYTES;
+        const uint32_t tS = tmem + C::TM_S + (t & 1) * BR;
+        // dV += P^T dO  (hi then lo half of P)
         if (!(ok = mbar_wait(bar_p, t & 1, abort_flag, p.status, WB_P))) break;
         tc_fence_after();
 #pragma unroll
@@ -319,23 +332,38 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < BR / 16; ++kk) {
             const uint32_t bo = (dcol0 / 64) * BR * 128 + kk * 2048;
-            umma_ts(tmem + C::TM_DV, tmem + C::TM_S + half * (BR / 2) + kk * 8,
+            umma_ts(tmem + C::TM_DV, tS + pcol(kk) + half * 16,
                     sdesc_sw128(adO + bo, BR * 128, 1024), ID_KV,
                     (t > 0 || kk > 0 || half > 0) ? 1u : 0u);
           }
+        // S^T of the next step into the other buffer.  With one Q/dO stage
+        // the next Q only arrives after this step's dK releases the stage,
+        // so S^T_{t+1} then waits until after dQ_t (below).
+        auto next_s = [&]() -> bool {
+          if (t + 1 >= n_steps) return true;
+          if (!mbar_wait(bar_qfull + (t + 1) % QS, ((t + 1) / QS) & 1, abort_flag, p.status,
+                         WB_QFULL))
+            return false;
+          tc_fence_after();
+          mma_sdp(tmem + C::TM_S + ((t + 1) & 1) * BR, aK, stage_q(t + 1));
+          umma_commit(bar_s + ((t + 1) & 1));
+          return true;
+        };
+        if (QS > 1 && !(ok = next_s())) break;
         // dK += dS^T Q
         if (!(ok = mbar_wait(bar_ds, t & 1, abort_flag, p.status, WB_DS))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BR / 16; ++kk) {
           const uint32_t bo = (dcol0 / 64) * BR * 128 + kk * 2048;
-          umma_ts(tmem + C::TM_DK, tmem + C::TM_DP + kk * 8, sdesc_sw128(aQ + bo, BR * 128, 1024),
-                  ID_KV, (t > 0 || kk > 0) ? 1u : 0u);
+          umma_ts(tmem + C::TM_DK, tmem + C::TM_DP + pcol(kk),
+                  sdesc_sw128(aQ + bo, BR * 128, 1024), ID_KV, (t > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(bar_qempty + st);
         // dQ^T = K^T dS^T  (M = 128 rows of d, N = BR queries, K = 128 keys).
         // For d = 64 the upper 64 rows of M read the V tile and are ignored.
-        if (!(ok = mbar_wait(bar_dqempty, (t & 1) ^ 1, abort_flag, p.status, WB_DQEMPTY))) break;
+        if (t > 0 && !(ok = mbar_wait(bar_dqempty, (t - 1) & 1, abort_flag, p.status, WB_DQEMPTY)))
+          break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BC / 16; ++kk) {
@@ -344,174 +372,200 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
                   sdesc_sw128(adS + kk * 2048, BC * 128, 1024), ID_DQ, kk > 0);
         }
         umma_commit(bar_dqfull);
+        if (QS == 1 && !(ok = next_s())) break;
+        // dP^T of the next step (overwrites dS^T_t, read by dK_t above)
+        if (t + 1 < n_steps) {
+          mma_sdp(tmem + C::TM_DP, aV, stage_q(t + 1) + C::QT_BYTES);
+          umma_commit(bar_dp);
+        }
       }
       umma_commit(bar_final);
       volatile int no_abort = 0;
       mbar_wait(bar_final, 0, &no_abort, nullptr, WB_DRAIN);
     }
-  } else {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ compute warps
-    const int r = threadIdx.x;                     // key row == TMEM lane
-    const uint32_t tl = tmem + (uint32_t(warp * 32) << 16);
+    const int g = warp >> 2;                       // compute group: query columns [32g, 32g+32)
+    const int w = warp & 3;                        // TMEM lane quarter
+    const int r = w * 32 + lane;                   // key row == TMEM lane (also d row for dQ^T)
+    const uint32_t tl = tmem + (uint32_t(w * 32) << 16);
     const int key = key0 + r;
     const float sl2 = p.scale_log2;
     bool ok = true;
-    for (int t = 0; t < n_steps; ++t) {
-      const int hh = t / n_i;
-      const int qi = i0 + (t - hh * n_i);
-      const int bh = b * p.Hq + hkv * p.group + hh;
-      const int st = t % QS;
-      const float* sl = reinterpret_cast<const float*>(sStage + st * C::STAGE_STRIDE +
-                                                       2 * C::QT_BYTES);
-      const float* sd = sl + BR;
-      const int q0 = qi * BR;
-      // Queries visible to this key: q >= key (causal); columns c < cstart
-      // are masked.  Padding keys (>= Nk) are masked in every column.
-      const bool need_mask = (CAUSAL && (key0 + BC - 1 > q0)) || (key0 + BC > p.Nk);
-      const int cstart = key >= p.Nk ? BR : (CAUSAL ? key - q0 : 0);
 
-      ok = mbar_wait(bar_qfull + st, (t / QS) & 1, abort_flag, p.status, WB_QFULL) &&
-           mbar_wait(bar_s, t & 1, abort_flag, p.status, WB_S);
-      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-      tc_fence_after();
-      // P^T for this key row, kept in registers for dS.  It goes back to TMEM
-      // (over S^T) as two bf16 halves, hi = bf16(P) in columns [0, BR/2) and
-      // lo = bf16(P - hi) in [BR/2, BR): dV accumulates P_hi^T dO + P_lo^T dO,
-      // so the rounding of P to bf16 does not pile up across the many query
-      // rows (and query heads of a GQA group) that feed one dV row.
-      float P[BR];
-#pragma unroll
-      for (int c = 0; c < BR / 32; ++c) {
-        uint32_t u[32];
-        FA_TMEM_LD32(tl + C::TM_S + c * 32, u);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int cc = c * 32 + i;
-          float pv = ex2(fmaf(__uint_as_float(u[i]), sl2, -sl[cc]));
-          if (need_mask && cc < cstart) pv = 0.f;
-          P[cc] = pv;
-        }
-      }
-#pragma unroll
-      for (int c = 0; c < BR / 32; ++c) {
-        uint32_t hi[16], lo[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p0 = P[c * 32 + 2 * i], p1 = P[c * 32 + 2 * i + 1];
-          const uint32_t h = pack_bf16(p0, p1);
-          hi[i] = h;
-          lo[i] = pack_bf16(p0 - __uint_as_float(h << 16), p1 - __uint_as_float(h & 0xFFFF0000u));
-        }
-        FA_TMEM_ST16(tl + C::TM_S + c * 16, hi);
-        FA_TMEM_ST16(tl + C::TM_S + BR / 2 + c * 16, lo);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar_p);
-
-      ok = mbar_wait(bar_dp, t & 1, abort_flag, p.status, WB_DP);
-      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-      tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < BR / 32; ++c) {
-        uint32_t u[32];
-        FA_TMEM_LD32(tl + C::TM_DP + c * 32, u);
-        tmem_wait_ld();
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const int cc = c * 32 + i;
-          const float d0 = P[cc] * (__uint_as_float(u[i]) - sd[cc]);
-          const float d1 = P[cc + 1] * (__uint_as_float(u[i + 1]) - sd[cc + 1]);
-          pk[i / 2] = pack_bf16(d0, d1);
-        }
-        FA_TMEM_ST16(tl + C::TM_DP + c * 16, pk);
-        // dS^T row r, queries c*32 .. c*32+31: half of a 128-byte swizzled row
-        uint8_t* row = sdS + (c >> 1) * BC * 128 + r * 128;
-#pragma unroll
-        for (int u4 = 0; u4 < 4; ++u4) {
-          const int unit = (c & 1) * 4 + u4;
-          *reinterpret_cast<uint4*>(row + ((unit ^ (r & 7)) * 16)) =
-              make_uint4(pk[4 * u4], pk[4 * u4 + 1], pk[4 * u4 + 2], pk[4 * u4 + 3]);
-        }
-      }
-      tmem_wait_st();
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(bar_ds);
-
-      // dQ^T for this step: lane r holds d column dcol0 + r for BR queries.
-      ok = mbar_wait(bar_dqfull, t & 1, abort_flag, p.status, WB_DQFULL);
-      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+    // Read out dQ^T of step u (lanes = d, columns = this group's 32 queries)
+    // and reduce-add it into the fp32 accumulator (coalesced over d).
+    auto dq_readout = [&](int u) -> bool {
+      bool okk = mbar_wait(bar_dqfull, u & 1, abort_flag, p.status, WB_DQFULL);
+      if (!__all_sync(0xffffffffu, okk)) return false;
       tc_fence_after();
       if (r < DH) {
+        uint32_t v[32];
+        FA_TMEM_LD32(tl + C::TM_DQ + g * 32, v);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar_dqempty);
+        const int hh = u / n_i;
+        const int q0 = (i0 + (u - hh * n_i)) * BR + g * 32;
+        const int bh = b * p.Hq + hkv * p.group + hh;
         float* dst = p.dqacc + (size_t(bh) * p.Nq + q0) * D + dcol0 + r;
-        const int nvalid = min(BR, p.Nq - q0);
+        if (q0 + 32 <= p.Nq) {
 #pragma unroll
-        for (int c = 0; c < BR / 32; ++c) {
-          uint32_t u[32];
-          FA_TMEM_LD32(tl + C::TM_DQ + c * 32, u);
-          tmem_wait_ld();
-          if (c == BR / 32 - 1) {
-            tc_fence_before();
-            mbar_arrive(bar_dqempty);
-          }
+          for (int i = 0; i < 32; ++i) atomicAdd(dst + i * D, __uint_as_float(v[i]));
+        } else {
+          const int nvalid = p.Nq - q0;
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            if (c * 32 + i < nvalid) atomicAdd(dst + size_t(c * 32 + i) * D, __uint_as_float(u[i]));
+            if (i < nvalid) atomicAdd(dst + i * D, __uint_as_float(v[i]));
         }
       } else {
         tc_fence_before();
         mbar_arrive(bar_dqempty);
       }
-    }
+      return true;
+    };
 
-    // ---- epilogue: dK = scale * dK_acc and dV, bf16, through shared memory
+    for (int t = 0; t < n_steps; ++t) {
+      const int hh = t / n_i;
+      const int qi = i0 + (t - hh * n_i);
+      const int st = t % QS;
+      const float* sl = reinterpret_cast<const float*>(sStage + st * C::STAGE_STRIDE +
+                                                       2 * C::QT_BYTES) + g * 32;
+      const float* sd = sl + BR;
+      const int qg = qi * BR + g * 32;              // first query of this group's columns
+      // Columns c < cstart are masked: causal (query < key) or padding key.
+      const bool need_mask = (CAUSAL && key0 + BC - 1 > qg) || (key0 + BC > p.Nk);
+      const int cstart = key >= p.Nk ? 32 : (CAUSAL ? key - qg : 0);
+      const uint32_t tS = tl + C::TM_S + (t & 1) * BR + g * 32;
+      const uint32_t tDP = tl + C::TM_DP + g * 32;
+
+      ok = mbar_wait(bar_qfull + st, (t / QS) & 1, abort_flag, p.status, WB_QFULL) &&
+           mbar_wait(bar_s + (t & 1), (t >> 1) & 1, abort_flag, p.status, WB_S);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      tc_fence_after();
+      // ---- P^T for this key row and the group's 32 queries: hi = bf16(P)
+      // over columns [0,16) of the group's S^T columns, lo = bf16(P - hi)
+      // over [16,32); dV accumulates both, so rounding P to bf16 does not
+      // pile up over the many query rows (and GQA heads) that feed one dV row.
+      float P[32];
+      {
+        uint32_t u[32];
+        FA_TMEM_LD32(tS, u);
+        float lse2[32];
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4*>(lse2 + i) =
+            *reinterpret_cast<const float4*>(sl + i);
+        tmem_wait_ld();
+        const float2 sl22 = make_float2(sl2, sl2);
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const float2 x = ffma2(make_float2(__uint_as_float(u[i]), __uint_as_float(u[i + 1])),
+                                 sl22, make_float2(-lse2[i], -lse2[i + 1]));
+          P[i] = ex2(x.x);
+          P[i + 1] = ex2(x.y);
+        }
+        if (need_mask) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) P[i] = (i < cstart) ? 0.f : P[i];
+        }
+        uint32_t hi[16], lo[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const uint32_t h = pack_bf16(P[2 * i], P[2 * i + 1]);
+          hi[i] = h;
+          const float2 rem = fadd2(make_float2(P[2 * i], P[2 * i + 1]),
+                                   make_float2(-__uint_as_float(h << 16),
+                                               -__uint_as_float(h & 0xFFFF0000u)));
+          lo[i] = pack_bf16(rem.x, rem.y);
+        }
+        FA_TMEM_ST16(tS, hi);
+        FA_TMEM_ST16(tS + 16, lo);
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      mbar_arrive(bar_p);
+
+      // ---- dQ of the previous step (its MMA ran while P was formed)
+      if (t > 0 && !(ok = dq_readout(t - 1))) break;
+
+      // ---- dS^T = P^T o (dP^T - D)
+      ok = mbar_wait(bar_dp, t & 1, abort_flag, p.status, WB_DP);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      tc_fence_after();
+      {
+        uint32_t u[32];
+        FA_TMEM_LD32(tDP, u);
+        float dd[32];
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4*>(dd + i) =
+            *reinterpret_cast<const float4*>(sd + i);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float2 x = fadd2(make_float2(__uint_as_float(u[2 * i]),
+                                             __uint_as_float(u[2 * i + 1])),
+                                 make_float2(-dd[2 * i], -dd[2 * i + 1]));
+          const float2 y = fmul2(make_float2(P[2 * i], P[2 * i + 1]), x);
+          pk[i] = pack_bf16(y.x, y.y);
+        }
+        FA_TMEM_ST16(tDP, pk);
+        // dS^T row r, queries 32g..32g+31: half of a 128-byte swizzled row
+        uint8_t* row = sdS + r * 128;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const int unit = g * 4 + q4;
+          *reinterpret_cast<uint4*>(row + ((unit ^ (r & 7)) * 16)) =
+              make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+        }
+        tmem_wait_st();
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar_ds);
+    }
+    if (ok && n_steps > 0) ok = dq_readout(n_steps - 1);
+
+    // ---- epilogue: group 0 writes dK = scale * dK_acc, group 1 writes dV,
+    // bf16 through the (now free) Q/dO stages, one 4 KiB box per warp and
+    // 64 columns.
     if (ok && n_steps > 0) {
       ok = mbar_wait(bar_final, 0, abort_flag, p.status, WB_FINAL);
       ok = __all_sync(0xffffffffu, ok);
       if (ok) tc_fence_after();
     }
     if (ok) {
-      // The Q/dO stages are free now: stage dK then dV (each [DH/64][128][128B]).
+      const int tcol = g == 0 ? C::TM_DK : C::TM_DV;
+      const float mul = g == 0 ? p.scale : 1.f;
+      uint8_t* stage = sStage + g * (BC * DH * 2);
 #pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        const int tcol = which == 0 ? C::TM_DK : C::TM_DV;
-        const float mul = which == 0 ? p.scale : 1.f;
-        uint8_t* stage = sStage + which * (BC * DH * 2);
+      for (int c = 0; c < DH / 32; ++c) {
+        uint32_t u[32];
+        if (n_steps > 0) {
+          FA_TMEM_LD32(tl + tcol + c * 32, u);
+          tmem_wait_ld();
+        } else {
 #pragma unroll
-        for (int c = 0; c < DH / 32; ++c) {
-          uint32_t u[32];
-          if (n_steps > 0) {
-            FA_TMEM_LD32(tl + tcol + c * 32, u);
-            tmem_wait_ld();
-          } else {
+          for (int i = 0; i < 32; ++i) u[i] = 0u;
+        }
+        uint32_t pk[16];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) u[i] = 0u;
-          }
-          uint32_t pk[16];
+        for (int i = 0; i < 16; ++i)
+          pk[i] = pack_bf16(__uint_as_float(u[2 * i]) * mul, __uint_as_float(u[2 * i + 1]) * mul);
+        uint8_t* box = stage + ((c >> 1) * 4 + w) * 4096 + lane * 128;
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            pk[i] = pack_bf16(__uint_as_float(u[2 * i]) * mul, __uint_as_float(u[2 * i + 1]) * mul);
-          uint8_t* box = stage + ((c >> 1) * 4 + warp) * 4096 + lane * 128;
-#pragma unroll
-          for (int u4 = 0; u4 < 4; ++u4) {
-            const int unit = (c & 1) * 4 + u4;
-            *reinterpret_cast<uint4*>(box + ((unit ^ (lane & 7)) * 16)) =
-                make_uint4(pk[4 * u4], pk[4 * u4 + 1], pk[4 * u4 + 2], pk[4 * u4 + 3]);
-          }
+        for (int u4 = 0; u4 < 4; ++u4) {
+          const int unit = (c & 1) * 4 + u4;
+          *reinterpret_cast<uint4*>(box + ((unit ^ (lane & 7)) * 16)) =
+              make_uint4(pk[4 * u4], pk[4 * u4 + 1], pk[4 * u4 + 2], pk[4 * u4 + 3]);
         }
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0 && key0 + warp * 32 < p.Nk) {
-        for (int which = 0; which < 2; ++which) {
-          const CUtensorMap* tm = which == 0 ? &tmdK : &tmdV;
-          const uint8_t* stage = sStage + which * (BC * DH * 2);
-          for (int c = 0; c < DH / 64; ++c)
-            tma_store_3d(tm, stage + (c * 4 + warp) * 4096, dcol0 + c * 64, key0 + warp * 32, bkv);
-        }
+      if (lane == 0 && key0 + w * 32 < p.Nk) {
+        const CUtensorMap* tm = g == 0 ? &tmdK : &tmdV;
+        for (int c = 0; c < DH / 64; ++c)
+          tma_store_3d(tm, stage + (c * 4 + w) * 4096, dcol0 + c * 64, key0 + w * 32, bkv);
         bulk_commit();
         bulk_wait0();
       }
@@ -520,7 +574,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
