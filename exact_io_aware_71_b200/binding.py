@@ -23,7 +23,7 @@ STATUS_NAMES = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED",
 
 # Exported symbols declared in include/fa.h.
 SYMBOLS = ("fa_fwd", "fa_bwd", "fa_bwd_stage", "fa_bwd_workspace_size", "fa_status_string",
-           "fa_device_status", "fa_bwd_noalloc")
+           "fa_device_status", "fa_bwd_noalloc", "fa_debug_inject")
 
 # Bytes of the built-in scratch behind fa_bwd_noalloc (FA_NOALLOC_SCRATCH_BYTES).
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -64,6 +64,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fa_status_string.restype = ctypes.c_char_p
     lib.fa_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
     lib.fa_device_status.restype = i
+    lib.fa_debug_inject.argtypes = [i, ctypes.c_double]
+    lib.fa_debug_inject.restype = i
     _lib = lib
     return lib
 
@@ -100,6 +102,11 @@ def fa_bwd_workspace_size(B, Hq, Hkv, Nq, Nk, d, causal) -> int:
 
 def fa_status_string(status: int) -> str:
     return load().fa_status_string(status).decode()
+
+
+def fa_debug_inject(stall_kv_loads: int, wait_limit_seconds: float) -> int:
+    """Test control for the timeout path (see include/fa.h)."""
+    return load().fa_debug_inject(int(stall_kv_loads), float(wait_limit_seconds))
 
 
 def fa_device_status(stream=None):

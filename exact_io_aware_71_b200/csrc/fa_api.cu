@@ -3,6 +3,7 @@
 // this file only validates, describes the tensors to the TMA unit and launches.
 #include <cmath>
 #include <cstdint>
+#include <cstddef>
 #include <cstring>
 #include <mutex>
 #include <algorithm>
@@ -254,11 +255,28 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
 
 int fa_device_status(cudaStream_t stream, int* where) {
   if (cudaStreamSynchronize(stream) != cudaSuccess) return FA_ERR_CUDA;
-  DevStatus h{0u, 0u}, zero{0u, 0u};
-  if (cudaMemcpyFromSymbol(&h, g_status, sizeof(h)) != cudaSuccess) return FA_ERR_CUDA;
-  if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return FA_ERR_CUDA;
-  if (where) *where = int(h.where);
-  return h.timeout ? FA_ERR_DEVICE_TIMEOUT : FA_OK;
+  unsigned int h[2] = {0u, 0u};
+  const unsigned int zero[2] = {0u, 0u};
+  // Only the two report words; the test controls behind them are left alone.
+  if (cudaMemcpyFromSymbol(h, g_status, sizeof(h)) != cudaSuccess) return FA_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_status, zero, sizeof(zero)) != cudaSuccess) return FA_ERR_CUDA;
+  if (where) *where = int(h[1]);
+  return h[0] ? FA_ERR_DEVICE_TIMEOUT : FA_OK;
+}
+
+int fa_debug_inject(int stall_kv_loads, double wait_limit_seconds) {
+  if ((stall_kv_loads != 0 && stall_kv_loads != 1) || !(wait_limit_seconds >= 0.0) ||
+      wait_limit_seconds > 60.0)
+    return FA_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return FA_ERR_CUDA;
+  const unsigned long long ns = (unsigned long long)(wait_limit_seconds * 1e9);
+  const int stall = stall_kv_loads;
+  if (cudaMemcpyToSymbol(g_status, &ns, sizeof(ns), offsetof(DevStatus, wait_limit_ns)) !=
+          cudaSuccess ||
+      cudaMemcpyToSymbol(g_status, &stall, sizeof(stall), offsetof(DevStatus, stall_kv)) !=
+          cudaSuccess)
+    return FA_ERR_CUDA;
+  return cudaDeviceSynchronize() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 }  // extern "C"

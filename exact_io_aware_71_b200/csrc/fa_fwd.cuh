@@ -308,7 +308,7 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
       }
       // Ring order = MMA consumption order: K0, V0, K1, V1, ...
       int cnt = 0;
-      bool ok = true;
+      bool ok = !p.status->stall_kv;   // test control: withhold K/V (see fa_debug_inject)
       for (int j = 0; j < nmax && ok; ++j) {
         for (int kv = 0; kv < 2 && ok; ++kv) {
           const int slot = cnt % NS;
@@ -541,7 +541,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
       for (int c = 0; c < C::KCH; ++c)
         tma_load_3d(sQ + c * BR * 128, &tmQ, bar_q, c * 64, q_row0, bh);
       int cnt = 0;
-      bool ok = true;
+      bool ok = !p.status->stall_kv;   // test control: withhold K/V (see fa_debug_inject)
       auto load = [&](const CUtensorMap* tm, int j) {
         const int slot = cnt % NS;
         const uint32_t ph = (cnt / NS) & 1;
@@ -556,7 +556,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
         ++cnt;
       };
       // Ring order = MMA consumption order: K0, K1, V0, K2, V1, ...
-      load(&tmK, 0);
+      if (ok) load(&tmK, 0);
       for (int j = 1; j < n_blocks && ok; ++j) {
         load(&tmK, j);
         if (ok) load(&tmV, j - 1);

@@ -14,10 +14,15 @@
 
 namespace fa {
 
-// Device-side status words, one per error kind; read back by the host.
+// Per-device status and test controls (one instance per device).  The
+// kernels write `timeout`/`where`; the host reads and clears them.  The two
+// controls are set only by fa_debug_inject for tests of the timeout path.
 struct DevStatus {
-  unsigned int timeout;      // a bounded wait expired
-  unsigned int where;        // which wait (kernel-defined code) expired first
+  unsigned int timeout;              // a bounded wait expired
+  unsigned int where;                // which wait (kernel-defined code) expired first
+  unsigned long long wait_limit_ns;  // 0 = FA_WAIT_LIMIT_NS
+  int stall_kv;                      // forward producers withhold K/V tiles
+  int pad;
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -76,11 +81,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = globaltimer();
+  uint64_t limit = FA_WAIT_LIMIT_NS;
+  if (st) {
+    const uint64_t l = *reinterpret_cast<volatile unsigned long long*>(&st->wait_limit_ns);
+    if (l) limit = l;
+  }
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(a, parity)) return true;
     if ((it & 255u) == 0) {
       if (*abort) return false;
-      if (globaltimer() - t0 > FA_WAIT_LIMIT_NS) {
+      if (globaltimer() - t0 > limit) {
         *abort = 1;
         if (st) {
           if (atomicCAS(&st->timeout, 0u, 1u) == 0u) st->where = where;

@@ -135,6 +135,17 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
                    const void* dO, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq,
                    int Nk, int d, int causal, float scale, cudaStream_t stream);
 
+/*
+ * Test control for the timeout path (for tests; not for production use).
+ * With stall_kv_loads = 1, forward launches on the current device withhold
+ * their K/V tiles, so the kernels' bounded pipeline waits expire: each CTA
+ * records FA_ERR_DEVICE_TIMEOUT (see fa_device_status), frees its resources
+ * and returns without writing o or lse.  wait_limit_seconds > 0 replaces the
+ * default 4 s limit of every pipeline wait; 0 restores it.  Synchronous;
+ * call fa_debug_inject(0, 0) to return to normal operation.
+ */
+int fa_debug_inject(int stall_kv_loads, double wait_limit_seconds);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* fa_status_string(int status);
 
