@@ -68,22 +68,27 @@ struct BwdCfg {
 inline int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
 // Workspace: dQacc fp32 [B*Hq, Nq, d] | Dpad fp32 [B*Hq, Nq_pad] | Lpad fp32 [B*Hq, Nq_pad]
+// Workspace: dQacc fp32 [B*Hq, Nq, d] | Dpad fp32 [B*Hq, Nq_pad] |
+// Lpad fp32 [B*Hq, Nq_pad] | (GQA/MQA only) dKacc, dVacc fp32 [B*Hkv, Nk, d]
+// for the partial sums of a kv group split across CTAs.
 struct BwdWorkspace {
-  size_t dq_off, d_off, l_off, total;
+  size_t dq_off, d_off, l_off, kv_off, kv_elems, total;
 };
-inline BwdWorkspace bwd_workspace_layout(int B, int Hq, int Nq, int d) {
+inline BwdWorkspace bwd_workspace_layout(int B, int Hq, int Hkv, int Nq, int Nk, int d) {
   const size_t bh = size_t(B) * Hq;
   const size_t nq_pad = size_t(round_up(Nq, 128));
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   BwdWorkspace w;
   w.dq_off = 0;
-  w.d_off = (bh * Nq * d * 4 + 255) / 256 * 256;
-  w.l_off = w.d_off + (bh * nq_pad * 4 + 255) / 256 * 256;
-  w.total = w.l_off + (bh * nq_pad * 4 + 255) / 256 * 256;
+  w.d_off = up(bh * Nq * d * 4);
+  w.l_off = w.d_off + up(bh * nq_pad * 4);
+  w.kv_off = w.l_off + up(bh * nq_pad * 4);
+  w.kv_elems = (Hq > Hkv) ? size_t(B) * Hkv * Nk * d : 0;   // per tensor
+  w.total = w.kv_off + up(2 * w.kv_elems * 4);
   return w;
 }
 inline size_t bwd_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d) {
-  (void)Hkv; (void)Nk;
-  return bwd_workspace_layout(B, Hq, Nq, d).total;
+  return bwd_workspace_layout(B, Hq, Hkv, Nq, Nk, d).total;
 }
 
 // ------------------------------------------------------------------ pre
@@ -93,7 +98,8 @@ template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(
     const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
     const float* __restrict__ lse, float* __restrict__ dqacc, float* __restrict__ Dpad,
-    float* __restrict__ Lpad, int rows_bh, int Nq, int Nq_pad) {
+    float* __restrict__ Lpad, int rows_bh, int Nq, int Nq_pad, float* __restrict__ kvacc,
+    long long kv_n4) {
   constexpr int TPR = D / 8;                       // threads per row
   constexpr int RPB = 256 / TPR;                   // rows per block pass
   const int sub = threadIdx.x % TPR;
@@ -130,6 +136,29 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(
       Lpad[pi] = valid ? lse[size_t(bh) * Nq + q] * 1.4426950408889634f : INFINITY;
     }
   }
+  // dK/dV partial-sum accumulators (only when a kv group is split across CTAs)
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < kv_n4;
+       i += (long long)gridDim.x * blockDim.x)
+    reinterpret_cast<float4*>(kvacc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// dk, dv = bf16 of the fp32 partial-sum accumulators (dK already scaled).
+__global__ void __launch_bounds__(256) fa_bwd_kv_kernel(const float* __restrict__ kvacc,
+                                                        __nv_bfloat16* __restrict__ dk,
+                                                        __nv_bfloat16* __restrict__ dv,
+                                                        long long n8) {
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < 2 * n8;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long j = i < n8 ? i : i - n8;
+    const float4 a = reinterpret_cast<const float4*>(kvacc)[2 * i];
+    const float4 b = reinterpret_cast<const float4*>(kvacc)[2 * i + 1];
+    uint4 out;
+    out.x = pack_bf16(a.x, a.y);
+    out.y = pack_bf16(a.z, a.w);
+    out.z = pack_bf16(b.x, b.y);
+    out.w = pack_bf16(b.z, b.w);
+    reinterpret_cast<uint4*>(i < n8 ? dk : dv)[j] = out;
+  }
 }
 
 // ------------------------------------------------------------------ dq convert
@@ -160,6 +189,10 @@ struct BwdParams {
   const float* Dpad;
   const float* Lpad;
   float* dqacc;
+  int gsplit;         // CTAs sharing one kv group's query heads (1 = none)
+  int hps;            // query heads per CTA: group / gsplit
+  float* dkacc;       // fp32 dK / dV partial sums when gsplit > 1
+  float* dvacc;
   DevStatus* status;
 };
 
@@ -212,8 +245,12 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
 
   // Work unit: (batch, kv head, key block, d half).  Key blocks near the
   // start see the most query blocks under the causal mask; they go first.
+  // With a large GQA/MQA group and few key blocks, the group's query heads
+  // are split over `gsplit` CTAs that add fp32 partial dK / dV.
   const int split = blockIdx.x % C::NSPLIT;
-  const int rest = blockIdx.x / C::NSPLIT;
+  int rest = blockIdx.x / C::NSPLIT;
+  const int gs = rest % p.gsplit;
+  rest /= p.gsplit;
   const int kb = rest % p.n_kblocks;
   const int bkv = rest / p.n_kblocks;
   const int b = bkv / p.Hkv;
@@ -221,8 +258,19 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
   const int key0 = kb * BC;
   const int i0 = CAUSAL ? (key0 / BR) : 0;              // first query block that sees key0
   const int n_i = max(0, p.n_qblocks - i0);
-  const int n_steps = p.group * n_i;
+  const int n_steps = p.hps * n_i;
   const int dcol0 = split * DH;                         // first d column owned here
+  const int head0 = hkv * p.group + gs * p.hps;         // first query head (within batch b)
+  // Without the causal mask every key block visits every query block; key
+  // blocks start at different query blocks so that their fp32 dQ reduce-adds
+  // do not all land on the same rows at once.
+  const int rot = CAUSAL ? 0 : int((long long)kb * n_i / p.n_kblocks);
+  auto step_q = [&](int t, int& hh, int& qi) {
+    hh = t / n_i;
+    int li = t - hh * n_i + rot;
+    if (li >= n_i) li -= n_i;
+    qi = i0 + li;
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(bar_kv, 1);
@@ -262,9 +310,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
       }
       int issued = 0;
       for (int t = 0; t < n_steps; ++t) {
-        const int hh = t / n_i;
-        const int qi = i0 + (t - hh * n_i);
-        const int bh = b * p.Hq + hkv * p.group + hh;
+        int hh, qi;
+        step_q(t, hh, qi);
+        const int bh = b * p.Hq + head0 + hh;
         const int st = t % QS;
         if (!mbar_wait(bar_qempty + st, ((t / QS) & 1) ^ 1, abort_flag, p.status, WB_QEMPTY))
           break;
@@ -405,9 +453,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(bar_dqempty);
-        const int hh = u / n_i;
-        const int q0 = (i0 + (u - hh * n_i)) * BR + g * 32;
-        const int bh = b * p.Hq + hkv * p.group + hh;
+        int hh, qi;
+        step_q(u, hh, qi);
+        const int q0 = qi * BR + g * 32;
+        const int bh = b * p.Hq + head0 + hh;
         float* dst = p.dqacc + (size_t(bh) * p.Nq + q0) * D + dcol0 + r;
         if (q0 + 32 <= p.Nq) {
 #pragma unroll
@@ -426,8 +475,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
     };
 
     for (int t = 0; t < n_steps; ++t) {
-      const int hh = t / n_i;
-      const int qi = i0 + (t - hh * n_i);
+      int hh, qi;
+      step_q(t, hh, qi);
       const int st = t % QS;
       const float* sl = reinterpret_cast<const float*>(sStage + st * C::STAGE_STRIDE +
                                                        2 * C::QT_BYTES) + g * 32;
@@ -534,7 +583,31 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (ok) tc_fence_after();
     }
-    if (ok) {
+    if (ok && p.gsplit > 1) {
+      // Partial sums of this CTA's query heads: fp32 reduce-adds, row by row
+      // (all lanes load from TMEM together; rows past Nk add nothing).
+      if (n_steps > 0) {
+        const int tcol = g == 0 ? C::TM_DK : C::TM_DV;
+        const float mul = g == 0 ? p.scale : 1.f;
+        float* dst = (g == 0 ? p.dkacc : p.dvacc) + (size_t(bkv) * p.Nk + key) * D + dcol0;
+        const bool row_ok = key < p.Nk;
+#pragma unroll
+        for (int c = 0; c < DH / 32; ++c) {
+          uint32_t u[32];
+          FA_TMEM_LD32(tl + tcol + c * 32, u);
+          tmem_wait_ld();
+          if (row_ok) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + c * 32 + i),
+                           "f"(__uint_as_float(u[i]) * mul), "f"(__uint_as_float(u[i + 1]) * mul),
+                           "f"(__uint_as_float(u[i + 2]) * mul),
+                           "f"(__uint_as_float(u[i + 3]) * mul)
+                           : "memory");
+          }
+        }
+      }
+    } else if (ok) {
       const int tcol = g == 0 ? C::TM_DK : C::TM_DV;
       const float mul = g == 0 ? p.scale : 1.f;
       uint8_t* stage = sStage + g * (BC * DH * 2);
@@ -589,13 +662,29 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
                  int Hkv, int Nq, int Nk, float scale, void* workspace, DevStatus* status,
                  cudaStream_t stream) {
   using C = BwdCfg<D>;
-  const BwdWorkspace w = bwd_workspace_layout(B, Hq, Nq, D);
+  const BwdWorkspace w = bwd_workspace_layout(B, Hq, Hkv, Nq, Nk, D);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* dqacc = reinterpret_cast<float*>(ws + w.dq_off);
   float* Dpad = reinterpret_cast<float*>(ws + w.d_off);
   float* Lpad = reinterpret_cast<float*>(ws + w.l_off);
+  float* kvacc = reinterpret_cast<float*>(ws + w.kv_off);
   const int Nq_pad = round_up(Nq, 128);
   const int bhq = B * Hq;
+  const int group = Hq / Hkv;
+  const int n_kblocks = (Nk + C::BC - 1) / C::BC;
+  // Split a kv group's query heads over several CTAs when the key blocks
+  // alone would leave SMs idle: the smallest divisor of the group that
+  // gives at least two CTAs per SM (same choice in every stage call).
+  int gsplit = 1;
+  if (group > 1) {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long base = (long long)n_kblocks * B * Hkv * C::NSPLIT;
+    gsplit = group;
+    for (int s = 1; s <= group; ++s)
+      if (group % s == 0 && base * s >= 2LL * sms) { gsplit = s; break; }
+  }
 
   CUtensorMap mq, mk, mv, mdo, mdk, mdv;
   if ((stages & 2) && (!make_map_bf16(&mq, q, D, Nq, int64_t(bhq), C::BR) ||
@@ -612,7 +701,7 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
     const long long blocks = std::min<long long>((rows + RPB - 1) / RPB, 148LL * 16);
     fa_bwd_pre_kernel<D><<<unsigned(blocks), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, dqacc,
-        Dpad, Lpad, bhq, Nq, Nq_pad);
+        Dpad, Lpad, bhq, Nq, Nq_pad, kvacc, gsplit > 1 ? (long long)(2 * w.kv_elems / 4) : 0LL);
     if (cudaGetLastError() != cudaSuccess) return 5;
   }
   if (stages & 2) {
@@ -622,8 +711,12 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
       return 5;
     BwdParams p;
     p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Nq = Nq; p.Nk = Nk; p.Nq_pad = Nq_pad;
-    p.group = Hq / Hkv;
-    p.n_kblocks = (Nk + C::BC - 1) / C::BC;
+    p.group = group;
+    p.n_kblocks = n_kblocks;
+    p.gsplit = gsplit;
+    p.hps = group / gsplit;
+    p.dkacc = kvacc;
+    p.dvacc = kvacc + w.kv_elems;
     p.n_qblocks = (Nq + C::BR - 1) / C::BR;
     p.scale = scale;
     p.scale_log2 = scale * 1.4426950408889634f;
@@ -631,7 +724,7 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
     p.Lpad = Lpad;
     p.dqacc = dqacc;
     p.status = status;
-    const unsigned grid = unsigned(p.n_kblocks) * unsigned(B * Hkv) * C::NSPLIT;
+    const unsigned grid = unsigned(p.n_kblocks) * unsigned(B * Hkv) * C::NSPLIT * gsplit;
     kern<<<grid, C::NTHREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdk, mdv, p);
     if (cudaGetLastError() != cudaSuccess) return 5;
   }
@@ -641,6 +734,13 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
     fa_bwd_dq_kernel<<<unsigned(blocks), 256, 0, stream>>>(
         dqacc, static_cast<__nv_bfloat16*>(dq), n8, scale);
     if (cudaGetLastError() != cudaSuccess) return 5;
+    if (gsplit > 1) {
+      const long long kv8 = (long long)w.kv_elems / 8;
+      const long long kblocks = std::min<long long>((2 * kv8 + 255) / 256, 148LL * 16);
+      fa_bwd_kv_kernel<<<unsigned(kblocks), 256, 0, stream>>>(
+          kvacc, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), kv8);
+      if (cudaGetLastError() != cudaSuccess) return 5;
+    }
   }
   return 0;
 }

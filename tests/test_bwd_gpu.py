@@ -90,14 +90,20 @@ def test_large_magnitude_scores(qmul):
     full_check(W(1, 2, 2, 512, 512, 64, True, seed=9), qmul=qmul, frobenius_only=("dK",))
 
 
-def test_backward_repeatable_within_tolerance():
+@pytest.mark.parametrize("hkv", [4, 2])
+def test_backward_repeatable_within_tolerance(hkv):
     """dQ is accumulated with unordered fp32 atomics, so runs may differ in
-    the last bits; dK and dV are accumulated in a fixed order."""
-    wl = W(1, 4, 2, 640, 640, 128, True)
+    the last bits.  With one kv head per query head, dK and dV are
+    accumulated in a fixed order and repeat bit for bit; when a GQA group's
+    query heads are split over CTAs (as here, few key blocks), dK and dV are
+    fp32 atomic sums too."""
+    wl = W(1, 4, hkv, 640, 640, 128, True)
     _, g1 = run(wl)
     _, g2 = run(wl)
-    assert np.array_equal(g1[1], g2[1]) and np.array_equal(g1[2], g2[2])
-    assert np.abs(g1[0] - g2[0]).max() <= 2e-2
+    if hkv == 4:
+        assert np.array_equal(g1[1], g2[1]) and np.array_equal(g1[2], g2[2])
+    for a, b in zip(g1, g2):
+        assert np.abs(a - b).max() <= 2e-2
 
 
 # --------------------------------------------------------------- full-size workloads
