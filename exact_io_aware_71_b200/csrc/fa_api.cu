@@ -142,8 +142,20 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
     }
     if (regs * C::NTHREADS < C::REGS_NEEDED) return FA_ERR_UNSUPPORTED;
     p.n_units = (p.n_qblocks + 1) / 2;
-    return launch_kernel(fa_fwd_pair_kernel<D, CAUSAL>, C::SMEM_BYTES, C::NTHREADS,
-                         unsigned(p.n_units) * unsigned(p.B * p.Hq), mq, mk, mv, mo, p, stream);
+    // Persistent (one CTA per SM, each walking a strided unit list) for short
+    // rows, where unit boundaries are frequent, and for causal rows up to 16k,
+    // whose units differ in length; one CTA per unit otherwise (measured
+    // faster for long rows, where the hardware's own CTA dispatch balances
+    // the units).  The kernel is the same; a CTA whose stride covers the
+    // whole list runs exactly one unit.
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long units = (long long)p.n_units * p.B * p.Hq;
+    const bool persistent = p.Nk <= 4096 || (CAUSAL && p.Nk <= 16384);
+    const unsigned grid = unsigned(persistent ? std::min<long long>(units, sms) : units);
+    return launch_kernel(fa_fwd_pair_kernel<D, CAUSAL>, C::SMEM_BYTES, C::NTHREADS, grid, mq, mk,
+                         mv, mo, p, stream);
   }
 }
 

@@ -23,8 +23,8 @@
 //    producer, warp 9 the MMA issuer (10, 11 idle).  TMEM holds S and O of
 //    each tile (2 x (128 + d) columns); while one warpgroup exponentiates its
 //    S, the tensor pipe works on the other tile, and two softmax warps share
-//    each SM sub-partition.  The softmax warpgroups take 216 registers per
-//    thread from the third warpgroup's share (setmaxnreg).
+//    each SM sub-partition.  The softmax warpgroups take 208 registers per
+//    thread from the third warpgroup's share (setmaxnreg, 208 / 88).
 //  * fa_fwd_kernel (d = 256): one 128-row tile per CTA with two S buffers
 //    (O alone takes 256 TMEM columns), warps 0-3 softmax, 4 producer, 5 MMA.
 #pragma once
@@ -67,13 +67,15 @@ struct RowState {
 //          P is written back over them as packed bf16 (BC/2 columns)
 //   tO     the row's O accumulator (D fp32 columns)
 //   j      block index within the tile's sequence; key0 = j * BC
+//   gj     running block index of this TMEM tile across the CTA's work
+//          (phases of the barriers); equals j when a CTA has one tile
 //   q_tile first query row of the tile, grow this thread's query row
 //   o_done the two barriers that complete after P V of even / odd blocks
 // The caller has waited for S; the function waits for P_{j-1} V_{j-1} only
 // if it has to rescale O.  Returns false if that wait gave up.
 template <int BC, int D, bool CAUSAL>
 __device__ __forceinline__ bool softmax_block(RowState& st, uint32_t tS, uint32_t tO, int j,
-                                              int q_tile, int grow, int Nk, float sl2,
+                                              int gj, int q_tile, int grow, int Nk, float sl2,
                                               uint64_t* o_done, volatile int* abort,
                                               DevStatus* status) {
   float s[BC];
@@ -113,7 +115,7 @@ __device__ __forceinline__ bool softmax_block(RowState& st, uint32_t tS, uint32_
       // barriers alternate by block parity: warps of a warpgroup may be one
       // block apart, and one barrier would let a warp at block j+1 take
       // P_{j-1}V_{j-1}'s completion (same parity) for P_j V_j's.
-      bool ok = mbar_wait(o_done + ((j - 1) & 1), ((j - 1) >> 1) & 1, abort, status, W_O_DONE);
+      bool ok = mbar_wait(o_done + ((gj - 1) & 1), ((gj - 1) >> 1) & 1, abort, status, W_O_DONE);
       if (!__all_sync(0xffffffffu, ok)) return false;
       tc_fence_after();
 #pragma unroll
@@ -213,14 +215,23 @@ struct FwdPairCfg {
   static constexpr int TM_TILE = 256;               // tile t: S at t*256, O at t*256 + 128
   static constexpr int TMEM_COLS = 512;
   static constexpr int NTHREADS = 384;
-  static constexpr int REGS_SOFTMAX = 216;          // per thread, warpgroups 0 and 1
-  static constexpr int REGS_OTHER = 72;             // per thread, warpgroup 2
+  static constexpr int REGS_SOFTMAX = 208;          // per thread, warpgroups 0 and 1
+  static constexpr int REGS_OTHER = 88;             // per thread, warpgroup 2
   static constexpr int REGS_NEEDED = 256 * REGS_SOFTMAX + 128 * REGS_OTHER;
   static constexpr int SMEM_BYTES = 2 * Q_BYTES + NS * KV_BYTES + 1024 + 1024;
   static_assert(128 + D <= TM_TILE, "TMEM budget");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
+// The CTAs are persistent: grid = min(#units, #SMs) and CTA c takes units
+// c, c + grid, ...  A unit is (batch, head, tile pair); the list is
+// head-major so that concurrently running units share K/V in L2, and under
+// the causal mask each head's longest pair comes first.  All roles walk the
+// same list; barrier phases run on across units.  Between units of a tile,
+// "Q free" (the epilogue's TMA store has read the staging buffer) gates the
+// next Q load and "O free" (the epilogue has read O from TMEM) gates the
+// next unit's first P V, while the tensor pipe already computes the next
+// unit's first S.
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
     fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
@@ -236,42 +247,58 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
   uint8_t* sQ = smem;                          // 2 tiles of [KCH][BR][128B]; O staging later
   uint8_t* sKV = smem + 2 * C::Q_BYTES;        // NS slots of [KCH][BC][128B]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + NS * C::KV_BYTES);
-  uint64_t* bar_q = bars + 0;                  // [2]
+  uint64_t* bar_q = bars + 0;                  // [2] Q tile loaded
   uint64_t* bar_kv_full = bars + 2;            // [NS]
   uint64_t* bar_kv_empty = bars + 2 + NS;      // [NS]
   uint64_t* bar_s_full = bars + 2 + 2 * NS;    // [2] per tile
   uint64_t* bar_p_full = bars + 4 + 2 * NS;    // [2] per tile
   uint64_t* bar_o_done = bars + 6 + 2 * NS;    // [2 tiles][2 parities]
-  uint64_t* bar_drain = bars + 10 + 2 * NS;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 12 + 2 * NS);
+  uint64_t* bar_q_free = bars + 10 + 2 * NS;   // [2] Q/staging buffer free (4 warps)
+  uint64_t* bar_o_free = bars + 12 + 2 * NS;   // [2] O read out of TMEM (128 threads)
+  uint64_t* bar_drain = bars + 14 + 2 * NS;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 16 + 2 * NS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int bhq = p.B * p.Hq;
+  const int total_units = p.n_units * bhq;
 
-  // Unit = (batch, head, tile pair).  Consecutive CTAs share a head so that
-  // its K/V stay hot in L2; causal pairs run longest first within a head.
-  const int bh = blockIdx.x / p.n_units;
-  int pu = blockIdx.x - bh * p.n_units;
-  if (CAUSAL) pu = p.n_units - 1 - pu;
-  const int b = bh / p.Hq;
-  const int h = bh - b * p.Hq;
-  const int bkv = b * p.Hkv + h / p.group;
-  const int q0 = pu * 2 * BR;
-  int nt[2];
+  // Unit u -> (bh, q0) and the number of key blocks of each tile.
+  // Non-causal units are equal: head-major order, so concurrent units share
+  // K/V in L2.  Causal units shrink with the pair index: pair-major from the
+  // longest pair down, and the k-th round of units is dealt to the CTAs in
+  // alternating direction (CTA c gets slot c, then grid-1-c, ...), which
+  // evens out the total work per CTA.
+  auto unit = [&](int u, int& bh, int& q0, int* nt) {
+    int pu;
+    if (CAUSAL) {
+      const int g = gridDim.x;
+      const int round = u / g, c = u - round * g;
+      // snake order; a partial last round keeps its order (a bijection)
+      const int v = ((round & 1) && (round + 1) * g <= total_units) ? round * g + (g - 1 - c) : u;
+      pu = p.n_units - 1 - v / bhq;
+      bh = v - (p.n_units - 1 - pu) * bhq;
+    } else {
+      bh = u / p.n_units;
+      pu = u - bh * p.n_units;
+    }
+    q0 = pu * 2 * BR;
 #pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    const int qt = q0 + t * BR;
-    const int kv_end = CAUSAL ? min(p.Nk, qt + BR) : p.Nk;
-    nt[t] = (qt < p.Nq) ? (kv_end + BC - 1) / BC : 0;   // tile 1 may lie past Nq
-  }
-  const int nmax = max(nt[0], nt[1]);
+    for (int t = 0; t < 2; ++t) {
+      const int qt = q0 + t * BR;
+      const int kv_end = CAUSAL ? min(p.Nk, qt + BR) : p.Nk;
+      nt[t] = (qt < p.Nq) ? (kv_end + BC - 1) / BC : 0;   // tile 1 may lie past Nq
+    }
+  };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar_q + i, 1);
       mbar_init(bar_s_full + i, 1);
       mbar_init(bar_p_full + i, BR);
+      mbar_init(bar_q_free + i, 4);
+      mbar_init(bar_o_free + i, BR);
     }
     for (int i = 0; i < NS; ++i) {
       mbar_init(bar_kv_full + i, 1);
@@ -299,36 +326,54 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      for (int t = 0; t < 2; ++t) {
-        if (nt[t] == 0) continue;
-        mbar_arrive_expect_tx(bar_q + t, C::Q_BYTES);
-        for (int c = 0; c < C::KCH; ++c)
-          tma_load_3d(sQ + t * C::Q_BYTES + c * BR * 128, &tmQ, bar_q + t, c * 64, q0 + t * BR,
-                      bh);
-      }
-      // Ring order = MMA consumption order: K0, V0, K1, V1, ...
-      int cnt = 0;
+      int cnt = 0;                                 // K/V ring position
+      int uses[2] = {0, 0};                        // units in which each tile was active
       bool ok = !p.status->stall_kv;   // test control: withhold K/V (see fa_debug_inject)
-      for (int j = 0; j < nmax && ok; ++j) {
-        for (int kv = 0; kv < 2 && ok; ++kv) {
+      for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
+        int bh, q0, nt[2];
+        unit(u, bh, q0, nt);
+        const int bkv = (bh / p.Hq) * p.Hkv + (bh % p.Hq) / p.group;
+        // Ring order = MMA consumption order: K0, V0, K1, V1, ...  The first
+        // ring items of a unit go out before its Q loads, which wait for the
+        // previous unit's epilogue to release the Q/staging buffers.
+        const int items = 2 * max(nt[0], nt[1]);
+        auto ring = [&](int item) -> bool {
           const int slot = cnt % NS;
           if (!mbar_wait(bar_kv_empty + slot, ((cnt / NS) & 1) ^ 1, abort_flag, p.status,
-                         W_KV_EMPTY)) {
-            ok = false;
-            break;
-          }
+                         W_KV_EMPTY))
+            return false;
           mbar_arrive_expect_tx(bar_kv_full + slot, C::KV_BYTES);
           uint8_t* dst = sKV + slot * C::KV_BYTES;
-          const CUtensorMap* tm = kv == 0 ? &tmK : &tmV;
+          const CUtensorMap* tm = (item & 1) ? &tmV : &tmK;
           for (int c = 0; c < C::KCH; ++c)
-            tma_load_3d(dst + c * BC * 128, tm, bar_kv_full + slot, c * 64, j * BC, bkv);
+            tma_load_3d(dst + c * BC * 128, tm, bar_kv_full + slot, c * 64, (item >> 1) * BC, bkv);
           ++cnt;
+          return true;
+        };
+        const int early = min(items, NS);
+        for (int it = 0; it < early && ok; ++it) ok = ring(it);
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (nt[t] == 0) continue;
+          if (uses[t] > 0 &&
+              !(ok = mbar_wait(bar_q_free + t, (uses[t] - 1) & 1, abort_flag, p.status, W_Q)))
+            break;
+          mbar_arrive_expect_tx(bar_q + t, C::Q_BYTES);
+          for (int c = 0; c < C::KCH; ++c)
+            tma_load_3d(sQ + t * C::Q_BYTES + c * BR * 128, &tmQ, bar_q + t, c * 64,
+                        q0 + t * BR, bh);
+          ++uses[t];
         }
+        for (int it = early; it < items && ok; ++it) ok = ring(it);
       }
       if (!ok) {
+        // Let the copies already issued land before the CTA exits.
         for (int i = cnt - 1; i >= 0 && i >= cnt - NS; --i) {
           volatile int no_abort = 0;
           mbar_wait(bar_kv_full + (i % NS), (i / NS) & 1, &no_abort, nullptr, W_DRAIN);
+        }
+        for (int t = 0; t < 2; ++t) {
+          volatile int no_abort = 0;
+          if (uses[t] > 0) mbar_wait(bar_q + t, (uses[t] - 1) & 1, &no_abort, nullptr, W_DRAIN);
         }
       }
     }
@@ -339,7 +384,9 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
       constexpr uint32_t IDESC_O = idesc_bf16_f32(BR, D, 0, 1);
       const uint32_t sQ_addr = smem_u32(sQ);
       const uint32_t sKV_addr = smem_u32(sKV);
-      int cnt = 0;
+      int cnt = 0;                                 // K/V ring position
+      int uses[2] = {0, 0};                        // units in which each tile was active
+      int gb[2] = {0, 0};                          // running block count per tile
       bool ok = true;
       auto acquire = [&](int& slot) -> bool {
         slot = cnt % NS;
@@ -360,8 +407,14 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
         }
         umma_commit(bar_s_full + t);
       };
-      auto mma_pv = [&](int t, int j, int slot) -> bool {
-        if (!mbar_wait(bar_p_full + t, j & 1, abort_flag, p.status, W_P_FULL)) return false;
+      // P_t V_j of the tile's block j (running index gj).  Its first block
+      // in a unit overwrites O, so it waits until the tile's previous
+      // epilogue has read O out of TMEM.
+      auto mma_pv = [&](int t, int j, int gj, int slot) -> bool {
+        if (j == 0 && uses[t] > 1 &&
+            !mbar_wait(bar_o_free + t, (uses[t] - 2) & 1, abort_flag, p.status, W_O_DONE))
+          return false;
+        if (!mbar_wait(bar_p_full + t, gj & 1, abort_flag, p.status, W_P_FULL)) return false;
         tc_fence_after();
         const uint32_t vbase = sKV_addr + slot * C::KV_BYTES;
         const uint32_t tt = tmem + t * C::TM_TILE;
@@ -370,41 +423,44 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
           const uint64_t bd = sdesc_sw128(vbase + kk * 16 * 128, BC * 128, 1024);
           umma_ts(tt + 128, tt + kk * 8, bd, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(bar_o_done + t * 2 + (j & 1));
+        umma_commit(bar_o_done + t * 2 + (gj & 1));
         return true;
       };
-      int sK = 0, sV = 0;
-      ok = acquire(sK);
-      if (ok) ok = mbar_wait(bar_q + 0, 0, abort_flag, p.status, W_Q);
-      if (ok) {
-        tc_fence_after();
-        mma_s(0, sK);
-        if (nt[1] > 0) {
-          ok = mbar_wait(bar_q + 1, 0, abort_flag, p.status, W_Q);
-          if (ok) {
-            tc_fence_after();
-            mma_s(1, sK);
+      for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
+        int bh, q0, nt[2];
+        unit(u, bh, q0, nt);
+        const int nmax = max(nt[0], nt[1]);
+        int sK = 0, sV = 0;
+        if (!(ok = acquire(sK))) break;
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (nt[t] == 0) continue;
+          if (!(ok = mbar_wait(bar_q + t, uses[t] & 1, abort_flag, p.status, W_Q))) break;
+          tc_fence_after();
+          ++uses[t];
+          mma_s(t, sK);
+        }
+        if (!ok) break;
+        umma_commit(bar_kv_empty + sK);
+        // Per block j: P0 V_j, then S0_{j+1} (it overwrites P0_j in TMEM, so
+        // it must follow P0_j V_j; tcgen05 MMAs run in issue order), then the
+        // same for tile 1.  Each K/V slot is released after its last reader.
+        for (int j = 0; j < nmax && ok; ++j) {
+          if (!(ok = acquire(sV))) break;
+          if (j < nt[0] && !(ok = mma_pv(0, j, gb[0] + j, sV))) break;
+          const bool next = j + 1 < nmax;
+          if (next) {
+            if (!(ok = acquire(sK))) break;
+            if (j + 1 < nt[0]) mma_s(0, sK);
+          }
+          if (j < nt[1] && !(ok = mma_pv(1, j, gb[1] + j, sV))) break;
+          umma_commit(bar_kv_empty + sV);
+          if (next) {
+            if (j + 1 < nt[1]) mma_s(1, sK);
+            umma_commit(bar_kv_empty + sK);
           }
         }
-        umma_commit(bar_kv_empty + sK);
-      }
-      // Per block j: P0 V_j, then S0_{j+1} (it overwrites P0_j in TMEM, so it
-      // must follow P0_j V_j; tcgen05 MMAs run in issue order), then the
-      // same for tile 1.  Each K/V slot is released after its last reader.
-      for (int j = 0; j < nmax && ok; ++j) {
-        if (!(ok = acquire(sV))) break;
-        if (j < nt[0] && !(ok = mma_pv(0, j, sV))) break;
-        const bool next = j + 1 < nmax;
-        if (next) {
-          if (!(ok = acquire(sK))) break;
-          if (j + 1 < nt[0]) mma_s(0, sK);
-        }
-        if (j < nt[1] && !(ok = mma_pv(1, j, sV))) break;
-        umma_commit(bar_kv_empty + sV);
-        if (next) {
-          if (j + 1 < nt[1]) mma_s(1, sK);
-          umma_commit(bar_kv_empty + sK);
-        }
+        gb[0] += nt[0];
+        gb[1] += nt[1];
       }
       umma_commit(bar_drain);
       volatile int no_abort = 0;
@@ -418,29 +474,38 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
     const int t = warp >> 2;                        // 0 or 1 (warps 0..7)
     const int w = warp & 3;                         // TMEM lane quarter
     const int row = w * 32 + lane;
-    const int q_tile = q0 + t * BR;
-    const int grow = q_tile + row;
     const uint32_t tl = tmem + t * C::TM_TILE + (uint32_t(w * 32) << 16);
     uint64_t* o_done = bar_o_done + t * 2;
-    RowState st{-INFINITY, 0.f, 0.f};
-    bool ok = nt[t] > 0;
-    for (int j = 0; j < nt[t] && ok; ++j) {
-      ok = mbar_wait(bar_s_full + t, j & 1, abort_flag, p.status, W_S_FULL);
+    int gb = 0;                                     // running block count of this tile
+    bool ok = true;
+    for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
+      int bh, q0, nt[2];
+      unit(u, bh, q0, nt);
+      const int n = nt[t];
+      if (n == 0) continue;
+      const int q_tile = q0 + t * BR;
+      const int grow = q_tile + row;
+      RowState st{-INFINITY, 0.f, 0.f};
+      for (int j = 0; j < n && ok; ++j) {
+        ok = mbar_wait(bar_s_full + t, (gb + j) & 1, abort_flag, p.status, W_S_FULL);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        tc_fence_after();
+        ok = softmax_block<BC, D, CAUSAL>(st, tl, tl + 128, j, gb + j, q_tile, grow, p.Nk,
+                                          p.scale_log2, o_done, abort_flag, p.status);
+        if (!ok) break;
+        mbar_arrive(bar_p_full + t);
+      }
+      if (!ok) break;
+      const int jl = gb + n - 1;
+      ok = mbar_wait(o_done + (jl & 1), (jl >> 1) & 1, abort_flag, p.status, W_O_DONE);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
-      ok = softmax_block<BC, D, CAUSAL>(st, tl, tl + 128, j, q_tile, grow, p.Nk, p.scale_log2,
-                                        o_done, abort_flag, p.status);
-      if (!ok) break;
-      mbar_arrive(bar_p_full + t);
-    }
-    if (ok) {
-      const int jl = nt[t] - 1;
-      ok = mbar_wait(o_done + (jl & 1), (jl >> 1) & 1, abort_flag, p.status, W_O_DONE);
-      if (__all_sync(0xffffffffu, ok)) {
-        tc_fence_after();
-        softmax_finish<D>(st, tl + 128, sQ + t * C::Q_BYTES, w, lane, &tmO, q_tile, p.Nq, bh,
-                          p.lse, grow);
-      }
+      softmax_finish<D>(st, tl + 128, sQ + t * C::Q_BYTES, w, lane, &tmO, q_tile, p.Nq, bh,
+                        p.lse, grow);
+      tc_fence_before();
+      mbar_arrive(bar_o_free + t);                  // O has been read out of TMEM
+      if (lane == 0) mbar_arrive(bar_q_free + t);   // this warp's staging boxes were stored
+      gb += n;
     }
   }
 
@@ -647,7 +712,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
       ok = mbar_wait(bar_s_full + (j & 1), (j >> 1) & 1, abort_flag, p.status, W_S_FULL);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
-      ok = softmax_block<BC, D, CAUSAL>(st, tl + C::TM_S + (j & 1) * BC, tl + C::TM_O, j, q_row0,
+      ok = softmax_block<BC, D, CAUSAL>(st, tl + C::TM_S + (j & 1) * BC, tl + C::TM_O, j, j, q_row0,
                                         grow, p.Nk, p.scale_log2, bar_o_done, abort_flag,
                                         p.status);
       if (!ok) break;
