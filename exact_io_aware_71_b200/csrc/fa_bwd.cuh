@@ -15,7 +15,7 @@
 //                   the diagonal ("step" t):
 //                     S^T  = K_j Q_i^T           (TMEM, lanes = keys)
 //                     P^T  = exp2(S^T * scale*log2e - LSE_i*log2e)
-//                     dV_j += P^T dO_i           (P^T read from TMEM as bf16 hi + lo)
+//                     dV_j += P^T dO_i           (P^T from TMEM; bf16 hi + lo for GQA, d=256)
 //                     dP^T = V_j dO_i^T
 //                     dS^T = P^T o (dP^T - D_i)
 //                     dK_j += dS^T Q_i           (dS^T read from TMEM)
@@ -189,6 +189,7 @@ struct BwdParams {
   const float* Dpad;
   const float* Lpad;
   float* dqacc;
+  int split_p;        // dV uses P as bf16 hi + lo (1) or bf16 P alone (0)
   int gsplit;         // CTAs sharing one kv group's query heads (1 = none)
   int hps;            // query heads per CTA: group / gsplit
   float* dkacc;       // fp32 dK / dV partial sums when gsplit > 1
@@ -375,8 +376,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
         // dV += P^T dO  (hi then lo half of P)
         if (!(ok = mbar_wait(bar_p, t & 1, abort_flag, p.status, WB_P))) break;
         tc_fence_after();
-#pragma unroll
-        for (int half = 0; half < 2; ++half)
+        for (int half = 0; half < 1 + p.split_p; ++half)
 #pragma unroll
           for (int kk = 0; kk < BR / 16; ++kk) {
             const uint32_t bo = (dcol0 / 64) * BR * 128 + kk * 2048;
@@ -493,9 +493,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
       // ---- P^T for this key row and the group's 32 queries: hi = bf16(P)
-      // over columns [0,16) of the group's S^T columns, lo = bf16(P - hi)
-      // over [16,32); dV accumulates both, so rounding P to bf16 does not
-      // pile up over the many query rows (and GQA heads) that feed one dV row.
+      // over columns [0,16) of the group's S^T columns and, when split_p,
+      // lo = bf16(P - hi) over [16,32); dV then accumulates both, so rounding
+      // P to bf16 does not pile up over the query rows of a whole GQA group.
       float P[32];
       {
         uint32_t u[32];
@@ -517,18 +517,21 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) P[i] = (i < cstart) ? 0.f : P[i];
         }
-        uint32_t hi[16], lo[16];
+        uint32_t hi[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const uint32_t h = pack_bf16(P[2 * i], P[2 * i + 1]);
-          hi[i] = h;
-          const float2 rem = fadd2(make_float2(P[2 * i], P[2 * i + 1]),
-                                   make_float2(-__uint_as_float(h << 16),
-                                               -__uint_as_float(h & 0xFFFF0000u)));
-          lo[i] = pack_bf16(rem.x, rem.y);
-        }
+        for (int i = 0; i < 16; ++i) hi[i] = pack_bf16(P[2 * i], P[2 * i + 1]);
         FA_TMEM_ST16(tS, hi);
-        FA_TMEM_ST16(tS + 16, lo);
+        if (p.split_p) {
+          uint32_t lo[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float2 rem = fadd2(make_float2(P[2 * i], P[2 * i + 1]),
+                                     make_float2(-__uint_as_float(hi[i] << 16),
+                                                 -__uint_as_float(hi[i] & 0xFFFF0000u)));
+            lo[i] = pack_bf16(rem.x, rem.y);
+          }
+          FA_TMEM_ST16(tS + 16, lo);
+        }
         tmem_wait_st();
       }
       tc_fence_before();
@@ -713,6 +716,11 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
     p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Nq = Nq; p.Nk = Nk; p.Nq_pad = Nq_pad;
     p.group = group;
     p.n_kblocks = n_kblocks;
+    // dV's rounding error from a bf16 P grows with the number of query rows
+    // that weigh heavily on one key: with a GQA group it is multiplied by the
+    // group size, and at d = 256 |dV| is large enough that the output
+    // rounding leaves no room.  There P goes in as hi + lo (one more MMA).
+    p.split_p = (group > 1 || D == 256) ? 1 : 0;
     p.gsplit = gsplit;
     p.hps = group / gsplit;
     p.dkacc = kvacc;
