@@ -10,6 +10,10 @@ from .binding import (  # noqa: F401
     backward,
     fa_bwd,
     fa_bwd_stage,
+    fa_bwd_strided,
+    fa_fwd_strided,
+    FaStrides,
+    strides_of,
     fa_bwd_workspace_size,
     fa_device_status,
     fa_fwd,

@@ -23,12 +23,26 @@ STATUS_NAMES = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED",
 
 # Exported symbols declared in include/fa.h.
 SYMBOLS = ("fa_fwd", "fa_bwd", "fa_bwd_stage", "fa_bwd_workspace_size", "fa_status_string",
-           "fa_device_status", "fa_bwd_noalloc", "fa_debug_inject")
+           "fa_device_status", "fa_bwd_noalloc", "fa_debug_inject", "fa_fwd_strided",
+           "fa_bwd_strided")
 
 # Bytes of the built-in scratch behind fa_bwd_noalloc (FA_NOALLOC_SCRATCH_BYTES).
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
 FA_BWD_ALL, FA_BWD_PRE, FA_BWD_MAIN, FA_BWD_DQ = 0, 1, 2, 3
+
+
+class FaStrides(ctypes.Structure):
+    """fa_strides: element strides (batch, head, row) of a [B, H, N, d] view."""
+    _fields_ = [("batch", ctypes.c_longlong), ("head", ctypes.c_longlong),
+                ("row", ctypes.c_longlong)]
+
+
+def strides_of(t) -> FaStrides:
+    """fa_strides of a torch tensor viewed as [B, H, N, d] with d contiguous."""
+    if t.stride(-1) != 1:
+        raise ValueError("the last (head-dim) axis must be contiguous")
+    return FaStrides(t.stride(0), t.stride(1), t.stride(2))
 
 
 class FaError(RuntimeError):
@@ -55,6 +69,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, vp, sz, vp]
     lib.fa_bwd.restype = i
     lib.fa_bwd_stage.argtypes = [i] + lib.fa_bwd.argtypes
+    sp = ctypes.POINTER(FaStrides)
+    lib.fa_fwd_strided.argtypes = [vp, vp, vp, vp, vp, sp, i, i, i, i, i, i, i, f, vp]
+    lib.fa_fwd_strided.restype = i
+    lib.fa_bwd_strided.argtypes = [vp] * 9 + [sp] + [i] * 7 + [f, vp, sz, vp]
+    lib.fa_bwd_strided.restype = i
     lib.fa_bwd_stage.restype = i
     lib.fa_bwd_noalloc.argtypes = lib.fa_bwd.argtypes[:17] + [vp]
     lib.fa_bwd_noalloc.restype = i
@@ -74,6 +93,19 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
 def fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, stream) -> int:
     return load().fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, int(causal), float(scale),
                          stream)
+
+
+def fa_fwd_strided(q, k, v, o, lse, strides, B, Hq, Hkv, Nq, Nk, d, causal, scale, stream) -> int:
+    arr = (FaStrides * 4)(*strides) if strides is not None else None
+    return load().fa_fwd_strided(q, k, v, o, lse, arr, B, Hq, Hkv, Nq, Nk, d, int(causal),
+                                 float(scale), stream)
+
+
+def fa_bwd_strided(q, k, v, o, lse, dO, dq, dk, dv, strides, B, Hq, Hkv, Nq, Nk, d, causal,
+                   scale, workspace, workspace_bytes, stream) -> int:
+    arr = (FaStrides * 8)(*strides) if strides is not None else None
+    return load().fa_bwd_strided(q, k, v, o, lse, dO, dq, dk, dv, arr, B, Hq, Hkv, Nq, Nk, d,
+                                 int(causal), float(scale), workspace, workspace_bytes, stream)
 
 
 def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, causal, scale,
@@ -128,32 +160,37 @@ def _dims(q, k):
 
 
 def forward(q, k, v, causal: bool, scale: float, out=None, lse=None):
-    """O, LSE for contiguous bf16 CUDA tensors q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d]."""
+    """O, LSE for bf16 CUDA tensors q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d] (any
+    strides with a contiguous last axis, e.g. permuted [B,N,H,d] storage)."""
     import torch
     B, Hq, Hkv, Nq, Nk, d = _dims(q, k)
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty(B, Hq, Nq, dtype=torch.float32, device=q.device)
-    st = fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                B, Hq, Hkv, Nq, Nk, d, causal, scale, _stream_handle())
+    st = fa_fwd_strided(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                        [strides_of(t) for t in (q, k, v, out)], B, Hq, Hkv, Nq, Nk, d, causal,
+                        scale, _stream_handle())
     if st != FA_OK:
-        raise FaError(st, "fa_fwd")
+        raise FaError(st, "fa_fwd_strided")
     return out, lse
 
 
-def backward(q, k, v, o, lse, do, causal: bool, scale: float, workspace=None):
-    """dQ, dK, dV (bf16) for the forward inputs/outputs and dO."""
+def backward(q, k, v, o, lse, do, causal: bool, scale: float, workspace=None, grads=None):
+    """dQ, dK, dV (bf16) for the forward inputs/outputs and dO; gradients
+    take the strides of q, k, v unless `grads` gives the output tensors."""
     import torch
     B, Hq, Hkv, Nq, Nk, d = _dims(q, k)
     need = fa_bwd_workspace_size(B, Hq, Hkv, Nq, Nk, d, causal)
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    st = fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
-                B, Hq, Hkv, Nq, Nk, d, causal, scale, workspace.data_ptr(), workspace.numel(),
-                _stream_handle())
+    dq, dk, dv = grads if grads is not None else (torch.empty_like(q), torch.empty_like(k),
+                                                  torch.empty_like(v))
+    ts = (q, k, v, o, do, dq, dk, dv)
+    st = fa_bwd_strided(*(t.data_ptr() for t in ts[:4]), lse.data_ptr(),
+                        *(t.data_ptr() for t in ts[4:]), [strides_of(t) for t in ts],
+                        B, Hq, Hkv, Nq, Nk, d, causal, scale, workspace.data_ptr(),
+                        workspace.numel(), _stream_handle())
     if st != FA_OK:
-        raise FaError(st, "fa_bwd")
+        raise FaError(st, "fa_bwd_strided")
     return dq, dk, dv

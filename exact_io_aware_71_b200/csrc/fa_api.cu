@@ -15,10 +15,6 @@
 #include "fa.h"
 #include "fa_fwd.cuh"
 
-namespace fa {
-bool make_map_bf16(CUtensorMap* m, const void* base, int d, int rows, int64_t heads,
-                   int box_rows);
-}
 #include "fa_bwd.cuh"
 
 namespace fa {
@@ -32,6 +28,22 @@ using namespace fa;
 // ---------------------------------------------------------------- checks
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+// Element strides of contiguous [B, H, N, d].
+Strides contiguous(int H, int N, int d) {
+  return Strides{(long long)H * N * d, (long long)N * d, (long long)d};
+}
+
+// Each stride positive, a multiple of 8 elements (16 bytes) and below the
+// TMA limit of 2^40 bytes.
+bool strides_ok(const fa_strides* s, int n) {
+  for (int i = 0; i < n; ++i) {
+    const long long v[3] = {s[i].batch, s[i].head, s[i].row};
+    for (long long x : v)
+      if (x <= 0 || (x & 7) != 0 || x >= (1LL << 39)) return false;
+  }
+  return true;
+}
 
 int check_sizes(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale) {
   if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1) return FA_ERR_INVALID_ARG;
@@ -65,17 +77,19 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 }  // namespace
 
-// A [heads, rows, d] bf16 tensor seen as 3-D for TMA, 64-element (128-byte)
-// inner boxes with the 128-byte swizzle; rows outside [0, rows) read as zero.
-bool fa::make_map_bf16(CUtensorMap* m, const void* base, int d, int rows, int64_t heads,
-                   int box_rows) {
+// A bf16 tensor seen as [batch, heads, rows, d] (d contiguous, the other
+// dimensions at element strides st) as a 4-D TMA tensor (d, rows, heads,
+// batch): 64-element (128-byte) inner boxes of box_rows rows, 128-byte
+// swizzle; rows outside [0, rows) read as zero and are not written.
+bool fa::make_map_bf16(CUtensorMap* m, const void* base, int d, int rows, int heads, int batch,
+                       const Strides& st, int box_rows) {
   auto enc = encode_fn();
   if (!enc) return false;
-  cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(rows), cuuint64_t(heads)};
-  cuuint64_t strides[2] = {cuuint64_t(d) * 2, cuuint64_t(rows) * cuuint64_t(d) * 2};
-  cuuint32_t box[3] = {64u, cuuint32_t(box_rows), 1u};
-  cuuint32_t estr[3] = {1u, 1u, 1u};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+  cuuint64_t dims[4] = {cuuint64_t(d), cuuint64_t(rows), cuuint64_t(heads), cuuint64_t(batch)};
+  cuuint64_t strides[3] = {cuuint64_t(st.n) * 2, cuuint64_t(st.h) * 2, cuuint64_t(st.b) * 2};
+  cuuint32_t box[4] = {64u, cuuint32_t(box_rows), 1u, 1u};
+  cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -177,20 +191,26 @@ const char* fa_status_string(int s) {
   }
 }
 
-int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-           int Hkv, int Nq, int Nk, int d, int causal, float scale, cudaStream_t stream) {
-  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+int fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse,
+                   const fa_strides* strides, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                   int causal, float scale, cudaStream_t stream) {
+  if (!q || !k || !v || !o || !lse || !strides) return FA_ERR_INVALID_ARG;
   int st = check_sizes(B, Hq, Hkv, Nq, Nk, d, causal, scale);
   if (st != FA_OK) return st;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(lse))
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(lse) ||
+      !strides_ok(strides, 4))
     return FA_ERR_MISALIGNED;
+  Strides sq{strides[0].batch, strides[0].head, strides[0].row};
+  Strides sk{strides[1].batch, strides[1].head, strides[1].row};
+  Strides sv{strides[2].batch, strides[2].head, strides[2].row};
+  Strides so{strides[3].batch, strides[3].head, strides[3].row};
 
   const int bc = (d == 256) ? 64 : 128;
   CUtensorMap mq, mk, mv, mo;
-  if (!make_map_bf16(&mq, q, d, Nq, int64_t(B) * Hq, 128) ||
-      !make_map_bf16(&mk, k, d, Nk, int64_t(B) * Hkv, bc) ||
-      !make_map_bf16(&mv, v, d, Nk, int64_t(B) * Hkv, bc) ||
-      !make_map_bf16(&mo, o, d, Nq, int64_t(B) * Hq, 32))
+  if (!make_map_bf16(&mq, q, d, Nq, Hq, B, sq, 128) ||
+      !make_map_bf16(&mk, k, d, Nk, Hkv, B, sk, bc) ||
+      !make_map_bf16(&mv, v, d, Nk, Hkv, B, sv, bc) ||
+      !make_map_bf16(&mo, o, d, Nq, Hq, B, so, 32))
     return FA_ERR_CUDA;
 
   FwdParams p;
@@ -211,15 +231,29 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
                 : launch_fwd<256, false>(mq, mk, mv, mo, p, stream);
 }
 
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+           int Hkv, int Nq, int Nk, int d, int causal, float scale, cudaStream_t stream) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1) return FA_ERR_INVALID_ARG;
+  const Strides a = contiguous(Hq, Nq, d), b = contiguous(Hkv, Nk, d);
+  const fa_strides s[4] = {{a.b, a.h, a.n}, {b.b, b.h, b.n}, {b.b, b.h, b.n}, {a.b, a.h, a.n}};
+  return fa_fwd_strided(q, k, v, o, lse, s, B, Hq, Hkv, Nq, Nk, d, causal, scale, stream);
+}
+
 size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal) {
   if (check_sizes(B, Hq, Hkv, Nq, Nk, d, causal, 1.0f) != FA_OK) return 0;
   return bwd_workspace_bytes(B, Hq, Hkv, Nq, Nk, d);
 }
 
-int fa_bwd_stage(int stage, const void* q, const void* k, const void* v, const void* o,
-                 const float* lse, const void* dO, void* dq, void* dk, void* dv, int B, int Hq,
-                 int Hkv, int Nq, int Nk, int d, int causal, float scale, void* workspace,
-                 size_t workspace_bytes, cudaStream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// The backward pass on strided tensors, stage by stage (see fa_bwd_stage).
+int bwd_impl(int stage, const void* q, const void* k, const void* v, const void* o,
+             const float* lse, const void* dO, void* dq, void* dk, void* dv,
+             const fa_strides* strides, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+             int causal, float scale, void* workspace, size_t workspace_bytes,
+             cudaStream_t stream) {
   int stages;
   switch (stage) {
     case FA_BWD_ALL: stages = 7; break;
@@ -228,19 +262,53 @@ int fa_bwd_stage(int stage, const void* q, const void* k, const void* v, const v
     case FA_BWD_DQ: stages = 4; break;
     default: return FA_ERR_INVALID_ARG;
   }
-  if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv || !strides)
+    return FA_ERR_INVALID_ARG;
   int st = check_sizes(B, Hq, Hkv, Nq, Nk, d, causal, scale);
   if (st != FA_OK) return st;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(lse) ||
-      !aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+      !aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      !strides_ok(strides, 8))
     return FA_ERR_MISALIGNED;
   const size_t need = bwd_workspace_bytes(B, Hq, Hkv, Nq, Nk, d);
   if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
   DevStatus* sp = status_ptr();
   if (!sp) return FA_ERR_CUDA;
-  return launch_bwd(stages, q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, causal,
+  Strides s8[8];
+  for (int i = 0; i < 8; ++i) s8[i] = Strides{strides[i].batch, strides[i].head, strides[i].row};
+  return launch_bwd(stages, q, k, v, o, lse, dO, dq, dk, dv, s8, B, Hq, Hkv, Nq, Nk, d, causal,
                     scale, workspace, sp, stream);
+}
+
+void contiguous8(fa_strides* s, int Hq, int Hkv, int Nq, int Nk, int d) {
+  const Strides a = contiguous(Hq, Nq, d), b = contiguous(Hkv, Nk, d);
+  const fa_strides qa{a.b, a.h, a.n}, kb{b.b, b.h, b.n};
+  // q, k, v, o, dO, dq, dk, dv
+  s[0] = qa; s[1] = kb; s[2] = kb; s[3] = qa; s[4] = qa; s[5] = qa; s[6] = kb; s[7] = kb;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_bwd_strided(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                   const void* dO, void* dq, void* dk, void* dv, const fa_strides* strides, int B,
+                   int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale,
+                   void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  return bwd_impl(FA_BWD_ALL, q, k, v, o, lse, dO, dq, dk, dv, strides, B, Hq, Hkv, Nq, Nk, d,
+                  causal, scale, workspace, workspace_bytes, stream);
+}
+
+int fa_bwd_stage(int stage, const void* q, const void* k, const void* v, const void* o,
+                 const float* lse, const void* dO, void* dq, void* dk, void* dv, int B, int Hq,
+                 int Hkv, int Nq, int Nk, int d, int causal, float scale, void* workspace,
+                 size_t workspace_bytes, cudaStream_t stream) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1) return FA_ERR_INVALID_ARG;
+  fa_strides s[8];
+  contiguous8(s, Hq, Hkv, Nq, Nk, d);
+  return bwd_impl(stage, q, k, v, o, lse, dO, dq, dk, dv, s, B, Hq, Hkv, Nq, Nk, d, causal,
+                  scale, workspace, workspace_bytes, stream);
 }
 
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,

@@ -94,12 +94,17 @@ inline size_t bwd_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d)
 // ------------------------------------------------------------------ pre
 // One group of D/8 threads per row; each thread handles 8 consecutive
 // elements (16 bytes) of O and dO and zeroes 8 floats of dQacc.
+// Element strides (batch, head, row) of a [B, H, N, d] view; d contiguous.
+struct Strides {
+  long long b, h, n;
+};
+
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(
     const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
     const float* __restrict__ lse, float* __restrict__ dqacc, float* __restrict__ Dpad,
-    float* __restrict__ Lpad, int rows_bh, int Nq, int Nq_pad, float* __restrict__ kvacc,
-    long long kv_n4) {
+    float* __restrict__ Lpad, int rows_bh, int Hq, int Nq, int Nq_pad, Strides so, Strides sdo,
+    float* __restrict__ kvacc, long long kv_n4) {
   constexpr int TPR = D / 8;                       // threads per row
   constexpr int RPB = 256 / TPR;                   // rows per block pass
   const int sub = threadIdx.x % TPR;
@@ -113,8 +118,11 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(
     const bool valid = q < Nq;
     if (valid) {
       const size_t e = (size_t(bh) * Nq + q) * D + sub * 8;
-      const uint4 ov = *reinterpret_cast<const uint4*>(o + e);
-      const uint4 dv = *reinterpret_cast<const uint4*>(dO + e);
+      const long long bb = bh / Hq, hh = bh - bb * Hq;
+      const uint4 ov = *reinterpret_cast<const uint4*>(o + bb * so.b + hh * so.h + q * so.n +
+                                                       sub * 8);
+      const uint4 dv = *reinterpret_cast<const uint4*>(dO + bb * sdo.b + hh * sdo.h +
+                                                       q * sdo.n + sub * 8);
       const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
       const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
 #pragma unroll
@@ -143,13 +151,20 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(
 }
 
 // dk, dv = bf16 of the fp32 partial-sum accumulators (dK already scaled).
+template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_kv_kernel(const float* __restrict__ kvacc,
                                                         __nv_bfloat16* __restrict__ dk,
                                                         __nv_bfloat16* __restrict__ dv,
-                                                        long long n8) {
+                                                        long long n8, int Hkv, int Nk,
+                                                        Strides sdk, Strides sdv) {
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < 2 * n8;
        i += (long long)gridDim.x * blockDim.x) {
-    const long long j = i < n8 ? i : i - n8;
+    const long long j = i < n8 ? i : i - n8;       // 8-element chunk of [B*Hkv, Nk, D]
+    const long long row = j / (D / 8), c8 = j - row * (D / 8);
+    const long long bh = row / Nk, n = row - bh * Nk;
+    const long long bb = bh / Hkv, hh = bh - bb * Hkv;
+    const Strides& so = i < n8 ? sdk : sdv;
+    const long long dst = bb * so.b + hh * so.h + n * so.n + c8 * 8;
     const float4 a = reinterpret_cast<const float4*>(kvacc)[2 * i];
     const float4 b = reinterpret_cast<const float4*>(kvacc)[2 * i + 1];
     uint4 out;
@@ -157,16 +172,21 @@ __global__ void __launch_bounds__(256) fa_bwd_kv_kernel(const float* __restrict_
     out.y = pack_bf16(a.z, a.w);
     out.z = pack_bf16(b.x, b.y);
     out.w = pack_bf16(b.z, b.w);
-    reinterpret_cast<uint4*>(i < n8 ? dk : dv)[j] = out;
+    *reinterpret_cast<uint4*>((i < n8 ? dk : dv) + dst) = out;
   }
 }
 
 // ------------------------------------------------------------------ dq convert
+template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const float* __restrict__ dqacc,
                                                         __nv_bfloat16* __restrict__ dq,
-                                                        long long n8, float scale) {
+                                                        long long n8, float scale, int Hq, int Nq,
+                                                        Strides sdq) {
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
        i += (long long)gridDim.x * blockDim.x) {
+    const long long row = i / (D / 8), c8 = i - row * (D / 8);
+    const long long bh = row / Nq, n = row - bh * Nq;
+    const long long bb = bh / Hq, hh = bh - bb * Hq;
     const float4 a = reinterpret_cast<const float4*>(dqacc)[2 * i];
     const float4 b = reinterpret_cast<const float4*>(dqacc)[2 * i + 1];
     uint4 out;
@@ -174,7 +194,7 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const float* __restrict_
     out.y = pack_bf16(a.z * scale, a.w * scale);
     out.z = pack_bf16(b.x * scale, b.y * scale);
     out.w = pack_bf16(b.z * scale, b.w * scale);
-    reinterpret_cast<uint4*>(dq)[i] = out;
+    *reinterpret_cast<uint4*>(dq + bb * sdq.b + hh * sdq.h + n * sdq.n + c8 * 8) = out;
   }
 }
 
@@ -306,8 +326,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
       prefetch_tmap(&tmdO);
       mbar_arrive_expect_tx(bar_kv, 2 * C::K_BYTES);
       for (int c = 0; c < C::KCH; ++c) {
-        tma_load_3d(sK + c * BC * 128, &tmK, bar_kv, c * 64, key0, bkv);
-        tma_load_3d(sV + c * BC * 128, &tmV, bar_kv, c * 64, key0, bkv);
+        tma_load_bh(sK + c * BC * 128, &tmK, bar_kv, c * 64, key0, bkv, p.Hkv);
+        tma_load_bh(sV + c * BC * 128, &tmV, bar_kv, c * 64, key0, bkv, p.Hkv);
       }
       int issued = 0;
       for (int t = 0; t < n_steps; ++t) {
@@ -323,8 +343,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
         float* sd = sl + BR;
         mbar_arrive_expect_tx(bar_qfull + st, C::STAGE_BYTES);
         for (int c = 0; c < C::KCH; ++c) {
-          tma_load_3d(sq + c * BR * 128, &tmQ, bar_qfull + st, c * 64, qi * BR, bh);
-          tma_load_3d(sdo + c * BR * 128, &tmdO, bar_qfull + st, c * 64, qi * BR, bh);
+          tma_load_bh(sq + c * BR * 128, &tmQ, bar_qfull + st, c * 64, qi * BR, bh, p.Hq);
+          tma_load_bh(sdo + c * BR * 128, &tmdO, bar_qfull + st, c * 64, qi * BR, bh, p.Hq);
         }
         const size_t ro = size_t(bh) * p.Nq_pad + size_t(qi) * BR;
         bulk_load_1d(sl, p.Lpad + ro, BR * 4, bar_qfull + st);
@@ -641,7 +661,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
       if (lane == 0 && key0 + w * 32 < p.Nk) {
         const CUtensorMap* tm = g == 0 ? &tmdK : &tmdV;
         for (int c = 0; c < DH / 64; ++c)
-          tma_store_3d(tm, stage + (c * 4 + w) * 4096, dcol0 + c * 64, key0 + w * 32, bkv);
+          tma_store_bh(tm, stage + (c * 4 + w) * 4096, dcol0 + c * 64, key0 + w * 32, bkv, p.Hkv);
         bulk_commit();
         bulk_wait0();
       }
@@ -657,13 +677,14 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
 }
 
 // ------------------------------------------------------------------ launch
-bool make_map_bf16(CUtensorMap* m, const void* base, int d, int rows, int64_t heads, int box_rows);
+bool make_map_bf16(CUtensorMap* m, const void* base, int d, int rows, int heads, int batch,
+                   const Strides& st, int box_rows);
 
 template <int D, bool CAUSAL>
 int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const void* o,
-                 const float* lse, const void* dO, void* dq, void* dk, void* dv, int B, int Hq,
-                 int Hkv, int Nq, int Nk, float scale, void* workspace, DevStatus* status,
-                 cudaStream_t stream) {
+                 const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                 const Strides* st, int B, int Hq, int Hkv, int Nq, int Nk, float scale,
+                 void* workspace, DevStatus* status, cudaStream_t stream) {
   using C = BwdCfg<D>;
   const BwdWorkspace w = bwd_workspace_layout(B, Hq, Hkv, Nq, Nk, D);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -690,12 +711,13 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
   }
 
   CUtensorMap mq, mk, mv, mdo, mdk, mdv;
-  if ((stages & 2) && (!make_map_bf16(&mq, q, D, Nq, int64_t(bhq), C::BR) ||
-      !make_map_bf16(&mk, k, D, Nk, int64_t(B) * Hkv, C::BC) ||
-      !make_map_bf16(&mv, v, D, Nk, int64_t(B) * Hkv, C::BC) ||
-      !make_map_bf16(&mdo, dO, D, Nq, int64_t(bhq), C::BR) ||
-      !make_map_bf16(&mdk, dk, D, Nk, int64_t(B) * Hkv, 32) ||
-      !make_map_bf16(&mdv, dv, D, Nk, int64_t(B) * Hkv, 32)))
+  // strides: q, k, v, o, dO, dq, dk, dv
+  if ((stages & 2) && (!make_map_bf16(&mq, q, D, Nq, Hq, B, st[0], C::BR) ||
+      !make_map_bf16(&mk, k, D, Nk, Hkv, B, st[1], C::BC) ||
+      !make_map_bf16(&mv, v, D, Nk, Hkv, B, st[2], C::BC) ||
+      !make_map_bf16(&mdo, dO, D, Nq, Hq, B, st[4], C::BR) ||
+      !make_map_bf16(&mdk, dk, D, Nk, Hkv, B, st[6], 32) ||
+      !make_map_bf16(&mdv, dv, D, Nk, Hkv, B, st[7], 32)))
     return 5;
 
   if (stages & 1) {
@@ -704,7 +726,8 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
     const long long blocks = std::min<long long>((rows + RPB - 1) / RPB, 148LL * 16);
     fa_bwd_pre_kernel<D><<<unsigned(blocks), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, dqacc,
-        Dpad, Lpad, bhq, Nq, Nq_pad, kvacc, gsplit > 1 ? (long long)(2 * w.kv_elems / 4) : 0LL);
+        Dpad, Lpad, bhq, Hq, Nq, Nq_pad, st[3], st[4], kvacc,
+        gsplit > 1 ? (long long)(2 * w.kv_elems / 4) : 0LL);
     if (cudaGetLastError() != cudaSuccess) return 5;
   }
   if (stages & 2) {
@@ -739,14 +762,15 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
   if (stages & 4) {
     const long long n8 = (long long)bhq * Nq * D / 8;
     const long long blocks = std::min<long long>((n8 + 255) / 256, 148LL * 16);
-    fa_bwd_dq_kernel<<<unsigned(blocks), 256, 0, stream>>>(
-        dqacc, static_cast<__nv_bfloat16*>(dq), n8, scale);
+    fa_bwd_dq_kernel<D><<<unsigned(blocks), 256, 0, stream>>>(
+        dqacc, static_cast<__nv_bfloat16*>(dq), n8, scale, Hq, Nq, st[5]);
     if (cudaGetLastError() != cudaSuccess) return 5;
     if (gsplit > 1) {
       const long long kv8 = (long long)w.kv_elems / 8;
       const long long kblocks = std::min<long long>((2 * kv8 + 255) / 256, 148LL * 16);
-      fa_bwd_kv_kernel<<<unsigned(kblocks), 256, 0, stream>>>(
-          kvacc, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), kv8);
+      fa_bwd_kv_kernel<D><<<unsigned(kblocks), 256, 0, stream>>>(
+          kvacc, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), kv8, Hkv, Nk,
+          st[6], st[7]);
       if (cudaGetLastError() != cudaSuccess) return 5;
     }
   }
@@ -755,14 +779,15 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
 
 // stages: bit 0 = preprocess, bit 1 = main, bit 2 = dq convert.
 inline int launch_bwd(int stages, const void* q, const void* k, const void* v, const void* o,
-                      const float* lse, const void* dO, void* dq, void* dk, void* dv, int B,
-                      int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale,
-                      void* workspace, DevStatus* status, cudaStream_t stream) {
-#define FA_BWD_CASE(DD)                                                                        \
-  if (d == DD)                                                                                 \
-    return causal ? launch_bwd_t<DD, true>(stages, q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, \
-                                           Nq, Nk, scale, workspace, status, stream)           \
-                  : launch_bwd_t<DD, false>(stages, q, k, v, o, lse, dO, dq, dk, dv, B, Hq,    \
+                      const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                      const Strides* st, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                      int causal, float scale, void* workspace, DevStatus* status,
+                      cudaStream_t stream) {
+#define FA_BWD_CASE(DD)                                                                          \
+  if (d == DD)                                                                                   \
+    return causal ? launch_bwd_t<DD, true>(stages, q, k, v, o, lse, dO, dq, dk, dv, st, B, Hq,  \
+                                           Hkv, Nq, Nk, scale, workspace, status, stream)       \
+                  : launch_bwd_t<DD, false>(stages, q, k, v, o, lse, dO, dq, dk, dv, st, B, Hq, \
                                             Hkv, Nq, Nk, scale, workspace, status, stream);
   FA_BWD_CASE(64)
   FA_BWD_CASE(128)

@@ -172,7 +172,7 @@ __device__ __forceinline__ bool softmax_block(RowState& st, uint32_t tS, uint32_
 template <int D>
 __device__ __forceinline__ void softmax_finish(const RowState& st, uint32_t tO, uint8_t* stage,
                                                int w, int lane, const CUtensorMap* tmO,
-                                               int q_tile, int Nq, int bh, float* lse,
+                                               int q_tile, int Nq, int bh, int H, float* lse,
                                                int grow) {
   const float inv = 1.0f / st.lr;
 #pragma unroll
@@ -196,7 +196,7 @@ __device__ __forceinline__ void softmax_finish(const RowState& st, uint32_t tO, 
   __syncwarp();
   if (lane == 0 && q_tile + w * 32 < Nq) {
     for (int c = 0; c < D / 64; ++c)
-      tma_store_3d(tmO, stage + (c * 4 + w) * 4096, c * 64, q_tile + w * 32, bh);
+      tma_store_bh(tmO, stage + (c * 4 + w) * 4096, c * 64, q_tile + w * 32, bh, H);
     bulk_commit();
     bulk_wait0();
   }
@@ -346,7 +346,8 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
           uint8_t* dst = sKV + slot * C::KV_BYTES;
           const CUtensorMap* tm = (item & 1) ? &tmV : &tmK;
           for (int c = 0; c < C::KCH; ++c)
-            tma_load_3d(dst + c * BC * 128, tm, bar_kv_full + slot, c * 64, (item >> 1) * BC, bkv);
+            tma_load_bh(dst + c * BC * 128, tm, bar_kv_full + slot, c * 64, (item >> 1) * BC, bkv,
+                        p.Hkv);
           ++cnt;
           return true;
         };
@@ -359,8 +360,8 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
             break;
           mbar_arrive_expect_tx(bar_q + t, C::Q_BYTES);
           for (int c = 0; c < C::KCH; ++c)
-            tma_load_3d(sQ + t * C::Q_BYTES + c * BR * 128, &tmQ, bar_q + t, c * 64,
-                        q0 + t * BR, bh);
+            tma_load_bh(sQ + t * C::Q_BYTES + c * BR * 128, &tmQ, bar_q + t, c * 64,
+                        q0 + t * BR, bh, p.Hq);
           ++uses[t];
         }
         for (int it = early; it < items && ok; ++it) ok = ring(it);
@@ -500,7 +501,7 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
       ok = mbar_wait(o_done + (jl & 1), (jl >> 1) & 1, abort_flag, p.status, W_O_DONE);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
-      softmax_finish<D>(st, tl + 128, sQ + t * C::Q_BYTES, w, lane, &tmO, q_tile, p.Nq, bh,
+      softmax_finish<D>(st, tl + 128, sQ + t * C::Q_BYTES, w, lane, &tmO, q_tile, p.Nq, bh, p.Hq,
                         p.lse, grow);
       tc_fence_before();
       mbar_arrive(bar_o_free + t);                  // O has been read out of TMEM
@@ -604,7 +605,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
       prefetch_tmap(&tmV);
       mbar_arrive_expect_tx(bar_q, C::Q_BYTES);
       for (int c = 0; c < C::KCH; ++c)
-        tma_load_3d(sQ + c * BR * 128, &tmQ, bar_q, c * 64, q_row0, bh);
+        tma_load_bh(sQ + c * BR * 128, &tmQ, bar_q, c * 64, q_row0, bh, p.Hq);
       int cnt = 0;
       bool ok = !p.status->stall_kv;   // test control: withhold K/V (see fa_debug_inject)
       auto load = [&](const CUtensorMap* tm, int j) {
@@ -617,7 +618,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
         mbar_arrive_expect_tx(bar_kv_full + slot, C::KV_BYTES);
         uint8_t* dst = sKV + slot * C::KV_BYTES;
         for (int c = 0; c < C::KCH; ++c)
-          tma_load_3d(dst + c * BC * 128, tm, bar_kv_full + slot, c * 64, j * BC, bkv);
+          tma_load_bh(dst + c * BC * 128, tm, bar_kv_full + slot, c * 64, j * BC, bkv, p.Hkv);
         ++cnt;
       };
       // Ring order = MMA consumption order: K0, K1, V0, K2, V1, ...
@@ -723,7 +724,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
       ok = mbar_wait(bar_o_done + (jl & 1), (jl >> 1) & 1, abort_flag, p.status, W_O_DONE);
       if (__all_sync(0xffffffffu, ok)) {
         tc_fence_after();
-        softmax_finish<D>(st, tl + C::TM_O, sQ, warp, lane, &tmO, q_row0, p.Nq, bh, p.lse, grow);
+        softmax_finish<D>(st, tl + C::TM_O, sQ, warp, lane, &tmO, q_row0, p.Nq, bh, p.Hq, p.lse,
+                          grow);
       }
     }
   }

@@ -124,6 +124,33 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* m, const void* s
       : "memory");
 }
 
+// 4-D tile copies over a (d, rows, heads, batch) view; callers pass the
+// (batch * heads + head) index and the head count.
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* m, uint64_t* bar,
+                                            int c0, int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* m, const void* src, int c0,
+                                             int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(m)),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_bh(void* dst, const CUtensorMap* m, uint64_t* bar, int x,
+                                            int row, int bh, int H) {
+  tma_load_4d(dst, m, bar, x, row, bh % H, bh / H);
+}
+__device__ __forceinline__ void tma_store_bh(const CUtensorMap* m, const void* src, int x, int row,
+                                             int bh, int H) {
+  tma_store_4d(m, src, x, row, bh % H, bh / H);
+}
+
 __device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* m, const void* src, int c0,
                                                   int c1, int c2) {
   asm volatile(

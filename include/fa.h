@@ -43,11 +43,22 @@
 extern "C" {
 #endif
 
+/*
+ * Element strides of a tensor seen as [B, H, N, d] with d contiguous
+ * (stride 1).  Contiguous [B, H, N, d] is {H*N*d, N*d, d}; [B, N, H, d] is
+ * {N*H*d, d, H*d}; q, k, v taken from one packed [B, N, 3, H, d] tensor use
+ * {N*3*H*d, d, 3*H*d} with base pointers offset by 0, H*d and 2*H*d.  Each
+ * stride must be a positive multiple of 8 elements (16 bytes, a TMA rule).
+ */
+typedef struct {
+  long long batch, head, row;
+} fa_strides;
+
 typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID_ARG = 1,    /* null pointer, size < 1, Hq % Hkv != 0, bad scale */
   FA_ERR_UNSUPPORTED = 2,    /* d not in {64, 128, 256}, or sizes beyond int range */
-  FA_ERR_MISALIGNED = 3,     /* a pointer breaks the alignment rule above */
+  FA_ERR_MISALIGNED = 3,     /* a pointer or stride breaks the alignment rules above */
   FA_ERR_WORKSPACE = 4,      /* workspace null or smaller than fa_bwd_workspace_size() */
   FA_ERR_CUDA = 5,           /* a CUDA runtime/driver call or launch failed */
   FA_ERR_DEVICE_TIMEOUT = 6, /* a kernel gave up on a pipeline wait (see fa_device_status) */
@@ -64,6 +75,15 @@ typedef enum {
  */
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
            int Hkv, int Nq, int Nk, int d, int causal, float scale, cudaStream_t stream);
+
+/*
+ * Forward pass on strided tensors (layouts such as [B, N, H, d] or views of
+ * a packed QKV tensor; see fa_strides).  strides[0..3] describe q, k, v, o.
+ * lse stays contiguous [B, Hq, Nq].  Otherwise identical to fa_fwd.
+ */
+int fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse,
+                   const fa_strides* strides, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                   int causal, float scale, cudaStream_t stream);
 
 /*
  * Bytes of caller-owned device workspace fa_bwd needs for these sizes: the
@@ -84,6 +104,16 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
            const void* dO, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nk,
            int d, int causal, float scale, void* workspace, size_t workspace_bytes,
            cudaStream_t stream);
+
+/*
+ * Backward pass on strided tensors.  strides[0..7] describe q, k, v, o, dO,
+ * dq, dk, dv (see fa_strides); lse is contiguous [B, Hq, Nq].  The workspace
+ * is the same as for fa_bwd.  Otherwise identical to fa_bwd.
+ */
+int fa_bwd_strided(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                   const void* dO, void* dq, void* dk, void* dv, const fa_strides* strides, int B,
+                   int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale,
+                   void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* Stages of fa_bwd, for callers that time or schedule them separately. */
 typedef enum {

@@ -81,6 +81,31 @@ def test_bwd_stage_rejects_unknown_stage(stage):
     assert fa.fa_bwd_stage(stage, **a) == 1
 
 
+@pytest.mark.parametrize("bad,status", [
+    ({"s0": ("row", 4)}, 3), ({"s1": ("head", 0)}, 3), ({"s3": ("batch", -64)}, 3),
+    ({"s2": ("row", 1 << 40)}, 3),
+])
+def test_strided_rejects_bad_strides(bad, status):
+    b = {k: v for k, v in bad.items()}
+    s4 = [binding.FaStrides(1 << 20, 1 << 14, 64) for _ in range(4)]
+    for key, (field, val) in b.items():
+        setattr(s4[int(key[1:])], field, val)
+    st = fa.fa_fwd_strided(A, A, A, A, A, s4, 1, 2, 2, 128, 128, 64, 0, 0.125, None)
+    assert st == status
+    s8 = [binding.FaStrides(1 << 20, 1 << 14, 64) for _ in range(8)]
+    for key, (field, val) in b.items():
+        setattr(s8[int(key[1:])], field, val)
+    st = fa.fa_bwd_strided(A, A, A, A, A, A, A, A, A, s8, 1, 2, 2, 128, 128, 64, 0, 0.125, A,
+                           1 << 40, None)
+    assert st == status
+
+
+def test_strided_rejects_null_strides():
+    assert fa.fa_fwd_strided(A, A, A, A, A, None, 1, 2, 2, 128, 128, 64, 0, 0.125, None) == 1
+    assert fa.fa_bwd_strided(A, A, A, A, A, A, A, A, A, None, 1, 2, 2, 128, 128, 64, 0, 0.125,
+                             A, 1 << 40, None) == 1
+
+
 def test_workspace_size():
     assert fa.fa_bwd_workspace_size(1, 2, 2, 128, 128, 64, 0) > 0
     assert fa.fa_bwd_workspace_size(0, 2, 2, 128, 128, 64, 0) == 0
