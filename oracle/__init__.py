@@ -6,6 +6,7 @@ Every function is pinned by the ``-m "not gpu"`` tests in
 ``tests/test_oracle.py``; no function here is "parity unpinned".
 """
 from .attention import (  # noqa: F401
+    BLOCK,
     attention_backward,
     attention_backward_dq_rows,
     attention_forward,

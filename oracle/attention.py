@@ -39,6 +39,12 @@ Readings where the pages are silent (all listed in the design notes):
     "two small changes") maps query head h to kv head h // (Hq // Hkv).
   * Causal masking is top-left aligned: key j is visible to query i iff j <= i.
   * LSE is the natural-log logsumexp of the *scaled* scores.
+  * Block-sparse attention (QbitAI FA1 article, results section, names
+    block-sparse FlashAttention without defining it) takes a block mask of
+    128 x 128 (query, key) blocks, shared by all batches and heads; a zero
+    entry sets the block's scores to -inf, on top of the causal mask.  A row
+    that sees no key at all gets O = 0, LSE = -inf and no gradient (the
+    limits of an empty softmax).
 
 Rows of the score matrix are independent (FA2 post, section "Параллелизм":
 forward rows are independent), so processing query rows in chunks is exact;
@@ -49,6 +55,7 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = [
+    "BLOCK",
     "kv_head",
     "scores",
     "attention_forward",
@@ -73,24 +80,39 @@ def _as64(x) -> np.ndarray:
     return np.asarray(x, dtype=np.float64)
 
 
+# Block-sparse attention (QbitAI FA1 article, results section: block-sparse
+# FlashAttention): a query row sees key j only where the (query block, key
+# block) entry of a block mask is non-zero; blocks are BLOCK x BLOCK.
+BLOCK = 128
+
+
 def scores(q_rows: np.ndarray, k: np.ndarray, scale: float, causal: bool,
-           row_index: np.ndarray) -> np.ndarray:
+           row_index: np.ndarray, block_mask=None) -> np.ndarray:
     """Scaled, masked score rows S[r, j] for the query rows ``row_index``.
 
     q_rows: [R, d] (the rows themselves), k: [Nk, d], row_index: [R] absolute
-    query positions (needed for the causal mask)."""
+    query positions (needed for the causal and block masks)."""
     s = scale * (q_rows @ k.T)
+    j = np.arange(k.shape[0])[None, :]
     if causal:
-        j = np.arange(k.shape[0])[None, :]
         s = np.where(j > row_index[:, None], -np.inf, s)
+    if block_mask is not None:
+        bm = np.asarray(block_mask) != 0
+        visible = bm[(row_index // BLOCK)[:, None], j // BLOCK]
+        s = np.where(visible, s, -np.inf)
     return s
 
 
 def _softmax_stats(s: np.ndarray):
-    """Row max-shifted logsumexp and the normalised probabilities."""
+    """Row max-shifted logsumexp and the normalised probabilities.  A row with
+    no visible key has LSE = -inf and P = 0 (so O = 0 and no gradient)."""
     m = s.max(axis=1)
-    lse = m + np.log(np.exp(s - m[:, None]).sum(axis=1))
-    p = np.exp(s - lse[:, None])
+    empty = ~np.isfinite(m)
+    m_safe = np.where(empty, 0.0, m)
+    with np.errstate(divide="ignore"):
+        lse = m_safe + np.log(np.exp(s - m_safe[:, None]).sum(axis=1))
+    lse = np.where(empty, -np.inf, lse)
+    p = np.where(empty[:, None], 0.0, np.exp(s - np.where(empty, 0.0, lse)[:, None]))
     return lse, p
 
 
@@ -98,11 +120,12 @@ def _chunk_rows(nq: int, nk: int) -> int:
     return max(1, min(nq, _MAX_CHUNK_ELEMS // max(1, nk)))
 
 
-def attention_forward(q, k, v, causal: bool, scale: float):
+def attention_forward(q, k, v, causal: bool, scale: float, block_mask=None):
     """Exact attention forward.
 
     q: [B, Hq, Nq, d]; k, v: [B, Hkv, Nk, d] (any float dtype; upcast to fp64).
-    Returns (O [B, Hq, Nq, d] fp64, LSE [B, Hq, Nq] fp64)."""
+    block_mask: optional [ceil(Nq/BLOCK), ceil(Nk/BLOCK)], shared by all
+    batches and heads.  Returns (O [B, Hq, Nq, d] fp64, LSE [B, Hq, Nq] fp64)."""
     q, k, v = _as64(q), _as64(k), _as64(v)
     b_, hq, nq, d = q.shape
     hkv, nk = k.shape[1], k.shape[2]
@@ -114,7 +137,7 @@ def attention_forward(q, k, v, causal: bool, scale: float):
             kvh = kv_head(h, hq, hkv)
             for r0 in range(0, nq, step):
                 rows = np.arange(r0, min(nq, r0 + step))
-                s = scores(q[b, h, rows], k[b, kvh], scale, causal, rows)
+                s = scores(q[b, h, rows], k[b, kvh], scale, causal, rows, block_mask)
                 l_, p = _softmax_stats(s)
                 lse[b, h, rows] = l_
                 o[b, h, rows] = p @ v[b, kvh]
@@ -122,7 +145,7 @@ def attention_forward(q, k, v, causal: bool, scale: float):
 
 
 def attention_forward_rows(q, k, v, causal: bool, scale: float, b: int, h: int,
-                           rows):
+                           rows, block_mask=None):
     """O and LSE of selected query rows of one (batch, head).
 
     Exact for any subset because forward rows are independent.
@@ -133,13 +156,13 @@ def attention_forward_rows(q, k, v, causal: bool, scale: float, b: int, h: int,
     qr = _as64(q[b, h, rows])
     kk = _as64(k[b, kvh])
     vv = _as64(v[b, kvh])
-    s = scores(qr, kk, scale, causal, rows)
+    s = scores(qr, kk, scale, causal, rows, block_mask)
     l_, p = _softmax_stats(s)
     return p @ vv, l_
 
 
 def attention_backward(q, k, v, do, causal: bool, scale: float,
-                       heads=None, return_aux: bool = False):
+                       heads=None, return_aux: bool = False, block_mask=None):
     """Exact attention backward by the chain rule on the materialised P.
 
     q, do: [B, Hq, Nq, d]; k, v: [B, Hkv, Nk, d].
@@ -169,7 +192,7 @@ def attention_backward(q, k, v, do, causal: bool, scale: float,
             for r0 in range(0, nq, step):
                 rows = np.arange(r0, min(nq, r0 + step))
                 qh, doh = q[b, h, rows], do[b, h, rows]
-                s = scores(qh, kk, scale, causal, rows)
+                s = scores(qh, kk, scale, causal, rows, block_mask)
                 l_, p = _softmax_stats(s)
                 dv_acc += p.T @ doh
                 dp = doh @ vv.T
@@ -188,7 +211,7 @@ def attention_backward(q, k, v, do, causal: bool, scale: float,
 
 
 def attention_backward_dq_rows(q, k, v, do, causal: bool, scale: float, b: int, h: int,
-                               rows):
+                               rows, block_mask=None):
     """dQ of selected query rows of one (batch, head).
 
     Row i of dQ needs only row i of P and dP (D_i is a sum over that row), so
@@ -198,7 +221,7 @@ def attention_backward_dq_rows(q, k, v, do, causal: bool, scale: float, b: int, 
     rows = np.asarray(rows, dtype=np.int64)
     qr, dor = _as64(q[b, h, rows]), _as64(do[b, h, rows])
     kk, vv = _as64(k[b, kvh]), _as64(v[b, kvh])
-    s = scores(qr, kk, scale, causal, rows)
+    s = scores(qr, kk, scale, causal, rows, block_mask)
     _, p = _softmax_stats(s)
     dp = dor @ vv.T
     d_row = (p * dp).sum(axis=1)
