@@ -13,6 +13,12 @@ steps between a barrier + synchronize on both sides, CUDA events on the
 launching stream, max over ranks.  Inputs (448 MiB read per step) exceed
 the 126 MB L2, so no flush is needed between steps.
 
+``--block-density P`` measures block-sparse attention instead (QbitAI FA1
+article, results section): a seeded block mask keeps each 128 x 128 (query,
+key) block with probability P (diagonal blocks always), the step is
+fa_fwd_block_sparse + fa_bwd_block_sparse, and FLOPs count only the kept
+(query, key) pairs.
+
 ``--impl reference`` times the fp64 CPU oracle instead (the only other place
 this script runs it), on a bounded sample of the same workload.
 Multi-GPU (torchrun): every rank runs an independent batch of the same shape
@@ -38,7 +44,7 @@ if ROOT not in sys.path:
 DEFAULT_WORKLOAD = "train_b8h16n2048d128_full"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = ["exact_io_aware_71_b200/csrc/sm100.cuh", "exact_io_aware_71_b200/csrc/fa_fwd.cuh",
-                  "exact_io_aware_71_b200/csrc/fa_bwd.cuh"]
+                  "exact_io_aware_71_b200/csrc/fa_bwd.cuh", "exact_io_aware_71_b200/csrc/fa_mask.cuh"]
 METRIC = "attention fwd / fwd+bwd TFLOP/s (bf16, 1×B200) and % of dense BF16 peak"
 
 
@@ -53,6 +59,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU work for the oracle baseline sample")
+    ap.add_argument("--block-density", type=float, default=None,
+                    help="block-sparse attention with this fraction of 128x128 blocks kept")
     return ap.parse_args(argv)
 
 
@@ -157,7 +165,52 @@ def parse_clock_samples(text: str):
 _INPUT_CACHE = {}
 
 
-def time_oracle(wl, seconds: float, max_groups=None):
+def launches_per_step(wl, sms: int) -> int:
+    """Kernels one step launches: the forward kernel, the backward's
+    preprocess, main and dQ-convert kernels, and the dK/dV convert kernel
+    when a GQA group's query heads are split over CTAs (the library splits
+    when one CTA per (batch, kv head, key block) would give fewer than two
+    CTAs per SM)."""
+    g = wl.Hq // wl.Hkv
+    if g == 1:
+        return 4
+    base = ((wl.Nk + 127) // 128) * wl.B * wl.Hkv * (2 if wl.d == 256 else 1)
+    gsplit = next((s_ for s_ in range(1, g + 1) if g % s_ == 0 and base * s_ >= 2 * sms), g)
+    return 4 + (1 if gsplit > 1 else 0)
+
+
+def block_mask_for(wl, density):
+    """Seeded block mask of the block-sparse measurement (None: dense)."""
+    if density is None:
+        return None
+    from exact_io_aware_71_b200.inputs import make_block_mask
+    return make_block_mask(wl.Nq, wl.Nk, density, seed=wl.seed)
+
+
+def kept_fraction(wl, mask) -> float:
+    """Visible (query, key) pairs under the block mask (and the causal mask)
+    over those of the dense problem: the FLOP scale of block-sparse steps."""
+    import numpy as np
+    if mask is None:
+        return 1.0
+    m = np.asarray(mask, dtype=bool)
+    rows = np.minimum(wl.Nq, (np.arange(m.shape[0]) + 1) * 128) - np.arange(m.shape[0]) * 128
+    cols = np.minimum(wl.Nk, (np.arange(m.shape[1]) + 1) * 128) - np.arange(m.shape[1]) * 128
+    if not wl.causal:
+        return float((m * np.outer(rows, cols)).sum() / (wl.Nq * wl.Nk))
+    # causal: pairs (i, j) with j <= i inside each block
+    kept = dense = 0.0
+    for bi in range(m.shape[0]):
+        i = np.arange(bi * 128, bi * 128 + rows[bi])
+        for bj in range(m.shape[1]):
+            j0, j1 = bj * 128, bj * 128 + cols[bj]
+            n = np.clip(np.minimum(i + 1, j1) - j0, 0, None).sum()
+            dense += n
+            kept += n if m[bi, bj] else 0
+    return float(kept / dense)
+
+
+def time_oracle(wl, seconds: float, max_groups=None, mask=None):
     """fp64 oracle forward + backward on whole (batch, kv-head) groups of the
     workload, as many as fit in about `seconds`; returns (TFLOP/s, cores,
     sample description).  Work is exact per group, so the rate scales."""
@@ -173,7 +226,7 @@ def time_oracle(wl, seconds: float, max_groups=None):
     q, k, v, do = _INPUT_CACHE[wl.name]
     g = wl.Hq // wl.Hkv
     groups = [(b, j) for b in range(wl.B) for j in range(wl.Hkv)]
-    per_group_flops = 3.5 * wl.fwd_flops() / len(groups)
+    per_group_flops = 3.5 * wl.fwd_flops() * kept_fraction(wl, mask) / len(groups)
     done, t_total = 0, 0.0
     with threadpool_limits(limits=cores):
         for (b, j) in groups:
@@ -184,15 +237,17 @@ def time_oracle(wl, seconds: float, max_groups=None):
             ks = k[b:b + 1, j:j + 1].double().numpy()
             vs = v[b:b + 1, j:j + 1].double().numpy()
             t0 = time.perf_counter()
-            oracle.attention_backward(qs, ks, vs, dos, wl.causal, wl.scale, return_aux=True)
+            oracle.attention_backward(qs, ks, vs, dos, wl.causal, wl.scale, return_aux=True,
+                                      block_mask=None if mask is None else mask.numpy())
             t_total += time.perf_counter() - t0
             done += 1
             if max_groups is None and t_total >= seconds and done >= 2:
                 break
     tflops = done * per_group_flops / t_total / 1e12
     sample = (f"fp64 NumPy oracle fwd+bwd on {done} of {len(groups)} (batch, kv-head) groups "
-              f"({g} query head(s) each) of {wl.name}; {t_total:.1f} s of CPU work; "
-              f"rate scaled exactly by FLOPs")
+              f"({g} query head(s) each) of {wl.name}"
+              f"{'' if mask is None else ' with the same block mask'}; {t_total:.1f} s of CPU "
+              f"work; rate scaled exactly by FLOPs")
     return tflops, cores, sample, t_total, done * per_group_flops
 
 
@@ -220,11 +275,34 @@ def run_ours(args, rank, world, local_rank):
     bwd_args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                 do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr()) + dims
 
-    names = ["fa_fwd_kernel", "fa_bwd_pre_kernel", "fa_bwd_main_kernel", "fa_bwd_dq_kernel"]
+    mask = block_mask_for(wl, args.block_density)
+    frac = kept_fraction(wl, mask)
+    sparse = mask is not None
+    if sparse:
+        mask_d = mask.to(dev)
+        # one event pair per call: the backward's three kernels are timed together
+        names = ["fa_fwd_kernel", "fa_bwd (pre, main, dq)"]
+    else:
+        names = ["fa_fwd_kernel", "fa_bwd_pre_kernel", "fa_bwd_main_kernel", "fa_bwd_dq_kernel"]
+    nk = len(names)
 
     def step(evs=None):
         if evs:
             evs[0].record(stream)
+        if sparse:
+            st = fa.fa_fwd_block_sparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                        lse.data_ptr(), None, mask_d.data_ptr(), *dims, sh)
+            if st:
+                raise fa.FaError(st, "fa_fwd_block_sparse")
+            if evs:
+                evs[1].record(stream)
+            st = fa.fa_bwd_block_sparse(*bwd_args[:9], None, mask_d.data_ptr(), *dims,
+                                        ws.data_ptr(), wsb, sh)
+            if st:
+                raise fa.FaError(st, "fa_bwd_block_sparse")
+            if evs:
+                evs[2].record(stream)
+            return
         st = fa.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                        *dims, sh)
         if st:
@@ -260,7 +338,8 @@ def run_ours(args, rank, world, local_rank):
     if st:
         raise RuntimeError(f"device status {st} at wait {where} during warm-up")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)]
+           for _ in range(args.steps)]
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local_rank)
     barrier()
@@ -275,19 +354,20 @@ def run_ours(args, rank, world, local_rank):
     clk = clocks.stop()
     local_ms = e0.elapsed_time(e1)
     per_kernel_ms = [sum(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(args.steps))
-                     / args.steps for i in range(4)]
+                     / args.steps for i in range(nk)]
     st, where = fa.fa_device_status(sh)
     if st:
         raise RuntimeError(f"device status {st} at wait {where} in the timed region")
 
-    flops_step = 3.5 * wl.fwd_flops()
+    fwd_flops, bwd_flops = wl.fwd_flops() * frac, wl.bwd_flops() * frac
+    flops_step = fwd_flops + bwd_flops
     t_ms, flops_per_s = aggregate(local_ms, args.steps * flops_step, world, reduce_max)
     value = flops_per_s / 1e12
 
     # ---- roofline of the dominant kernel (largest share of the step)
     peaks, peak_src = load_peaks()
-    dom = max(range(4), key=lambda i: per_kernel_ms[i])
-    algo_flops = [wl.fwd_flops(), None, wl.bwd_flops(), None]
+    dom = max(range(nk), key=lambda i: per_kernel_ms[i])
+    algo_flops = [fwd_flops, bwd_flops] if sparse else [fwd_flops, None, bwd_flops, None]
     if algo_flops[dom] is not None:
         achieved = algo_flops[dom] / (per_kernel_ms[dom] / 1e3) / 1e12
         roof = {"bound": "tensor", "kernel": names[dom], "achieved": round(achieved, 2),
@@ -299,33 +379,43 @@ def run_ours(args, rank, world, local_rank):
     else:
         roof = {"bound": "hbm", "kernel": names[dom], "achieved": None, "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": None, "traffic": None}
-    fwd_tflops = wl.fwd_flops() / (per_kernel_ms[0] / 1e3) / 1e12
+    fwd_tflops = fwd_flops / (per_kernel_ms[0] / 1e3) / 1e12
     bwd_ms = sum(per_kernel_ms[1:])
-    bwd_tflops = wl.bwd_flops() / (bwd_ms / 1e3) / 1e12
+    bwd_tflops = bwd_flops / (bwd_ms / 1e3) / 1e12
 
     # ---- end to end through the public API with host buffers
-    e2e = run_e2e(args, wl, dev, stream, fa, q, k, v, do, reduce_max, world)
+    e2e = run_e2e(args, wl, dev, stream, fa, q, k, v, do, reduce_max, world,
+                  mask_d if sparse else None, frac)
 
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": round(t_ms / args.steps, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded iid N(0,1), bf16)",
-        "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "Nq": wl.Nq,
+        "config": {"workload": wl.name + (f"_blocksparse{args.block_density:g}" if sparse else ""),
+                   "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "Nq": wl.Nq,
                    "Nk": wl.Nk, "d": wl.d, "causal": wl.causal,
-                   "step": "fa_fwd + fa_bwd (pre, main, dq)",
+                   "step": ("fa_fwd_block_sparse + fa_bwd_block_sparse" if sparse
+                            else "fa_fwd + fa_bwd (pre, main, dq)"),
                    "parallelism": f"{world} independent replica(s), no collective",
                    "l2": "inputs larger than L2 (448 MiB read per step), no flush"},
         "fwd_tflops": round(fwd_tflops, 2), "bwd_tflops": round(bwd_tflops, 2),
         "fwd_frac_of_peak": round(fwd_tflops / peaks["bf16_tflops"], 4),
         "bwd_frac_of_peak": round(bwd_tflops / peaks["bf16_tflops"], 4),
         "per_kernel_ms": {n: round(t, 4) for n, t in zip(names, per_kernel_ms)},
-        "roofline": roof, "e2e": e2e, "clocks": clk, "gpu_launches": 4 * args.steps,
+        "roofline": roof, "e2e": e2e, "clocks": clk,
+        "gpu_launches": launches_per_step(wl, torch.cuda.get_device_properties(dev)
+                                          .multi_processor_count) * args.steps,
     }
+    if sparse:
+        out["config"]["block_mask"] = {
+            "block": 128, "density": args.block_density, "seed": wl.seed,
+            "kept_pair_fraction": round(frac, 4),
+            "flops": "nominal dense FLOPs x kept (query, key) pair fraction"}
     return out
 
 
-def run_e2e(args, wl, dev, stream, fa, q, k, v, do, reduce_max, world):
+def run_e2e(args, wl, dev, stream, fa, q, k, v, do, reduce_max, world, mask=None, frac=1.0):
     """Same metric through the public torch-level binding with host buffers:
     each step copies q, k, v, dO from pinned host memory, runs fa_fwd and
     fa_bwd, and reads o, lse, dq, dk, dv back to pinned host memory."""
@@ -343,9 +433,10 @@ def run_e2e(args, wl, dev, stream, fa, q, k, v, do, reduce_max, world):
     def step():
         for dst, src in zip(dev_in, (hq, hk, hv, hdo)):
             dst.copy_(src, non_blocking=True)
-        fa.forward(dev_in[0], dev_in[1], dev_in[2], wl.causal, wl.scale, out=o_, lse=lse_)
+        fa.forward(dev_in[0], dev_in[1], dev_in[2], wl.causal, wl.scale, out=o_, lse=lse_,
+                   block_mask=mask)
         g = fa.backward(dev_in[0], dev_in[1], dev_in[2], o_, lse_, dev_in[3], wl.causal,
-                        wl.scale, workspace=ws)
+                        wl.scale, workspace=ws, block_mask=mask)
         for dst, src in zip(outs_h, (o_, lse_) + g):
             dst.copy_(src, non_blocking=True)
 
@@ -359,8 +450,8 @@ def run_e2e(args, wl, dev, stream, fa, q, k, v, do, reduce_max, world):
         step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    t_ms, fps = aggregate(e0.elapsed_time(e1), args.e2e_steps * 3.5 * wl.fwd_flops(), world,
-                          reduce_max)
+    t_ms, fps = aggregate(e0.elapsed_time(e1), args.e2e_steps * 3.5 * wl.fwd_flops() * frac,
+                          world, reduce_max)
     bi = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
     bo = sum(t.numel() * t.element_size() for t in outs_h)
     return {"value": round(fps / 1e12, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": bi,
@@ -372,12 +463,13 @@ def run_e2e(args, wl, dev, stream, fa, q, k, v, do, reduce_max, world):
 def run_reference(args):
     from exact_io_aware_71_b200.inputs import workloads
     wl = workloads()[args.workload]
+    mask = block_mask_for(wl, args.block_density)
     for _ in range(args.warmup):
-        time_oracle(wl, 0.0, max_groups=1)
+        time_oracle(wl, 0.0, max_groups=1, mask=mask)
     t_all, f_all = 0.0, 0.0
     cores = len(os.sched_getaffinity(0))
     for _ in range(args.steps):
-        _, cores, sample, t, f = time_oracle(wl, 0.0, max_groups=1)
+        _, cores, sample, t, f = time_oracle(wl, 0.0, max_groups=1, mask=mask)
         t_all += t
         f_all += f
     value = f_all / t_all / 1e12
@@ -387,7 +479,9 @@ def run_reference(args):
         "ms_per_step": round(1e3 * t_all / args.steps, 2), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded iid N(0,1), bf16 inputs upcast to fp64)",
-        "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "Nq": wl.Nq,
+        "config": {"workload": wl.name + ("" if mask is None
+                                          else f"_blocksparse{args.block_density:g}"),
+                   "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "Nq": wl.Nq,
                    "Nk": wl.Nk, "d": wl.d, "causal": wl.causal,
                    "step": "oracle fwd+bwd on one (batch, kv-head) group of the workload"},
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores,
@@ -420,7 +514,9 @@ def main(argv=None):
         out = run_ours(args, rank, world, local_rank)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             from exact_io_aware_71_b200.inputs import workloads
-            tf, cores, sample, _, _ = time_oracle(workloads()[args.workload], args.cpu_seconds)
+            wl = workloads()[args.workload]
+            tf, cores, sample, _, _ = time_oracle(wl, args.cpu_seconds,
+                                                  mask=block_mask_for(wl, args.block_density))
             out["cpu_baseline"] = {"value": round(tf, 6), "unit": "TFLOP/s", "cores": cores,
                                    "kind": "oracle", "sample": sample}
         if rank == 0:

@@ -12,6 +12,9 @@ from .binding import (  # noqa: F401
     fa_bwd_stage,
     fa_bwd_strided,
     fa_fwd_strided,
+    fa_fwd_block_sparse,
+    fa_bwd_block_sparse,
+    MASK_BLOCK,
     FaStrides,
     strides_of,
     fa_bwd_workspace_size,

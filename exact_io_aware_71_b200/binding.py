@@ -24,7 +24,10 @@ STATUS_NAMES = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED",
 # Exported symbols declared in include/fa.h.
 SYMBOLS = ("fa_fwd", "fa_bwd", "fa_bwd_stage", "fa_bwd_workspace_size", "fa_status_string",
            "fa_device_status", "fa_bwd_noalloc", "fa_debug_inject", "fa_fwd_strided",
-           "fa_bwd_strided")
+           "fa_bwd_strided", "fa_fwd_block_sparse", "fa_bwd_block_sparse")
+
+# Rows / keys per block-mask entry (FA_MASK_BLOCK).
+MASK_BLOCK = 128
 
 # Bytes of the built-in scratch behind fa_bwd_noalloc (FA_NOALLOC_SCRATCH_BYTES).
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -75,6 +78,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fa_bwd_strided.argtypes = [vp] * 9 + [sp] + [i] * 7 + [f, vp, sz, vp]
     lib.fa_bwd_strided.restype = i
     lib.fa_bwd_stage.restype = i
+    lib.fa_fwd_block_sparse.argtypes = [vp] * 5 + [sp, vp] + [i] * 7 + [f, vp]
+    lib.fa_fwd_block_sparse.restype = i
+    lib.fa_bwd_block_sparse.argtypes = [vp] * 9 + [sp, vp] + [i] * 7 + [f, vp, sz, vp]
+    lib.fa_bwd_block_sparse.restype = i
     lib.fa_bwd_noalloc.argtypes = lib.fa_bwd.argtypes[:17] + [vp]
     lib.fa_bwd_noalloc.restype = i
     lib.fa_bwd_workspace_size.argtypes = [i, i, i, i, i, i, i]
@@ -106,6 +113,21 @@ def fa_bwd_strided(q, k, v, o, lse, dO, dq, dk, dv, strides, B, Hq, Hkv, Nq, Nk,
     arr = (FaStrides * 8)(*strides) if strides is not None else None
     return load().fa_bwd_strided(q, k, v, o, lse, dO, dq, dk, dv, arr, B, Hq, Hkv, Nq, Nk, d,
                                  int(causal), float(scale), workspace, workspace_bytes, stream)
+
+
+def fa_fwd_block_sparse(q, k, v, o, lse, strides, block_mask, B, Hq, Hkv, Nq, Nk, d, causal,
+                        scale, stream) -> int:
+    arr = (FaStrides * 4)(*strides) if strides is not None else None
+    return load().fa_fwd_block_sparse(q, k, v, o, lse, arr, block_mask, B, Hq, Hkv, Nq, Nk, d,
+                                      int(causal), float(scale), stream)
+
+
+def fa_bwd_block_sparse(q, k, v, o, lse, dO, dq, dk, dv, strides, block_mask, B, Hq, Hkv, Nq, Nk,
+                        d, causal, scale, workspace, workspace_bytes, stream) -> int:
+    arr = (FaStrides * 8)(*strides) if strides is not None else None
+    return load().fa_bwd_block_sparse(q, k, v, o, lse, dO, dq, dk, dv, arr, block_mask, B, Hq,
+                                      Hkv, Nq, Nk, d, int(causal), float(scale), workspace,
+                                      workspace_bytes, stream)
 
 
 def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, causal, scale,
@@ -159,26 +181,48 @@ def _dims(q, k):
     return B, Hq, Hkv, Nq, Nk, d
 
 
-def forward(q, k, v, causal: bool, scale: float, out=None, lse=None):
+def _mask_ptr(block_mask, Nq, Nk):
+    """Device address of a [ceil(Nq/128), ceil(Nk/128)] uint8 / bool CUDA mask."""
+    import torch
+    shape = ((Nq + MASK_BLOCK - 1) // MASK_BLOCK, (Nk + MASK_BLOCK - 1) // MASK_BLOCK)
+    if tuple(block_mask.shape) != shape:
+        raise ValueError(f"block mask must have shape {shape}, got {tuple(block_mask.shape)}")
+    if block_mask.dtype not in (torch.uint8, torch.bool) or not block_mask.is_cuda \
+            or not block_mask.is_contiguous():
+        raise ValueError("block mask must be a contiguous uint8 or bool CUDA tensor")
+    return block_mask.data_ptr()
+
+
+def forward(q, k, v, causal: bool, scale: float, out=None, lse=None, block_mask=None):
     """O, LSE for bf16 CUDA tensors q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d] (any
-    strides with a contiguous last axis, e.g. permuted [B,N,H,d] storage)."""
+    strides with a contiguous last axis, e.g. permuted [B,N,H,d] storage).
+    block_mask: optional block-sparse mask, [ceil(Nq/128), ceil(Nk/128)]."""
     import torch
     B, Hq, Hkv, Nq, Nk, d = _dims(q, k)
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty(B, Hq, Nq, dtype=torch.float32, device=q.device)
-    st = fa_fwd_strided(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                        [strides_of(t) for t in (q, k, v, out)], B, Hq, Hkv, Nq, Nk, d, causal,
-                        scale, _stream_handle())
+    ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr())
+    strides = [strides_of(t) for t in (q, k, v, out)]
+    if block_mask is None:
+        st = fa_fwd_strided(*ptrs, strides, B, Hq, Hkv, Nq, Nk, d, causal, scale,
+                            _stream_handle())
+        what = "fa_fwd_strided"
+    else:
+        st = fa_fwd_block_sparse(*ptrs, strides, _mask_ptr(block_mask, Nq, Nk), B, Hq, Hkv, Nq,
+                                 Nk, d, causal, scale, _stream_handle())
+        what = "fa_fwd_block_sparse"
     if st != FA_OK:
-        raise FaError(st, "fa_fwd_strided")
+        raise FaError(st, what)
     return out, lse
 
 
-def backward(q, k, v, o, lse, do, causal: bool, scale: float, workspace=None, grads=None):
+def backward(q, k, v, o, lse, do, causal: bool, scale: float, workspace=None, grads=None,
+             block_mask=None):
     """dQ, dK, dV (bf16) for the forward inputs/outputs and dO; gradients
-    take the strides of q, k, v unless `grads` gives the output tensors."""
+    take the strides of q, k, v unless `grads` gives the output tensors.
+    block_mask: the forward pass's block-sparse mask, if it had one."""
     import torch
     B, Hq, Hkv, Nq, Nk, d = _dims(q, k)
     need = fa_bwd_workspace_size(B, Hq, Hkv, Nq, Nk, d, causal)
@@ -187,10 +231,17 @@ def backward(q, k, v, o, lse, do, causal: bool, scale: float, workspace=None, gr
     dq, dk, dv = grads if grads is not None else (torch.empty_like(q), torch.empty_like(k),
                                                   torch.empty_like(v))
     ts = (q, k, v, o, do, dq, dk, dv)
-    st = fa_bwd_strided(*(t.data_ptr() for t in ts[:4]), lse.data_ptr(),
-                        *(t.data_ptr() for t in ts[4:]), [strides_of(t) for t in ts],
-                        B, Hq, Hkv, Nq, Nk, d, causal, scale, workspace.data_ptr(),
-                        workspace.numel(), _stream_handle())
+    ptrs = (*(t.data_ptr() for t in ts[:4]), lse.data_ptr(), *(t.data_ptr() for t in ts[4:]))
+    strides = [strides_of(t) for t in ts]
+    if block_mask is None:
+        st = fa_bwd_strided(*ptrs, strides, B, Hq, Hkv, Nq, Nk, d, causal, scale,
+                            workspace.data_ptr(), workspace.numel(), _stream_handle())
+        what = "fa_bwd_strided"
+    else:
+        st = fa_bwd_block_sparse(*ptrs, strides, _mask_ptr(block_mask, Nq, Nk), B, Hq, Hkv, Nq,
+                                 Nk, d, causal, scale, workspace.data_ptr(), workspace.numel(),
+                                 _stream_handle())
+        what = "fa_bwd_block_sparse"
     if st != FA_OK:
-        raise FaError(st, "fa_bwd_strided")
+        raise FaError(st, what)
     return dq, dk, dv

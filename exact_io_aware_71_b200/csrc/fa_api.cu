@@ -20,6 +20,7 @@
 namespace fa {
 __device__ DevStatus g_status;   // one status word per device (module global)
 }
+static_assert(FA_MASK_BLOCK == fa::MASK_BLOCK, "block-mask granularity of the C ABI");
 
 namespace {
 
@@ -134,14 +135,15 @@ int launch_kernel(KernelT kern, int smem, int threads, unsigned grid, const CUte
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-// d = 64 / 128: two query tiles per CTA; d = 256: one.
-template <int D, bool CAUSAL>
+// d = 64 / 128: two query tiles per CTA; d = 256: one.  SPARSE: p.mask is a
+// block mask.
+template <int D, bool CAUSAL, bool SPARSE>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                const CUtensorMap& mo, FwdParams p, cudaStream_t stream) {
   if constexpr (D == 256) {
     using C = FwdCfg<D>;
     p.n_units = p.n_qblocks;
-    return launch_kernel(fa_fwd_kernel<D, CAUSAL>, C::SMEM_BYTES, C::NTHREADS,
+    return launch_kernel(fa_fwd_kernel<D, CAUSAL, SPARSE>, C::SMEM_BYTES, C::NTHREADS,
                          unsigned(p.n_units) * unsigned(p.B * p.Hq), mq, mk, mv, mo, p, stream);
   } else {
     using C = FwdPairCfg<D>;
@@ -150,7 +152,7 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
     static int regs = -1;
     if (regs < 0) {
       cudaFuncAttributes fattr;
-      if (cudaFuncGetAttributes(&fattr, fa_fwd_pair_kernel<D, CAUSAL>) != cudaSuccess)
+      if (cudaFuncGetAttributes(&fattr, fa_fwd_pair_kernel<D, CAUSAL, SPARSE>) != cudaSuccess)
         return FA_ERR_CUDA;
       regs = fattr.numRegs;
     }
@@ -168,32 +170,22 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
     const long long units = (long long)p.n_units * p.B * p.Hq;
     const bool persistent = p.Nk <= 4096 || (CAUSAL && p.Nk <= 16384);
     const unsigned grid = unsigned(persistent ? std::min<long long>(units, sms) : units);
-    return launch_kernel(fa_fwd_pair_kernel<D, CAUSAL>, C::SMEM_BYTES, C::NTHREADS, grid, mq, mk,
-                         mv, mo, p, stream);
+    return launch_kernel(fa_fwd_pair_kernel<D, CAUSAL, SPARSE>, C::SMEM_BYTES, C::NTHREADS, grid,
+                         mq, mk, mv, mo, p, stream);
   }
 }
 
-}  // namespace
-
-extern "C" {
-
-const char* fa_status_string(int s) {
-  switch (s) {
-    case FA_OK: return "FA_OK";
-    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
-    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
-    case FA_ERR_MISALIGNED: return "FA_ERR_MISALIGNED";
-    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE";
-    case FA_ERR_CUDA: return "FA_ERR_CUDA";
-    case FA_ERR_DEVICE_TIMEOUT: return "FA_ERR_DEVICE_TIMEOUT";
-    case FA_ERR_TOO_LARGE: return "FA_ERR_TOO_LARGE";
-    default: return "FA_ERR_UNKNOWN";
-  }
+template <int D, bool CAUSAL>
+int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+               const CUtensorMap& mo, const FwdParams& p, cudaStream_t stream) {
+  return p.mask ? launch_fwd<D, CAUSAL, true>(mq, mk, mv, mo, p, stream)
+                : launch_fwd<D, CAUSAL, false>(mq, mk, mv, mo, p, stream);
 }
 
-int fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse,
-                   const fa_strides* strides, int B, int Hq, int Hkv, int Nq, int Nk, int d,
-                   int causal, float scale, cudaStream_t stream) {
+// The forward pass on strided tensors, with an optional block mask.
+int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse,
+             const fa_strides* strides, const unsigned char* mask, int B, int Hq, int Hkv,
+             int Nq, int Nk, int d, int causal, float scale, cudaStream_t stream) {
   if (!q || !k || !v || !o || !lse || !strides) return FA_ERR_INVALID_ARG;
   int st = check_sizes(B, Hq, Hkv, Nq, Nk, d, causal, scale);
   if (st != FA_OK) return st;
@@ -222,6 +214,10 @@ int fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* 
   p.lse = lse;
   p.status = status_ptr();
   if (!p.status) return FA_ERR_CUDA;
+  p.mask = mask;
+  p.mask_ld = (Nk + MASK_BLOCK - 1) / MASK_BLOCK;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.o_sb = so.b; p.o_sh = so.h; p.o_sn = so.n;
 
   if (d == 64) return causal ? launch_fwd<64, true>(mq, mk, mv, mo, p, stream)
                              : launch_fwd<64, false>(mq, mk, mv, mo, p, stream);
@@ -231,12 +227,61 @@ int fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* 
                 : launch_fwd<256, false>(mq, mk, mv, mo, p, stream);
 }
 
+// Element strides of the contiguous layouts of q, k, v, o.
+void contiguous4(fa_strides* s, int Hq, int Hkv, int Nq, int Nk, int d) {
+  const Strides a = contiguous(Hq, Nq, d), b = contiguous(Hkv, Nk, d);
+  s[0] = {a.b, a.h, a.n};
+  s[1] = {b.b, b.h, b.n};
+  s[2] = {b.b, b.h, b.n};
+  s[3] = {a.b, a.h, a.n};
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fa_status_string(int s) {
+  switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_MISALIGNED: return "FA_ERR_MISALIGNED";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_DEVICE_TIMEOUT: return "FA_ERR_DEVICE_TIMEOUT";
+    case FA_ERR_TOO_LARGE: return "FA_ERR_TOO_LARGE";
+    default: return "FA_ERR_UNKNOWN";
+  }
+}
+
+int fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse,
+                   const fa_strides* strides, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                   int causal, float scale, cudaStream_t stream) {
+  return fwd_impl(q, k, v, o, lse, strides, nullptr, B, Hq, Hkv, Nq, Nk, d, causal, scale,
+                  stream);
+}
+
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
            int Hkv, int Nq, int Nk, int d, int causal, float scale, cudaStream_t stream) {
   if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1) return FA_ERR_INVALID_ARG;
-  const Strides a = contiguous(Hq, Nq, d), b = contiguous(Hkv, Nk, d);
-  const fa_strides s[4] = {{a.b, a.h, a.n}, {b.b, b.h, b.n}, {b.b, b.h, b.n}, {a.b, a.h, a.n}};
-  return fa_fwd_strided(q, k, v, o, lse, s, B, Hq, Hkv, Nq, Nk, d, causal, scale, stream);
+  fa_strides s[4];
+  contiguous4(s, Hq, Hkv, Nq, Nk, d);
+  return fwd_impl(q, k, v, o, lse, s, nullptr, B, Hq, Hkv, Nq, Nk, d, causal, scale, stream);
+}
+
+int fa_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                        const fa_strides* strides, const unsigned char* block_mask, int B, int Hq,
+                        int Hkv, int Nq, int Nk, int d, int causal, float scale,
+                        cudaStream_t stream) {
+  if (!block_mask) return FA_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1) return FA_ERR_INVALID_ARG;
+  fa_strides s[4];
+  if (!strides) {
+    contiguous4(s, Hq, Hkv, Nq, Nk, d);
+    strides = s;
+  }
+  return fwd_impl(q, k, v, o, lse, strides, block_mask, B, Hq, Hkv, Nq, Nk, d, causal, scale,
+                  stream);
 }
 
 size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal) {
@@ -253,7 +298,7 @@ int bwd_impl(int stage, const void* q, const void* k, const void* v, const void*
              const float* lse, const void* dO, void* dq, void* dk, void* dv,
              const fa_strides* strides, int B, int Hq, int Hkv, int Nq, int Nk, int d,
              int causal, float scale, void* workspace, size_t workspace_bytes,
-             cudaStream_t stream) {
+             cudaStream_t stream, const unsigned char* mask = nullptr) {
   int stages;
   switch (stage) {
     case FA_BWD_ALL: stages = 7; break;
@@ -278,7 +323,7 @@ int bwd_impl(int stage, const void* q, const void* k, const void* v, const void*
   Strides s8[8];
   for (int i = 0; i < 8; ++i) s8[i] = Strides{strides[i].batch, strides[i].head, strides[i].row};
   return launch_bwd(stages, q, k, v, o, lse, dO, dq, dk, dv, s8, B, Hq, Hkv, Nq, Nk, d, causal,
-                    scale, workspace, sp, stream);
+                    scale, mask, workspace, sp, stream);
 }
 
 void contiguous8(fa_strides* s, int Hq, int Hkv, int Nq, int Nk, int d) {
@@ -298,6 +343,22 @@ int fa_bwd_strided(const void* q, const void* k, const void* v, const void* o, c
                    void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   return bwd_impl(FA_BWD_ALL, q, k, v, o, lse, dO, dq, dk, dv, strides, B, Hq, Hkv, Nq, Nk, d,
                   causal, scale, workspace, workspace_bytes, stream);
+}
+
+int fa_bwd_block_sparse(const void* q, const void* k, const void* v, const void* o,
+                        const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                        const fa_strides* strides, const unsigned char* block_mask, int B, int Hq,
+                        int Hkv, int Nq, int Nk, int d, int causal, float scale, void* workspace,
+                        size_t workspace_bytes, cudaStream_t stream) {
+  if (!block_mask) return FA_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1) return FA_ERR_INVALID_ARG;
+  fa_strides s[8];
+  if (!strides) {
+    contiguous8(s, Hq, Hkv, Nq, Nk, d);
+    strides = s;
+  }
+  return bwd_impl(FA_BWD_ALL, q, k, v, o, lse, dO, dq, dk, dv, strides, B, Hq, Hkv, Nq, Nk, d,
+                  causal, scale, workspace, workspace_bytes, stream, block_mask);
 }
 
 int fa_bwd_stage(int stage, const void* q, const void* k, const void* v, const void* o,

@@ -36,6 +36,7 @@
 // owning one 128-wide half of d for dK, dV and dQ (both recompute S and dP).
 #pragma once
 #include "sm100.cuh"
+#include "fa_mask.cuh"
 
 namespace fa {
 
@@ -215,6 +216,8 @@ struct BwdParams {
   float* dkacc;       // fp32 dK / dV partial sums when gsplit > 1
   float* dvacc;
   DevStatus* status;
+  const uint8_t* mask;  // block-sparse only: [ceil(Nq/128)][mask_ld] block mask
+  int mask_ld;          // ceil(Nk / 128)
 };
 
 enum : unsigned { WB_KV = 16, WB_QEMPTY, WB_QFULL, WB_S, WB_DP, WB_P, WB_DS, WB_DQFULL,
@@ -229,7 +232,9 @@ __device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_
       : "memory");
 }
 
-template <int D, bool CAUSAL>
+// Block-sparse (SPARSE): a key block visits only the query blocks whose mask
+// entry for it is set, in the same cyclic order for every role.
+template <int D, bool CAUSAL, bool SPARSE>
 __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
@@ -239,6 +244,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
                        const __grid_constant__ CUtensorMap tmdV, const BwdParams p) {
   using C = BwdCfg<D>;
   constexpr int BR = C::BR, BC = C::BC, DH = C::DH, QS = C::QS;
+  static_assert(BC == MASK_BLOCK, "a CTA's key block is one block-mask column");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -260,6 +266,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
   uint64_t* bar_final = bars + 8 + 2 * QS;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 9 + 2 * QS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  int* sparse_ni = reinterpret_cast<int*>(tmem_holder + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -278,19 +285,38 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
   const int hkv = bkv - b * p.Hkv;
   const int key0 = kb * BC;
   const int i0 = CAUSAL ? (key0 / BR) : 0;              // first query block that sees key0
-  const int n_i = max(0, p.n_qblocks - i0);
-  const int n_steps = p.hps * n_i;
+  const int span = max(0, p.n_qblocks - i0);
+  int n_i = span;                                       // query blocks visited per head
   const int dcol0 = split * DH;                         // first d column owned here
   const int head0 = hkv * p.group + gs * p.hps;         // first query head (within batch b)
   // Without the causal mask every key block visits every query block; key
   // blocks start at different query blocks so that their fp32 dQ reduce-adds
   // do not all land on the same rows at once.
-  const int rot = CAUSAL ? 0 : int((long long)kb * n_i / p.n_kblocks);
+  const int rot = CAUSAL ? 0 : int((long long)kb * span / p.n_kblocks);
   auto step_q = [&](int t, int& hh, int& qi) {
     hh = t / n_i;
     int li = t - hh * n_i + rot;
     if (li >= n_i) li -= n_i;
     qi = i0 + li;
+  };
+  // Block-sparse: query block i (BR rows) is visited iff its mask entry for
+  // this key block is set; the visited blocks are taken cyclically from
+  // i0 + rot, head after head.
+  auto qvis = [&](int i) -> bool {
+    return __ldg(p.mask + size_t(i * BR / MASK_BLOCK) * p.mask_ld + kb) != 0;
+  };
+  auto qnext = [&](int i) -> int {        // next visited block at or after i, cyclically
+    for (int k = 0; k < span; ++k, ++i) {
+      if (i >= p.n_qblocks) i = i0;
+      if (qvis(i)) return i;
+    }
+    return i0;                            // not reached while n_i > 0
+  };
+  struct Seq { int hh, qi, c; };
+  auto seq_begin = [&](Seq& q) { q.hh = 0; q.c = 0; q.qi = qnext(i0 + rot); };
+  auto seq_next = [&](Seq& q) {
+    if (++q.c == n_i) { q.c = 0; ++q.hh; q.qi = qnext(i0 + rot); }
+    else q.qi = qnext(q.qi + 1);
   };
 
   if (threadIdx.x == 0) {
@@ -314,10 +340,20 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
     tmem_alloc(tmem_holder, C::TMEM_COLS);
     tmem_relinquish();
   }
+  if constexpr (SPARSE) {
+    if (warp == 10) {                     // count the visited query blocks once
+      int c = 0;
+      for (int i = i0 + lane; i < p.n_qblocks; i += 32) c += qvis(i) ? 1 : 0;
+      c = __reduce_add_sync(0xffffffffu, c);
+      if (lane == 0) *sparse_ni = c;
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  if constexpr (SPARSE) n_i = *sparse_ni;
+  const int n_steps = p.hps * n_i;
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer
@@ -330,9 +366,17 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
         tma_load_bh(sV + c * BC * 128, &tmV, bar_kv, c * 64, key0, bkv, p.Hkv);
       }
       int issued = 0;
+      Seq sq;
+      if constexpr (SPARSE) seq_begin(sq);
       for (int t = 0; t < n_steps; ++t) {
         int hh, qi;
-        step_q(t, hh, qi);
+        if constexpr (SPARSE) {
+          hh = sq.hh;
+          qi = sq.qi;
+          seq_next(sq);
+        } else {
+          step_q(t, hh, qi);
+        }
         const int bh = b * p.Hq + head0 + hh;
         const int st = t % QS;
         if (!mbar_wait(bar_qempty + st, ((t / QS) & 1) ^ 1, abort_flag, p.status, WB_QEMPTY))
@@ -463,7 +507,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
 
     // Read out dQ^T of step u (lanes = d, columns = this group's 32 queries)
     // and reduce-add it into the fp32 accumulator (coalesced over d).
-    auto dq_readout = [&](int u) -> bool {
+    auto dq_readout = [&](int u, int hh, int qi) -> bool {
       bool okk = mbar_wait(bar_dqfull, u & 1, abort_flag, p.status, WB_DQFULL);
       if (!__all_sync(0xffffffffu, okk)) return false;
       tc_fence_after();
@@ -473,8 +517,6 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(bar_dqempty);
-        int hh, qi;
-        step_q(u, hh, qi);
         const int q0 = qi * BR + g * 32;
         const int bh = b * p.Hq + head0 + hh;
         float* dst = p.dqacc + (size_t(bh) * p.Nq + q0) * D + dcol0 + r;
@@ -494,9 +536,18 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
       return true;
     };
 
+    int prev_hh = 0, prev_qi = 0;                   // query block of step t - 1
+    Seq sq;
+    if constexpr (SPARSE) seq_begin(sq);
     for (int t = 0; t < n_steps; ++t) {
       int hh, qi;
-      step_q(t, hh, qi);
+      if constexpr (SPARSE) {
+        hh = sq.hh;
+        qi = sq.qi;
+        seq_next(sq);
+      } else {
+        step_q(t, hh, qi);
+      }
       const int st = t % QS;
       const float* sl = reinterpret_cast<const float*>(sStage + st * C::STAGE_STRIDE +
                                                        2 * C::QT_BYTES) + g * 32;
@@ -558,7 +609,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
       mbar_arrive(bar_p);
 
       // ---- dQ of the previous step (its MMA ran while P was formed)
-      if (t > 0 && !(ok = dq_readout(t - 1))) break;
+      if (t > 0 && !(ok = dq_readout(t - 1, prev_hh, prev_qi))) break;
 
       // ---- dS^T = P^T o (dP^T - D)
       ok = mbar_wait(bar_dp, t & 1, abort_flag, p.status, WB_DP);
@@ -595,8 +646,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar_ds);
+      prev_hh = hh;
+      prev_qi = qi;
     }
-    if (ok && n_steps > 0) ok = dq_readout(n_steps - 1);
+    if (ok && n_steps > 0) ok = dq_readout(n_steps - 1, prev_hh, prev_qi);
 
     // ---- epilogue: group 0 writes dK = scale * dK_acc, group 1 writes dV,
     // bf16 through the (now free) Q/dO stages, one 4 KiB box per warp and
@@ -684,7 +737,7 @@ template <int D, bool CAUSAL>
 int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const void* o,
                  const float* lse, const void* dO, void* dq, void* dk, void* dv,
                  const Strides* st, int B, int Hq, int Hkv, int Nq, int Nk, float scale,
-                 void* workspace, DevStatus* status, cudaStream_t stream) {
+                 const uint8_t* mask, void* workspace, DevStatus* status, cudaStream_t stream) {
   using C = BwdCfg<D>;
   const BwdWorkspace w = bwd_workspace_layout(B, Hq, Hkv, Nq, Nk, D);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -731,7 +784,7 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
     if (cudaGetLastError() != cudaSuccess) return 5;
   }
   if (stages & 2) {
-    auto kern = fa_bwd_main_kernel<D, CAUSAL>;
+    auto kern = mask ? fa_bwd_main_kernel<D, CAUSAL, true> : fa_bwd_main_kernel<D, CAUSAL, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
         cudaSuccess)
       return 5;
@@ -755,6 +808,8 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
     p.Lpad = Lpad;
     p.dqacc = dqacc;
     p.status = status;
+    p.mask = mask;
+    p.mask_ld = (Nk + MASK_BLOCK - 1) / MASK_BLOCK;
     const unsigned grid = unsigned(p.n_kblocks) * unsigned(B * Hkv) * C::NSPLIT * gsplit;
     kern<<<grid, C::NTHREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdk, mdv, p);
     if (cudaGetLastError() != cudaSuccess) return 5;
@@ -777,18 +832,19 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
   return 0;
 }
 
-// stages: bit 0 = preprocess, bit 1 = main, bit 2 = dq convert.
+// stages: bit 0 = preprocess, bit 1 = main, bit 2 = dq convert.  mask: the
+// block mask of block-sparse attention, or null.
 inline int launch_bwd(int stages, const void* q, const void* k, const void* v, const void* o,
                       const float* lse, const void* dO, void* dq, void* dk, void* dv,
                       const Strides* st, int B, int Hq, int Hkv, int Nq, int Nk, int d,
-                      int causal, float scale, void* workspace, DevStatus* status,
-                      cudaStream_t stream) {
+                      int causal, float scale, const uint8_t* mask, void* workspace,
+                      DevStatus* status, cudaStream_t stream) {
 #define FA_BWD_CASE(DD)                                                                          \
   if (d == DD)                                                                                   \
     return causal ? launch_bwd_t<DD, true>(stages, q, k, v, o, lse, dO, dq, dk, dv, st, B, Hq,  \
-                                           Hkv, Nq, Nk, scale, workspace, status, stream)       \
+                                           Hkv, Nq, Nk, scale, mask, workspace, status, stream) \
                   : launch_bwd_t<DD, false>(stages, q, k, v, o, lse, dO, dq, dk, dv, st, B, Hq, \
-                                            Hkv, Nq, Nk, scale, workspace, status, stream);
+                                            Hkv, Nq, Nk, scale, mask, workspace, status, stream);
   FA_BWD_CASE(64)
   FA_BWD_CASE(128)
   FA_BWD_CASE(256)

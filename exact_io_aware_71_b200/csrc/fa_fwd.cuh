@@ -29,6 +29,7 @@
 //    (O alone takes 256 TMEM columns), warps 0-3 softmax, 4 producer, 5 MMA.
 #pragma once
 #include "sm100.cuh"
+#include "fa_mask.cuh"
 
 // A row's O and sums are rescaled only when its running max (log2 units)
 // grows by more than this; in between, probabilities reach at most 2^threshold.
@@ -47,7 +48,27 @@ struct FwdParams {
   float scale_log2;   // scale * log2(e)
   float* lse;         // [B, Hq, Nq]
   DevStatus* status;
+  // Block-sparse attention only (null / unused otherwise): the block mask
+  // [ceil(Nq/128)][mask_ld] of 128 x 128 (query, key) blocks, shared by all
+  // batches and heads, and the output tensor itself, for the rows of query
+  // tiles that see no key (O = 0 there, written without the TMA epilogue).
+  const uint8_t* mask;
+  int mask_ld;        // ceil(Nk / 128)
+  __nv_bfloat16* o;
+  long long o_sb, o_sh, o_sn;
 };
+
+// A query row that sees no key at all (every block of its mask row is
+// zero): O = 0 and LSE = -inf, the limits of an empty softmax.
+template <int D>
+__device__ __forceinline__ void write_empty_row(const FwdParams& p, int bh, int grow) {
+  if (grow >= p.Nq) return;
+  const int b = bh / p.Hq, h = bh - b * p.Hq;
+  uint4* dst = reinterpret_cast<uint4*>(p.o + b * p.o_sb + h * p.o_sh + (long long)grow * p.o_sn);
+#pragma unroll
+  for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+  p.lse[size_t(bh) * p.Nq + grow] = -INFINITY;
+}
 
 // Wait codes recorded on a timeout.
 enum : unsigned { W_Q = 1, W_KV_EMPTY, W_KV_FULL, W_S_FULL, W_P_FULL, W_O_DONE, W_DRAIN };
@@ -66,16 +87,19 @@ struct RowState {
 //   tS     TMEM address (this warp's lanes) of the block's BC fp32 scores;
 //          P is written back over them as packed bf16 (BC/2 columns)
 //   tO     the row's O accumulator (D fp32 columns)
-//   j      block index within the tile's sequence; key0 = j * BC
+//   j      key block index; key0 = j * BC
+//   first  this is the first block the row sees (initialises the max)
 //   gj     running block index of this TMEM tile across the CTA's work
-//          (phases of the barriers); equals j when a CTA has one tile
+//          (phases of the barriers); equals j when a CTA has one tile and
+//          the blocks are not sparse
 //   q_tile first query row of the tile, grow this thread's query row
 //   o_done the two barriers that complete after P V of even / odd blocks
 // The caller has waited for S; the function waits for P_{j-1} V_{j-1} only
 // if it has to rescale O.  Returns false if that wait gave up.
 template <int BC, int D, bool CAUSAL>
 __device__ __forceinline__ bool softmax_block(RowState& st, uint32_t tS, uint32_t tO, int j,
-                                              int gj, int q_tile, int grow, int Nk, float sl2,
+                                              bool first, int gj, int q_tile, int grow, int Nk,
+                                              float sl2,
                                               uint64_t* o_done, volatile int* abort,
                                               DevStatus* status) {
   float s[BC];
@@ -104,7 +128,7 @@ __device__ __forceinline__ bool softmax_block(RowState& st, uint32_t tS, uint32_
     mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
   }
   const float mc = mx * sl2;
-  if (j == 0) {
+  if (first) {
     st.m = mc;
   } else {
     const bool need = mc > st.m + FA_RESCALE_LOG2_THRESHOLD;
@@ -223,6 +247,8 @@ struct FwdPairCfg {
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
+enum : uint32_t { KV_T0 = 1, KV_T1 = 2, KV_LAST = 4, KV_EMPTY = 8, KV_ACT0 = 16, KV_ACT1 = 32 };
+
 // The CTAs are persistent: grid = min(#units, #SMs) and CTA c takes units
 // c, c + grid, ...  A unit is (batch, head, tile pair); the list is
 // head-major so that concurrently running units share K/V in L2, and under
@@ -232,7 +258,11 @@ struct FwdPairCfg {
 // next Q load and "O free" (the epilogue has read O from TMEM) gates the
 // next unit's first P V, while the tensor pipe already computes the next
 // unit's first S.
-template <int D, bool CAUSAL>
+//
+// Block-sparse (SPARSE): a unit's K/V stream is the union of the key blocks
+// its two tiles see; a tile takes part in the blocks its own mask row keeps,
+// and a tile that sees none is written out as empty rows.
+template <int D, bool CAUSAL, bool SPARSE>
 __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
     fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
@@ -258,6 +288,11 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
   uint64_t* bar_drain = bars + 14 + 2 * NS;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 16 + 2 * NS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  // Block-sparse: the producer tags each K ring item with the tiles that
+  // take its block (KV_T0, KV_T1), the unit's last block (KV_LAST) and, on
+  // a unit's first item, the tiles that take any block (KV_ACT0, KV_ACT1);
+  // a unit that takes no block at all gets one KV_EMPTY item with no copy.
+  uint8_t* kv_meta = reinterpret_cast<uint8_t*>(tmem_holder + 2);   // [NS]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -291,7 +326,6 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
       nt[t] = (qt < p.Nq) ? (kv_end + BC - 1) / BC : 0;   // tile 1 may lie past Nq
     }
   };
-
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar_q + i, 1);
@@ -333,28 +367,60 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
         int bh, q0, nt[2];
         unit(u, bh, q0, nt);
         const int bkv = (bh / p.Hq) * p.Hkv + (bh % p.Hq) / p.group;
-        // Ring order = MMA consumption order: K0, V0, K1, V1, ...  The first
-        // ring items of a unit go out before its Q loads, which wait for the
-        // previous unit's epilogue to release the Q/staging buffers.
-        const int items = 2 * max(nt[0], nt[1]);
+        // Ring order = MMA consumption order: K0, V0, K1, V1, ... over the
+        // unit's (union of) key blocks.  The first ring items of a unit go
+        // out before its Q loads, which wait for the previous unit's
+        // epilogue to release the Q/staging buffers.
+        int cnt_t[2] = {nt[0], nt[1]}, nu = max(nt[0], nt[1]);
+        PairWalk pw;
+        uint32_t act = 0;
+        if constexpr (SPARSE) {
+          const uint8_t* row0 = p.mask + size_t(q0 / MASK_BLOCK) * p.mask_ld;
+          pw.init(row0, p.mask_ld, nt[0], nt[1]);
+          nu = pw.counts(cnt_t[0], cnt_t[1]);
+          act = (cnt_t[0] ? KV_ACT0 : 0u) | (cnt_t[1] ? KV_ACT1 : 0u);
+          if (nu == 0) {                             // one tagged item, no copy
+            const int slot = cnt % NS;
+            if (!(ok = mbar_wait(bar_kv_empty + slot, ((cnt / NS) & 1) ^ 1, abort_flag,
+                                 p.status, W_KV_EMPTY)))
+              break;
+            kv_meta[slot] = uint8_t(KV_EMPTY);
+            mbar_arrive(bar_kv_full + slot);
+            ++cnt;
+            continue;
+          }
+        }
+        const int items = 2 * nu;
+        int jc = -1;                               // key block of the latest K item
         auto ring = [&](int item) -> bool {
+          uint32_t meta = 0;
+          if constexpr (SPARSE) {
+            if (!(item & 1)) {
+              bool f0, f1;
+              jc = pw.next(jc + 1, f0, f1);
+              meta = (f0 ? KV_T0 : 0u) | (f1 ? KV_T1 : 0u) | (item + 2 == items ? KV_LAST : 0u) |
+                     (item == 0 ? act : 0u);
+            }
+          } else {
+            jc = item >> 1;
+          }
           const int slot = cnt % NS;
           if (!mbar_wait(bar_kv_empty + slot, ((cnt / NS) & 1) ^ 1, abort_flag, p.status,
                          W_KV_EMPTY))
             return false;
+          if (SPARSE && !(item & 1)) kv_meta[slot] = uint8_t(meta);
           mbar_arrive_expect_tx(bar_kv_full + slot, C::KV_BYTES);
           uint8_t* dst = sKV + slot * C::KV_BYTES;
           const CUtensorMap* tm = (item & 1) ? &tmV : &tmK;
           for (int c = 0; c < C::KCH; ++c)
-            tma_load_bh(dst + c * BC * 128, tm, bar_kv_full + slot, c * 64, (item >> 1) * BC, bkv,
-                        p.Hkv);
+            tma_load_bh(dst + c * BC * 128, tm, bar_kv_full + slot, c * 64, jc * BC, bkv, p.Hkv);
           ++cnt;
           return true;
         };
         const int early = min(items, NS);
         for (int it = 0; it < early && ok; ++it) ok = ring(it);
         for (int t = 0; t < 2 && ok; ++t) {
-          if (nt[t] == 0) continue;
+          if (cnt_t[t] == 0) continue;
           if (uses[t] > 0 &&
               !(ok = mbar_wait(bar_q_free + t, (uses[t] - 1) & 1, abort_flag, p.status, W_Q)))
             break;
@@ -430,38 +496,86 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
       for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
         int bh, q0, nt[2];
         unit(u, bh, q0, nt);
-        const int nmax = max(nt[0], nt[1]);
         int sK = 0, sV = 0;
-        if (!(ok = acquire(sK))) break;
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (nt[t] == 0) continue;
-          if (!(ok = mbar_wait(bar_q + t, uses[t] & 1, abort_flag, p.status, W_Q))) break;
-          tc_fence_after();
-          ++uses[t];
-          mma_s(t, sK);
-        }
-        if (!ok) break;
-        umma_commit(bar_kv_empty + sK);
-        // Per block j: P0 V_j, then S0_{j+1} (it overwrites P0_j in TMEM, so
-        // it must follow P0_j V_j; tcgen05 MMAs run in issue order), then the
-        // same for tile 1.  Each K/V slot is released after its last reader.
-        for (int j = 0; j < nmax && ok; ++j) {
-          if (!(ok = acquire(sV))) break;
-          if (j < nt[0] && !(ok = mma_pv(0, j, gb[0] + j, sV))) break;
-          const bool next = j + 1 < nmax;
-          if (next) {
-            if (!(ok = acquire(sK))) break;
-            if (j + 1 < nt[0]) mma_s(0, sK);
+        if constexpr (!SPARSE) {
+          const int nmax = max(nt[0], nt[1]);
+          if (!(ok = acquire(sK))) break;
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (nt[t] == 0) continue;
+            if (!(ok = mbar_wait(bar_q + t, uses[t] & 1, abort_flag, p.status, W_Q))) break;
+            tc_fence_after();
+            ++uses[t];
+            mma_s(t, sK);
           }
-          if (j < nt[1] && !(ok = mma_pv(1, j, gb[1] + j, sV))) break;
-          umma_commit(bar_kv_empty + sV);
-          if (next) {
-            if (j + 1 < nt[1]) mma_s(1, sK);
+          if (!ok) break;
+          umma_commit(bar_kv_empty + sK);
+          // Per block j: P0 V_j, then S0_{j+1} (it overwrites P0_j in TMEM,
+          // so it must follow P0_j V_j; tcgen05 MMAs run in issue order),
+          // then the same for tile 1.  Each K/V slot is released after its
+          // last reader.
+          for (int j = 0; j < nmax && ok; ++j) {
+            if (!(ok = acquire(sV))) break;
+            if (j < nt[0] && !(ok = mma_pv(0, j, gb[0] + j, sV))) break;
+            const bool next = j + 1 < nmax;
+            if (next) {
+              if (!(ok = acquire(sK))) break;
+              if (j + 1 < nt[0]) mma_s(0, sK);
+            }
+            if (j < nt[1] && !(ok = mma_pv(1, j, gb[1] + j, sV))) break;
+            umma_commit(bar_kv_empty + sV);
+            if (next) {
+              if (j + 1 < nt[1]) mma_s(1, sK);
+              umma_commit(bar_kv_empty + sK);
+            }
+          }
+          gb[0] += nt[0];
+          gb[1] += nt[1];
+        } else {
+          // The same order over the union of the tiles' key blocks, read
+          // from the K items' tags: a tile's S of its next block follows
+          // its own last P V, and l[t] counts the blocks tile t has taken.
+          if (!(ok = acquire(sK))) break;
+          uint32_t m = kv_meta[sK];
+          if (m & KV_EMPTY) {                        // the unit takes no block
             umma_commit(bar_kv_empty + sK);
+            continue;
           }
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (!(m & (KV_ACT0 << t))) continue;
+            if (!(ok = mbar_wait(bar_q + t, uses[t] & 1, abort_flag, p.status, W_Q))) break;
+            tc_fence_after();
+            ++uses[t];
+            if (m & (KV_T0 << t)) mma_s(t, sK);
+          }
+          if (!ok) break;
+          umma_commit(bar_kv_empty + sK);
+          int l[2] = {0, 0};
+          for (;;) {
+            const bool last = m & KV_LAST;
+            uint32_t mn = 0;
+            if (!(ok = acquire(sV))) break;
+            if (m & KV_T0) {
+              if (!(ok = mma_pv(0, l[0], gb[0] + l[0], sV))) break;
+              ++l[0];
+            }
+            if (!last) {
+              if (!(ok = acquire(sK))) break;
+              mn = kv_meta[sK];
+              if (mn & KV_T0) mma_s(0, sK);
+            }
+            if (m & KV_T1) {
+              if (!(ok = mma_pv(1, l[1], gb[1] + l[1], sV))) break;
+              ++l[1];
+            }
+            umma_commit(bar_kv_empty + sV);
+            if (last) break;
+            if (mn & KV_T1) mma_s(1, sK);
+            umma_commit(bar_kv_empty + sK);
+            m = mn;
+          }
+          gb[0] += l[0];
+          gb[1] += l[1];
         }
-        gb[0] += nt[0];
-        gb[1] += nt[1];
       }
       umma_commit(bar_drain);
       volatile int no_abort = 0;
@@ -482,19 +596,49 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
     for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
       int bh, q0, nt[2];
       unit(u, bh, q0, nt);
-      const int n = nt[t];
-      if (n == 0) continue;
+      if (nt[t] == 0) continue;                     // tile past Nq
+      int n = nt[t];
+      bool last_kept = true;
+      if constexpr (SPARSE) {
+        const uint8_t* row = p.mask + size_t(q0 / MASK_BLOCK + t) * p.mask_ld;
+        n = mask_count(row, nt[t]);
+        last_kept = __ldg(row + nt[t] - 1) != 0;
+      }
       const int q_tile = q0 + t * BR;
       const int grow = q_tile + row;
+      if constexpr (SPARSE) {
+        if (n == 0) {                               // sees no key
+          write_empty_row<D>(p, bh, grow);
+          continue;
+        }
+      }
       RowState st{-INFINITY, 0.f, 0.f};
-      for (int j = 0; j < n && ok; ++j) {
-        ok = mbar_wait(bar_s_full + t, (gb + j) & 1, abort_flag, p.status, W_S_FULL);
-        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-        tc_fence_after();
-        ok = softmax_block<BC, D, CAUSAL>(st, tl, tl + 128, j, gb + j, q_tile, grow, p.Nk,
-                                          p.scale_log2, o_done, abort_flag, p.status);
-        if (!ok) break;
-        mbar_arrive(bar_p_full + t);
+      if constexpr (!SPARSE) {
+        for (int j = 0; j < n && ok; ++j) {
+          ok = mbar_wait(bar_s_full + t, (gb + j) & 1, abort_flag, p.status, W_S_FULL);
+          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+          tc_fence_after();
+          ok = softmax_block<BC, D, CAUSAL>(st, tl, tl + 128, j, j == 0, gb + j, q_tile, grow,
+                                            p.Nk, p.scale_log2, o_done, abort_flag, p.status);
+          if (!ok) break;
+          mbar_arrive(bar_p_full + t);
+        }
+      } else {
+        // l: blocks taken so far (barrier phases).  Of the tile's blocks
+        // in range only the last one (nt - 1) can need the causal or
+        // key-length mask; every other kept block is passed as block 0,
+        // which needs neither when the tile has more than one block in
+        // range.
+        for (int l = 0; l < n && ok; ++l) {
+          const int j = (l == n - 1 && last_kept) ? nt[t] - 1 : 0;
+          ok = mbar_wait(bar_s_full + t, (gb + l) & 1, abort_flag, p.status, W_S_FULL);
+          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+          tc_fence_after();
+          ok = softmax_block<BC, D, CAUSAL>(st, tl, tl + 128, j, l == 0, gb + l, q_tile, grow,
+                                            p.Nk, p.scale_log2, o_done, abort_flag, p.status);
+          if (!ok) break;
+          mbar_arrive(bar_p_full + t);
+        }
       }
       if (!ok) break;
       const int jl = gb + n - 1;
@@ -536,7 +680,10 @@ struct FwdCfg {
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
-template <int D, bool CAUSAL>
+// Block-sparse (SPARSE): the tile walks only the key blocks its mask row
+// keeps (two 64-key blocks per mask block); the MMA issuer sees just the
+// sequence, the producer and softmax map it back to key blocks.
+template <int D, bool CAUSAL, bool SPARSE>
 __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -571,7 +718,26 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
   const int bkv = b * p.Hkv + h / p.group;
   const int q_row0 = qb * BR;
   const int kv_end = CAUSAL ? min(p.Nk, q_row0 + BR) : p.Nk;
-  const int n_blocks = (kv_end + BC - 1) / BC;
+  const int n_kv = (kv_end + BC - 1) / BC;             // key blocks in range
+  constexpr int SUB = MASK_BLOCK / BC;                 // key blocks per mask block
+  // Block-sparse: walks over the kept key blocks (one mask entry covers SUB
+  // of them); next_vis(rm, j) is the first kept block >= j, n_kv if none.
+  auto mask_row = [&](RowWalk& rm) {
+    rm.init(p.mask + size_t(qb) * p.mask_ld, (n_kv + SUB - 1) / SUB);
+  };
+  auto next_vis = [&](RowWalk& rm, int j) -> int {
+    if constexpr (!SPARSE) return min(j, n_kv);
+    if (j >= n_kv) return n_kv;
+    const int c = rm.next(j / SUB);
+    return c == MASK_NONE ? n_kv : max(j, c * SUB);
+  };
+  int n_blocks = n_kv;                                 // blocks the tile takes
+  if constexpr (SPARSE) {
+    RowWalk rm;
+    mask_row(rm);
+    n_blocks = 0;
+    for (int j = next_vis(rm, 0); j < n_kv; j = next_vis(rm, j + 1)) ++n_blocks;
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
@@ -599,7 +765,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    if (lane == 0 && n_blocks > 0) {
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
@@ -621,13 +787,22 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
           tma_load_bh(dst + c * BC * 128, tm, bar_kv_full + slot, c * 64, j * BC, bkv, p.Hkv);
         ++cnt;
       };
-      // Ring order = MMA consumption order: K0, K1, V0, K2, V1, ...
-      if (ok) load(&tmK, 0);
-      for (int j = 1; j < n_blocks && ok; ++j) {
-        load(&tmK, j);
-        if (ok) load(&tmV, j - 1);
+      // Ring order = MMA consumption order: K0, K1, V0, K2, V1, ... over the
+      // blocks the tile takes (jk: block of the latest K, jv: of the next V).
+      RowWalk rk, rv;
+      if constexpr (SPARSE) {
+        mask_row(rk);
+        mask_row(rv);
       }
-      if (ok) load(&tmV, n_blocks - 1);
+      int jk = next_vis(rk, 0), jv = jk;
+      if (ok) load(&tmK, jk);
+      for (int i = 1; i < n_blocks && ok; ++i) {
+        jk = next_vis(rk, jk + 1);
+        load(&tmK, jk);
+        if (ok) load(&tmV, jv);
+        jv = next_vis(rv, jv + 1);
+      }
+      if (ok) load(&tmV, jv);
       if (!ok) {
         // Let the copies already issued land before the CTA exits.
         for (int i = cnt - 1; i >= 0 && i >= cnt - NS; --i) {
@@ -638,7 +813,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
     }
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && n_blocks > 0) {
       constexpr uint32_t IDESC_S = idesc_bf16_f32(BR, BC, 0, 0);
       constexpr uint32_t IDESC_O = idesc_bf16_f32(BR, D, 0, 1);
       const uint32_t sQ_addr = smem_u32(sQ);
@@ -709,13 +884,19 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
     const int grow = q_row0 + row;
     RowState st{-INFINITY, 0.f, 0.f};
     bool ok = true;
-    for (int j = 0; j < n_blocks && ok; ++j) {
+    if (n_blocks == 0) {                                 // sees no key (sparse)
+      write_empty_row<D>(p, bh, grow);
+      ok = false;
+    }
+    RowWalk rm;
+    if constexpr (SPARSE) mask_row(rm);
+    for (int j = 0, jb = next_vis(rm, 0); j < n_blocks && ok; ++j, jb = next_vis(rm, jb + 1)) {
       ok = mbar_wait(bar_s_full + (j & 1), (j >> 1) & 1, abort_flag, p.status, W_S_FULL);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
-      ok = softmax_block<BC, D, CAUSAL>(st, tl + C::TM_S + (j & 1) * BC, tl + C::TM_O, j, j, q_row0,
-                                        grow, p.Nk, p.scale_log2, bar_o_done, abort_flag,
-                                        p.status);
+      ok = softmax_block<BC, D, CAUSAL>(st, tl + C::TM_S + (j & 1) * BC, tl + C::TM_O, jb, j == 0,
+                                        j, q_row0, grow, p.Nk, p.scale_log2, bar_o_done,
+                                        abort_flag, p.status);
       if (!ok) break;
       mbar_arrive(bar_p_full + (j & 1));
     }

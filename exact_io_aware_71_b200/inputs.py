@@ -80,6 +80,29 @@ def workloads() -> dict:
     return w
 
 
+MASK_BLOCK = 128
+
+
+def make_block_mask(Nq: int, Nk: int, density: float, seed: int, keep_diagonal: bool = True,
+                    empty_rows=()):
+    """Seeded block mask for block-sparse attention, uint8
+    [ceil(Nq/128), ceil(Nk/128)] on the CPU.  Each (query block, key block)
+    entry is kept with probability ``density`` (uniform draws from
+    ``torch.Generator('cpu').manual_seed(seed)``); with ``keep_diagonal``
+    the blocks (I, I) are always kept, so every query row sees some key;
+    query blocks listed in ``empty_rows`` are cleared entirely."""
+    nbq = (Nq + MASK_BLOCK - 1) // MASK_BLOCK
+    nbk = (Nk + MASK_BLOCK - 1) // MASK_BLOCK
+    g = torch.Generator("cpu").manual_seed(seed)
+    m = (torch.rand(nbq, nbk, generator=g) < density).to(torch.uint8)
+    if keep_diagonal:
+        i = torch.arange(min(nbq, nbk))
+        m[i, i] = 1
+    for r in empty_rows:
+        m[r] = 0
+    return m
+
+
 def make_inputs(wl: Workload, device="cpu", with_do: bool = True):
     """Return bf16 (q, k, v, dO) for a workload, drawn on the CPU.
 

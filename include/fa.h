@@ -115,6 +115,38 @@ int fa_bwd_strided(const void* q, const void* k, const void* v, const void* o, c
                    int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale,
                    void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/*
+ * Block-sparse attention (QbitAI FA1 article, results section: block-sparse
+ * FlashAttention).  A block mask removes whole blocks of the score matrix:
+ *   block_mask  device bytes, row-major [ceil(Nq / FA_MASK_BLOCK)]
+ *               [ceil(Nk / FA_MASK_BLOCK)], shared by every batch and head;
+ *               entry (I, J) != 0 keeps the FA_MASK_BLOCK x FA_MASK_BLOCK
+ *               block of query rows [I*128, I*128+128) and keys
+ *               [J*128, J*128+128) (clipped to Nq, Nk).  Read-only, owned by
+ *               the caller, unchanged until the kernels have finished.
+ * A removed block's scores count as -inf: the kernels neither load its K/V
+ * nor compute it, so the work shrinks with the fraction of blocks kept.
+ * With causal = 1 both masks apply.  A query row left with no visible key
+ * gets O = 0 and lse = -inf (the limits of an empty softmax), and adds
+ * nothing to any gradient.  An all-ones mask computes the dense result.
+ * strides: as for fa_fwd_strided / fa_bwd_strided (4 or 8 entries), or NULL
+ * for contiguous [B, H, N, d] tensors.  Everything else is as for fa_fwd and
+ * fa_bwd; the backward workspace is fa_bwd_workspace_size(...).  The same
+ * mask must be passed to both passes.
+ */
+#define FA_MASK_BLOCK 128
+
+int fa_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                        const fa_strides* strides, const unsigned char* block_mask, int B, int Hq,
+                        int Hkv, int Nq, int Nk, int d, int causal, float scale,
+                        cudaStream_t stream);
+
+int fa_bwd_block_sparse(const void* q, const void* k, const void* v, const void* o,
+                        const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                        const fa_strides* strides, const unsigned char* block_mask, int B, int Hq,
+                        int Hkv, int Nq, int Nk, int d, int causal, float scale, void* workspace,
+                        size_t workspace_bytes, cudaStream_t stream);
+
 /* Stages of fa_bwd, for callers that time or schedule them separately. */
 typedef enum {
   FA_BWD_ALL = 0,   /* the whole backward pass (same as fa_bwd) */

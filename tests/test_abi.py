@@ -125,3 +125,20 @@ def test_missing_library_fails_loudly(tmp_path):
             binding.load(str(tmp_path / "nope.so"))
     finally:
         binding._lib = saved
+
+
+def test_block_sparse_rejects_bad_arguments():
+    """A null mask is rejected; otherwise the sparse entry points run the
+    same argument checks as the dense ones (NULL strides = contiguous)."""
+    assert fa.fa_fwd_block_sparse(A, A, A, A, A, None, None, 1, 2, 2, 128, 128, 64, 0, 0.125,
+                                  None) == 1
+    assert fa.fa_bwd_block_sparse(A, A, A, A, A, A, A, A, A, None, None, 1, 2, 2, 128, 128, 64,
+                                  0, 0.125, A, 1 << 40, None) == 1
+    assert fa.fa_fwd_block_sparse(A, A, A, A, A, None, A, 1, 2, 2, 128, 128, 96, 0, 0.125,
+                                  None) == 2
+    assert fa.fa_fwd_block_sparse(A + 8, A, A, A, A, None, A, 1, 2, 2, 128, 128, 64, 0, 0.125,
+                                  None) == 3
+    assert fa.fa_bwd_block_sparse(A, A, A, A, A, A, A, A, A, None, A, 1, 2, 2, 128, 128, 64, 0,
+                                  0.125, None, 0, None) == 4
+    assert fa.fa_fwd_block_sparse(A, A, A, A, A, None, A, 0, 2, 2, 128, 128, 64, 0, 0.125,
+                                  None) == 1

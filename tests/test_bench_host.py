@@ -83,3 +83,32 @@ def test_peaks_fallback(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     pk, src = bench.load_peaks()
     assert src == "fallback" and pk["bf16_tflops"] == 1590.0
+
+
+def test_kept_fraction_of_block_masks():
+    """The FLOP scale of block-sparse steps: visible (query, key) pairs over
+    those of the dense problem, counted per element on small cases."""
+    import numpy as np
+    from exact_io_aware_71_b200.inputs import Workload
+    for causal in (False, True):
+        for nq, nk in ((300, 300), (260, 400), (400, 130)):
+            wl = Workload("t", 1, 1, 1, nq, nk, 64, causal, 0)
+            rng = np.random.default_rng(nq + nk)
+            m = rng.random(((nq + 127) // 128, (nk + 127) // 128)) < 0.5
+            i = np.arange(nq)[:, None]
+            j = np.arange(nk)[None, :]
+            vis = m[i // 128, j // 128]
+            base = (j <= i) if causal else np.ones((nq, nk), bool)
+            assert bench.kept_fraction(wl, m) == pytest.approx((vis & base).sum() / base.sum())
+            assert bench.kept_fraction(wl, None) == 1.0
+            assert bench.kept_fraction(wl, np.ones_like(m)) == pytest.approx(1.0)
+
+
+def test_launches_per_step():
+    from exact_io_aware_71_b200.inputs import workloads
+    w = workloads()
+    assert bench.launches_per_step(w["train_b8h16n2048d128_full"], 148) == 4
+    # 32 query heads on one kv head, 128 key blocks: split, plus the dK/dV convert
+    assert bench.launches_per_step(w["long_gqa_hkv1_n16384_d128_causal"], 148) == 5
+    # 8 kv heads x 128 key blocks = 1024 CTAs: no split
+    assert bench.launches_per_step(w["long_gqa_hkv8_n16384_d128_causal"], 148) == 4
