@@ -39,6 +39,13 @@ Readings where the pages are silent (all listed in the design notes):
     "two small changes") maps query head h to kv head h // (Hq // Hkv).
   * Causal masking is top-left aligned: key j is visible to query i iff j <= i.
   * LSE is the natural-log logsumexp of the *scaled* scores.
+  * Variable-length batches (not named on the pages; the FA2 article's
+    section on parallelism over the sequence for small batches is the
+    nearest passage): B sequences of different lengths are packed back to
+    back, q as [total_q, Hq, d] and k, v as [total_k, Hkv, d], with
+    cumulative offsets cu_q, cu_k of length B + 1.  Sequence b attends only
+    within itself, causal top-left within the sequence; a sequence with
+    queries but no keys gives O = 0, LSE = -inf.  LSE is [Hq, total_q].
   * Block-sparse attention (QbitAI FA1 article, results section, names
     block-sparse FlashAttention without defining it) takes a block mask of
     128 x 128 (query, key) blocks, shared by all batches and heads; a zero
@@ -56,6 +63,8 @@ import numpy as np
 
 __all__ = [
     "BLOCK",
+    "attention_forward_varlen",
+    "attention_backward_varlen",
     "kv_head",
     "scores",
     "attention_forward",
@@ -227,3 +236,49 @@ def attention_backward_dq_rows(q, k, v, do, causal: bool, scale: float, b: int, 
     d_row = (p * dp).sum(axis=1)
     ds = p * (dp - d_row[:, None])
     return scale * (ds @ kk)
+
+
+# ------------------------------------------------------------------ variable-length batches
+def _seq_views(x, cu, b):
+    """Rows cu[b]:cu[b+1] of a packed [total, H, d] tensor as [1, H, n, d]."""
+    return np.ascontiguousarray(_as64(x[cu[b]:cu[b + 1]]).transpose(1, 0, 2)[None])
+
+
+def attention_forward_varlen(q, k, v, cu_q, cu_k, causal: bool, scale: float):
+    """Exact attention of B packed sequences, each on its own.
+
+    q: [total_q, Hq, d]; k, v: [total_k, Hkv, d]; cu_q, cu_k: [B + 1]
+    cumulative offsets (non-decreasing, starting at 0).  Returns
+    (O [total_q, Hq, d], LSE [Hq, total_q]) in fp64."""
+    cu_q, cu_k = [int(x) for x in cu_q], [int(x) for x in cu_k]
+    hq, d = q.shape[1], q.shape[2]
+    o = np.zeros((q.shape[0], hq, d))
+    lse = np.full((hq, q.shape[0]), -np.inf)
+    for b in range(len(cu_q) - 1):
+        nq, nk = cu_q[b + 1] - cu_q[b], cu_k[b + 1] - cu_k[b]
+        if nq == 0 or nk == 0:
+            continue                      # no rows, or rows that see no key (O = 0)
+        ob, lb = attention_forward(_seq_views(q, cu_q, b), _seq_views(k, cu_k, b),
+                                   _seq_views(v, cu_k, b), causal, scale)
+        o[cu_q[b]:cu_q[b + 1]] = ob[0].transpose(1, 0, 2)
+        lse[:, cu_q[b]:cu_q[b + 1]] = lb[0]
+    return o, lse
+
+
+def attention_backward_varlen(q, k, v, do, cu_q, cu_k, causal: bool, scale: float):
+    """Gradients of sum(O * dO) for attention_forward_varlen; returns
+    (dQ [total_q, Hq, d], dK, dV [total_k, Hkv, d]) in fp64."""
+    cu_q, cu_k = [int(x) for x in cu_q], [int(x) for x in cu_k]
+    dq = np.zeros(q.shape)
+    dk = np.zeros(k.shape)
+    dv = np.zeros(v.shape)
+    for b in range(len(cu_q) - 1):
+        nq, nk = cu_q[b + 1] - cu_q[b], cu_k[b + 1] - cu_k[b]
+        if nq == 0 or nk == 0:
+            continue
+        g = attention_backward(_seq_views(q, cu_q, b), _seq_views(k, cu_k, b),
+                               _seq_views(v, cu_k, b), _seq_views(do, cu_q, b), causal, scale)
+        dq[cu_q[b]:cu_q[b + 1]] = g[0][0].transpose(1, 0, 2)
+        dk[cu_k[b]:cu_k[b + 1]] = g[1][0].transpose(1, 0, 2)
+        dv[cu_k[b]:cu_k[b + 1]] = g[2][0].transpose(1, 0, 2)
+    return dq, dk, dv
