@@ -15,6 +15,11 @@ from .binding import (  # noqa: F401
     fa_fwd_block_sparse,
     fa_bwd_block_sparse,
     MASK_BLOCK,
+    fa_fwd_varlen,
+    fa_bwd_varlen,
+    fa_bwd_varlen_workspace_size,
+    forward_varlen,
+    backward_varlen,
     FaStrides,
     strides_of,
     fa_bwd_workspace_size,

@@ -24,7 +24,8 @@ STATUS_NAMES = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED",
 # Exported symbols declared in include/fa.h.
 SYMBOLS = ("fa_fwd", "fa_bwd", "fa_bwd_stage", "fa_bwd_workspace_size", "fa_status_string",
            "fa_device_status", "fa_bwd_noalloc", "fa_debug_inject", "fa_fwd_strided",
-           "fa_bwd_strided", "fa_fwd_block_sparse", "fa_bwd_block_sparse")
+           "fa_bwd_strided", "fa_fwd_block_sparse", "fa_bwd_block_sparse", "fa_fwd_varlen",
+           "fa_bwd_varlen", "fa_bwd_varlen_workspace_size")
 
 # Rows / keys per block-mask entry (FA_MASK_BLOCK).
 MASK_BLOCK = 128
@@ -82,6 +83,12 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fa_fwd_block_sparse.restype = i
     lib.fa_bwd_block_sparse.argtypes = [vp] * 9 + [sp, vp] + [i] * 7 + [f, vp, sz, vp]
     lib.fa_bwd_block_sparse.restype = i
+    lib.fa_fwd_varlen.argtypes = [vp] * 7 + [i] * 9 + [f, vp]
+    lib.fa_fwd_varlen.restype = i
+    lib.fa_bwd_varlen.argtypes = [vp] * 11 + [i] * 9 + [f, vp, sz, vp]
+    lib.fa_bwd_varlen.restype = i
+    lib.fa_bwd_varlen_workspace_size.argtypes = [i] * 6
+    lib.fa_bwd_varlen_workspace_size.restype = sz
     lib.fa_bwd_noalloc.argtypes = lib.fa_bwd.argtypes[:17] + [vp]
     lib.fa_bwd_noalloc.restype = i
     lib.fa_bwd_workspace_size.argtypes = [i, i, i, i, i, i, i]
@@ -128,6 +135,23 @@ def fa_bwd_block_sparse(q, k, v, o, lse, dO, dq, dk, dv, strides, block_mask, B,
     return load().fa_bwd_block_sparse(q, k, v, o, lse, dO, dq, dk, dv, arr, block_mask, B, Hq,
                                       Hkv, Nq, Nk, d, int(causal), float(scale), workspace,
                                       workspace_bytes, stream)
+
+
+def fa_fwd_varlen(q, k, v, o, lse, cu_q, cu_k, B, max_q, max_k, total_q, total_k, Hq, Hkv, d,
+                  causal, scale, stream) -> int:
+    return load().fa_fwd_varlen(q, k, v, o, lse, cu_q, cu_k, B, max_q, max_k, total_q, total_k,
+                                Hq, Hkv, d, int(causal), float(scale), stream)
+
+
+def fa_bwd_varlen(q, k, v, o, lse, dO, dq, dk, dv, cu_q, cu_k, B, max_q, max_k, total_q, total_k,
+                  Hq, Hkv, d, causal, scale, workspace, workspace_bytes, stream) -> int:
+    return load().fa_bwd_varlen(q, k, v, o, lse, dO, dq, dk, dv, cu_q, cu_k, B, max_q, max_k,
+                                total_q, total_k, Hq, Hkv, d, int(causal), float(scale),
+                                workspace, workspace_bytes, stream)
+
+
+def fa_bwd_varlen_workspace_size(B, total_q, total_k, Hq, Hkv, d) -> int:
+    return load().fa_bwd_varlen_workspace_size(B, total_q, total_k, Hq, Hkv, d)
 
 
 def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, causal, scale,
@@ -244,4 +268,55 @@ def backward(q, k, v, o, lse, do, causal: bool, scale: float, workspace=None, gr
         what = "fa_bwd_block_sparse"
     if st != FA_OK:
         raise FaError(st, what)
+    return dq, dk, dv
+
+
+def _varlen_dims(q, k, cu_q, cu_k):
+    import torch
+    for t in (q, k):
+        if t.dim() != 3 or not t.is_contiguous():
+            raise ValueError("packed q / k / v must be contiguous [total, H, d]")
+    for c in (cu_q, cu_k):
+        if c.dtype != torch.int32 or not c.is_cuda or not c.is_contiguous() or c.dim() != 1:
+            raise ValueError("cu_seqlens must be contiguous int32 CUDA vectors of length B + 1")
+    if cu_q.numel() != cu_k.numel() or cu_q.numel() < 2:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must both have B + 1 >= 2 entries")
+    return cu_q.numel() - 1, q.shape[0], k.shape[0], q.shape[1], k.shape[1], q.shape[2]
+
+
+def forward_varlen(q, k, v, cu_q, cu_k, max_q, max_k, causal: bool, scale: float, out=None,
+                   lse=None):
+    """O [total_q, Hq, d] and LSE [Hq, total_q] of a packed variable-length
+    batch (q [total_q, Hq, d], k / v [total_k, Hkv, d], int32 cumulative
+    offsets cu_q / cu_k of length B + 1, all on the GPU)."""
+    import torch
+    B, tq, tk, Hq, Hkv, d = _varlen_dims(q, k, cu_q, cu_k)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(Hq, tq, dtype=torch.float32, device=q.device)
+    st = fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                       cu_q.data_ptr(), cu_k.data_ptr(), B, int(max_q), int(max_k), tq, tk, Hq,
+                       Hkv, d, causal, scale, _stream_handle())
+    if st != FA_OK:
+        raise FaError(st, "fa_fwd_varlen")
+    return out, lse
+
+
+def backward_varlen(q, k, v, o, lse, do, cu_q, cu_k, max_q, max_k, causal: bool, scale: float,
+                    workspace=None):
+    """dQ, dK, dV (packed, bf16) of a variable-length batch."""
+    import torch
+    B, tq, tk, Hq, Hkv, d = _varlen_dims(q, k, cu_q, cu_k)
+    need = fa_bwd_varlen_workspace_size(B, tq, tk, Hq, Hkv, d)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    st = fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                       do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                       cu_q.data_ptr(), cu_k.data_ptr(), B, int(max_q), int(max_k), tq, tk, Hq,
+                       Hkv, d, causal, scale, workspace.data_ptr(), workspace.numel(),
+                       _stream_handle())
+    if st != FA_OK:
+        raise FaError(st, "fa_bwd_varlen")
     return dq, dk, dv

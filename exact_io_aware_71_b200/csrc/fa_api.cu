@@ -135,15 +135,15 @@ int launch_kernel(KernelT kern, int smem, int threads, unsigned grid, const CUte
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-// d = 64 / 128: two query tiles per CTA; d = 256: one.  SPARSE: p.mask is a
-// block mask.
-template <int D, bool CAUSAL, bool SPARSE>
+// d = 64 / 128: two query tiles per CTA; d = 256: one.  MODE: dense,
+// block-sparse (p.mask) or packed variable-length batch (p.cu_q, p.cu_k).
+template <int D, bool CAUSAL, int MODE>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                const CUtensorMap& mo, FwdParams p, cudaStream_t stream) {
   if constexpr (D == 256) {
     using C = FwdCfg<D>;
     p.n_units = p.n_qblocks;
-    return launch_kernel(fa_fwd_kernel<D, CAUSAL, SPARSE>, C::SMEM_BYTES, C::NTHREADS,
+    return launch_kernel(fa_fwd_kernel<D, CAUSAL, MODE>, C::SMEM_BYTES, C::NTHREADS,
                          unsigned(p.n_units) * unsigned(p.B * p.Hq), mq, mk, mv, mo, p, stream);
   } else {
     using C = FwdPairCfg<D>;
@@ -152,7 +152,7 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
     static int regs = -1;
     if (regs < 0) {
       cudaFuncAttributes fattr;
-      if (cudaFuncGetAttributes(&fattr, fa_fwd_pair_kernel<D, CAUSAL, SPARSE>) != cudaSuccess)
+      if (cudaFuncGetAttributes(&fattr, fa_fwd_pair_kernel<D, CAUSAL, MODE>) != cudaSuccess)
         return FA_ERR_CUDA;
       regs = fattr.numRegs;
     }
@@ -170,7 +170,7 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
     const long long units = (long long)p.n_units * p.B * p.Hq;
     const bool persistent = p.Nk <= 4096 || (CAUSAL && p.Nk <= 16384);
     const unsigned grid = unsigned(persistent ? std::min<long long>(units, sms) : units);
-    return launch_kernel(fa_fwd_pair_kernel<D, CAUSAL, SPARSE>, C::SMEM_BYTES, C::NTHREADS, grid,
+    return launch_kernel(fa_fwd_pair_kernel<D, CAUSAL, MODE>, C::SMEM_BYTES, C::NTHREADS, grid,
                          mq, mk, mv, mo, p, stream);
   }
 }
@@ -178,8 +178,20 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
 template <int D, bool CAUSAL>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                const CUtensorMap& mo, const FwdParams& p, cudaStream_t stream) {
-  return p.mask ? launch_fwd<D, CAUSAL, true>(mq, mk, mv, mo, p, stream)
-                : launch_fwd<D, CAUSAL, false>(mq, mk, mv, mo, p, stream);
+  return p.cu_q ? launch_fwd<D, CAUSAL, MODE_VARLEN>(mq, mk, mv, mo, p, stream)
+         : p.mask ? launch_fwd<D, CAUSAL, MODE_SPARSE>(mq, mk, mv, mo, p, stream)
+                  : launch_fwd<D, CAUSAL, MODE_DENSE>(mq, mk, mv, mo, p, stream);
+}
+
+int launch_fwd_any(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                   const CUtensorMap& mo, const FwdParams& p, int d, int causal,
+                   cudaStream_t stream) {
+  if (d == 64) return causal ? launch_fwd<64, true>(mq, mk, mv, mo, p, stream)
+                             : launch_fwd<64, false>(mq, mk, mv, mo, p, stream);
+  if (d == 128) return causal ? launch_fwd<128, true>(mq, mk, mv, mo, p, stream)
+                              : launch_fwd<128, false>(mq, mk, mv, mo, p, stream);
+  return causal ? launch_fwd<256, true>(mq, mk, mv, mo, p, stream)
+                : launch_fwd<256, false>(mq, mk, mv, mo, p, stream);
 }
 
 // The forward pass on strided tensors, with an optional block mask.
@@ -218,13 +230,65 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse,
   p.mask_ld = (Nk + MASK_BLOCK - 1) / MASK_BLOCK;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.o_sb = so.b; p.o_sh = so.h; p.o_sn = so.n;
+  p.cu_q = p.cu_k = nullptr;
+  p.total_q = Nq;
+  p.total_k = Nk;
+  return launch_fwd_any(mq, mk, mv, mo, p, d, causal, stream);
+}
 
-  if (d == 64) return causal ? launch_fwd<64, true>(mq, mk, mv, mo, p, stream)
-                             : launch_fwd<64, false>(mq, mk, mv, mo, p, stream);
-  if (d == 128) return causal ? launch_fwd<128, true>(mq, mk, mv, mo, p, stream)
-                              : launch_fwd<128, false>(mq, mk, mv, mo, p, stream);
-  return causal ? launch_fwd<256, true>(mq, mk, mv, mo, p, stream)
-                : launch_fwd<256, false>(mq, mk, mv, mo, p, stream);
+// Checks shared by the packed variable-length entry points.
+int check_varlen(const int* cu_q, const int* cu_k, int B, int max_q, int max_k, int total_q,
+                 int total_k, int Hq, int Hkv, int d, int causal, float scale) {
+  if (!cu_q || !cu_k) return FA_ERR_INVALID_ARG;
+  if (total_q < 1 || total_k < 1) return FA_ERR_INVALID_ARG;
+  int st = check_sizes(B, Hq, Hkv, max_q, max_k, d, causal, scale);
+  if (st != FA_OK) return st;
+  if (!aligned4(cu_q) || !aligned4(cu_k)) return FA_ERR_MISALIGNED;
+  if (int64_t(Hq) * total_q * d >= (int64_t(1) << 40) || int64_t(B) + 1 >= (int64_t(1) << 24))
+    return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+// Element strides of packed [total, H, d] tensors, seen as [1, H, total, d].
+Strides packed(int H, int total, int d) {
+  return Strides{(long long)total * H * d, (long long)d, (long long)H * d};
+}
+
+int fwd_varlen_impl(const void* q, const void* k, const void* v, void* o, float* lse,
+                    const int* cu_q, const int* cu_k, int B, int max_q, int max_k, int total_q,
+                    int total_k, int Hq, int Hkv, int d, int causal, float scale,
+                    cudaStream_t stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  int st = check_varlen(cu_q, cu_k, B, max_q, max_k, total_q, total_k, Hq, Hkv, d, causal, scale);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(lse))
+    return FA_ERR_MISALIGNED;
+  const Strides sq = packed(Hq, total_q, d), sk = packed(Hkv, total_k, d);
+  const int bc = (d == 256) ? 64 : 128;
+  CUtensorMap mq, mk, mv, mo;
+  if (!make_map_bf16(&mq, q, d, total_q, Hq, 1, sq, 128) ||
+      !make_map_bf16(&mk, k, d, total_k, Hkv, 1, sk, bc) ||
+      !make_map_bf16(&mv, v, d, total_k, Hkv, 1, sk, bc) ||
+      !make_map_bf16(&mo, o, d, total_q, Hq, 1, sq, 32))
+    return FA_ERR_CUDA;
+  FwdParams p;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Nq = max_q; p.Nk = max_k;
+  p.group = Hq / Hkv;
+  p.n_qblocks = (max_q + 127) / 128;
+  p.causal = causal;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.lse = lse;
+  p.status = status_ptr();
+  if (!p.status) return FA_ERR_CUDA;
+  p.mask = nullptr;
+  p.mask_ld = 0;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.o_sb = sq.b; p.o_sh = sq.h; p.o_sn = sq.n;
+  p.cu_q = cu_q;
+  p.cu_k = cu_k;
+  p.total_q = total_q;
+  p.total_k = total_k;
+  return launch_fwd_any(mq, mk, mv, mo, p, d, causal, stream);
 }
 
 // Element strides of the contiguous layouts of q, k, v, o.
@@ -323,7 +387,7 @@ int bwd_impl(int stage, const void* q, const void* k, const void* v, const void*
   Strides s8[8];
   for (int i = 0; i < 8; ++i) s8[i] = Strides{strides[i].batch, strides[i].head, strides[i].row};
   return launch_bwd(stages, q, k, v, o, lse, dO, dq, dk, dv, s8, B, Hq, Hkv, Nq, Nk, d, causal,
-                    scale, mask, workspace, sp, stream);
+                    scale, mask, nullptr, workspace, sp, stream);
 }
 
 void contiguous8(fa_strides* s, int Hq, int Hkv, int Nq, int Nk, int d) {
@@ -392,6 +456,44 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
   if (!scratch) return FA_ERR_CUDA;
   return fa_bwd_stage(FA_BWD_ALL, q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, causal,
                       scale, scratch, FA_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+size_t fa_bwd_varlen_workspace_size(int B, int total_q, int total_k, int Hq, int Hkv, int d) {
+  if (B < 1 || total_q < 1 || total_k < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return 0;
+  if (d != 64 && d != 128 && d != 256) return 0;
+  return bwd_workspace_layout_varlen(B, Hq, Hkv, total_q, total_k, d).total;
+}
+
+int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                  const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int max_seqlen_q,
+                  int max_seqlen_k, int total_q, int total_k, int Hq, int Hkv, int d, int causal,
+                  float scale, cudaStream_t stream) {
+  return fwd_varlen_impl(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q,
+                         max_seqlen_k, total_q, total_k, Hq, Hkv, d, causal, scale, stream);
+}
+
+int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                  const void* dO, void* dq, void* dk, void* dv, const int* cu_seqlens_q,
+                  const int* cu_seqlens_k, int B, int max_seqlen_q, int max_seqlen_k,
+                  int total_q, int total_k, int Hq, int Hkv, int d, int causal, float scale,
+                  void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  int st = check_varlen(cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k, total_q,
+                        total_k, Hq, Hkv, d, causal, scale);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(lse) ||
+      !aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_MISALIGNED;
+  const size_t need = bwd_workspace_layout_varlen(B, Hq, Hkv, total_q, total_k, d).total;
+  if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
+  DevStatus* sp = status_ptr();
+  if (!sp) return FA_ERR_CUDA;
+  const Strides a = packed(Hq, total_q, d), b = packed(Hkv, total_k, d);
+  const Strides s8[8] = {a, b, b, a, a, a, b, b};   // q, k, v, o, dO, dq, dk, dv
+  const Varlen vl{cu_seqlens_q, cu_seqlens_k, total_q, total_k};
+  return launch_bwd(7, q, k, v, o, lse, dO, dq, dk, dv, s8, B, Hq, Hkv, max_seqlen_q,
+                    max_seqlen_k, d, causal, scale, nullptr, &vl, workspace, sp, stream);
 }
 
 int fa_device_status(cudaStream_t stream, int* where) {

@@ -68,7 +68,6 @@ struct BwdCfg {
 
 inline int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
-// Workspace: dQacc fp32 [B*Hq, Nq, d] | Dpad fp32 [B*Hq, Nq_pad] | Lpad fp32 [B*Hq, Nq_pad]
 // Workspace: dQacc fp32 [B*Hq, Nq, d] | Dpad fp32 [B*Hq, Nq_pad] |
 // Lpad fp32 [B*Hq, Nq_pad] | (GQA/MQA only) dKacc, dVacc fp32 [B*Hkv, Nk, d]
 // for the partial sums of a kv group split across CTAs.
@@ -92,6 +91,27 @@ inline size_t bwd_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d)
   return bwd_workspace_layout(B, Hq, Hkv, Nq, Nk, d).total;
 }
 
+// Packed variable-length batch of B sequences: dQacc fp32 [Hq, total_q, d] |
+// Dpad, Lpad fp32 [Hq, ld] with ld = round_up(total_q, 4) + 128 (B + 1),
+// each sequence's rows starting at varlen_pad_start | (GQA/MQA only)
+// dKacc, dVacc fp32 [Hkv, total_k, d].
+inline long long varlen_lpad_ld(int B, int total_q) {
+  return (long long)((total_q + 3) & ~3) + 128LL * (B + 1);
+}
+inline BwdWorkspace bwd_workspace_layout_varlen(int B, int Hq, int Hkv, int total_q, int total_k,
+                                                int d) {
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  const size_t ld = size_t(varlen_lpad_ld(B, total_q));
+  BwdWorkspace w;
+  w.dq_off = 0;
+  w.d_off = up(size_t(Hq) * total_q * d * 4);
+  w.l_off = w.d_off + up(size_t(Hq) * ld * 4);
+  w.kv_off = w.l_off + up(size_t(Hq) * ld * 4);
+  w.kv_elems = (Hq > Hkv) ? size_t(Hkv) * total_k * d : 0;
+  w.total = w.kv_off + up(2 * w.kv_elems * 4);
+  return w;
+}
+
 // ------------------------------------------------------------------ pre
 // One group of D/8 threads per row; each thread handles 8 consecutive
 // elements (16 bytes) of O and dO and zeroes 8 floats of dQacc.
@@ -99,6 +119,19 @@ inline size_t bwd_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d)
 struct Strides {
   long long b, h, n;
 };
+
+// Packed-batch helpers: sequence b's rows clamped to [0, total], and where
+// its padded fp32 row vectors (D, LSE) start in a head's workspace row:
+// 16-byte aligned, with room for ceil(n / 64) * 64 entries before the next
+// sequence (each sequence adds 128 entries of slack).
+__device__ __forceinline__ void varlen_rows(const int* cu, int b, int total, int& off, int& n) {
+  const int a = min(max(__ldg(cu + b), 0), total);
+  n = min(max(__ldg(cu + b + 1), a), total) - a;
+  off = a;
+}
+__device__ __forceinline__ long long varlen_pad_start(int off, int b) {
+  return (long long)((off + 3) & ~3) + 128LL * b;
+}
 
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(
@@ -146,6 +179,88 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(
     }
   }
   // dK/dV partial-sum accumulators (only when a kv group is split across CTAs)
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < kv_n4;
+       i += (long long)gridDim.x * blockDim.x)
+    reinterpret_cast<float4*>(kvacc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// The same for a packed variable-length batch: o and dO are [total_q, Hq, d]
+// at strides so / sdo (batch stride unused), lse is [Hq, total_q], dQacc is
+// [Hq, total_q, d].  Row n of the packed tensors belongs to the sequence b
+// with cu_q[b] <= n < cu_q[b+1] (found by bisection); its D and LSE*log2(e)
+// go to h * ld + varlen_pad_start(cu_q[b], b) + (n - cu_q[b]).  Afterwards
+// the entries from each sequence's length up to the next multiple of 64
+// are padding: D = 0, LSE = +inf, so the main kernel's P is 0 there.
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_pre_varlen_kernel(
+    const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
+    const float* __restrict__ lse, float* __restrict__ dqacc, float* __restrict__ Dpad,
+    float* __restrict__ Lpad, const int* __restrict__ cu_q, int B, int Hq, int total_q,
+    long long ld, Strides so, Strides sdo, float* __restrict__ kvacc, long long kv_n4) {
+  constexpr int TPR = D / 8;
+  constexpr int RPB = 256 / TPR;
+  const int sub = threadIdx.x % TPR;
+  const int rlocal = threadIdx.x / TPR;
+  auto start = [&](int bb) { return min(max(__ldg(cu_q + bb), 0), total_q); };
+  // The loop bound is a multiple of RPB so that every warp runs its
+  // shuffles with all lanes; rows past the end only do nothing.
+  const long long total = (long long)Hq * total_q;
+  const long long total_pad = (total + RPB - 1) / RPB * RPB;
+  for (long long r = (long long)blockIdx.x * RPB + rlocal; r < total_pad;
+       r += (long long)gridDim.x * RPB) {
+    const bool valid = r < total;
+    const int h = valid ? int(r / total_q) : 0;
+    const int n = valid ? int(r - (long long)h * total_q) : 0;
+    int lo = 0, hi = B - 1;                        // last sequence starting at or before n
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (start(mid) <= n) lo = mid; else hi = mid - 1;
+    }
+    const int off = start(lo);
+    const int len = min(max(__ldg(cu_q + lo + 1), off), total_q) - off;
+    const bool in_seq = valid && n >= off && n < off + len;
+    float acc = 0.f;
+    if (valid) {
+      const uint4 ov = *reinterpret_cast<const uint4*>(o + h * so.h + (long long)n * so.n +
+                                                       sub * 8);
+      const uint4 dv = *reinterpret_cast<const uint4*>(dO + h * sdo.h + (long long)n * sdo.n +
+                                                       sub * 8);
+      const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
+      const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 a = __bfloat1622float2(o2[i]);
+        const float2 b2 = __bfloat1622float2(d2[i]);
+        acc = fmaf(a.x, b2.x, acc);
+        acc = fmaf(a.y, b2.y, acc);
+      }
+      float4* z = reinterpret_cast<float4*>(dqacc + ((size_t)h * total_q + n) * D + sub * 8);
+      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int s = TPR / 2; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+    if (sub == 0 && in_seq) {
+      const long long pi = h * ld + varlen_pad_start(off, lo) + (n - off);
+      Dpad[pi] = acc;
+      Lpad[pi] = lse[(size_t)h * total_q + n] * 1.4426950408889634f;
+    }
+  }
+  // padding entries of every (head, sequence)
+  const long long npad = (long long)Hq * B * 64;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < npad;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int e = int(i % 64);
+    const int bb = int((i / 64) % B);
+    const int h = int(i / (64LL * B));
+    const int off = start(bb);
+    const int len = min(max(__ldg(cu_q + bb + 1), off), total_q) - off;
+    if (len + e < ((len + 63) & ~63)) {
+      const long long pi = h * ld + varlen_pad_start(off, bb) + len + e;
+      Dpad[pi] = 0.f;
+      Lpad[pi] = INFINITY;
+    }
+  }
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < kv_n4;
        i += (long long)gridDim.x * blockDim.x)
     reinterpret_cast<float4*>(kvacc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -218,7 +333,22 @@ struct BwdParams {
   DevStatus* status;
   const uint8_t* mask;  // block-sparse only: [ceil(Nq/128)][mask_ld] block mask
   int mask_ld;          // ceil(Nk / 128)
+  // Variable-length batches only: B packed sequences (cu_q / cu_k offsets,
+  // clamped to the totals on the device); Nq / Nk are the longest lengths.
+  // The workspace's D / LSE rows of sequence b at head h start at
+  // h * lpad_ld + varlen_pad_start(b); dK / dV rows that a TMA box would
+  // overrun into the next sequence are stored directly through dk / dv.
+  const int* cu_q;
+  const int* cu_k;
+  int total_q, total_k;
+  long long lpad_ld;
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  Strides sdk, sdv;
 };
+
+enum : int { BMODE_DENSE = 0, BMODE_SPARSE = 1, BMODE_VARLEN = 2 };
+
 
 enum : unsigned { WB_KV = 16, WB_QEMPTY, WB_QFULL, WB_S, WB_DP, WB_P, WB_DS, WB_DQFULL,
                   WB_DQEMPTY, WB_FINAL, WB_DRAIN };
@@ -234,7 +364,7 @@ __device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_
 
 // Block-sparse (SPARSE): a key block visits only the query blocks whose mask
 // entry for it is set, in the same cyclic order for every role.
-template <int D, bool CAUSAL, bool SPARSE>
+template <int D, bool CAUSAL, int MODE>
 __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
@@ -244,6 +374,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
                        const __grid_constant__ CUtensorMap tmdV, const BwdParams p) {
   using C = BwdCfg<D>;
   constexpr int BR = C::BR, BC = C::BC, DH = C::DH, QS = C::QS;
+  constexpr bool SPARSE = MODE == BMODE_SPARSE, VARLEN = MODE == BMODE_VARLEN;
   static_assert(BC == MASK_BLOCK, "a CTA's key block is one block-mask column");
 
   extern __shared__ uint8_t smem_raw[];
@@ -284,8 +415,18 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
   const int b = bkv / p.Hkv;
   const int hkv = bkv - b * p.Hkv;
   const int key0 = kb * BC;
+  // Sequence geometry: lengths, first packed rows and TMA "bh" coordinates
+  // (variable-length batches address packed tensors with one batch entry).
+  int nq = p.Nq, nk = p.Nk, qoff = 0, koff = 0;
+  if constexpr (VARLEN) {
+    varlen_rows(p.cu_q, b, p.total_q, qoff, nq);
+    varlen_rows(p.cu_k, b, p.total_k, koff, nk);
+    if (key0 >= nk) return;                             // past this sequence's keys
+  }
+  const int tkv = VARLEN ? hkv : bkv;
+  const int n_qblocks = VARLEN ? (nq + BR - 1) / BR : p.n_qblocks;
   const int i0 = CAUSAL ? (key0 / BR) : 0;              // first query block that sees key0
-  const int span = max(0, p.n_qblocks - i0);
+  const int span = max(0, n_qblocks - i0);
   int n_i = span;                                       // query blocks visited per head
   const int dcol0 = split * DH;                         // first d column owned here
   const int head0 = hkv * p.group + gs * p.hps;         // first query head (within batch b)
@@ -307,7 +448,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
   };
   auto qnext = [&](int i) -> int {        // next visited block at or after i, cyclically
     for (int k = 0; k < span; ++k, ++i) {
-      if (i >= p.n_qblocks) i = i0;
+      if (i >= n_qblocks) i = i0;
       if (qvis(i)) return i;
     }
     return i0;                            // not reached while n_i > 0
@@ -343,7 +484,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
   if constexpr (SPARSE) {
     if (warp == 10) {                     // count the visited query blocks once
       int c = 0;
-      for (int i = i0 + lane; i < p.n_qblocks; i += 32) c += qvis(i) ? 1 : 0;
+      for (int i = i0 + lane; i < n_qblocks; i += 32) c += qvis(i) ? 1 : 0;
       c = __reduce_add_sync(0xffffffffu, c);
       if (lane == 0) *sparse_ni = c;
     }
@@ -362,8 +503,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
       prefetch_tmap(&tmdO);
       mbar_arrive_expect_tx(bar_kv, 2 * C::K_BYTES);
       for (int c = 0; c < C::KCH; ++c) {
-        tma_load_bh(sK + c * BC * 128, &tmK, bar_kv, c * 64, key0, bkv, p.Hkv);
-        tma_load_bh(sV + c * BC * 128, &tmV, bar_kv, c * 64, key0, bkv, p.Hkv);
+        tma_load_bh(sK + c * BC * 128, &tmK, bar_kv, c * 64, koff + key0, tkv, p.Hkv);
+        tma_load_bh(sV + c * BC * 128, &tmV, bar_kv, c * 64, koff + key0, tkv, p.Hkv);
       }
       int issued = 0;
       Seq sq;
@@ -378,6 +519,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
           step_q(t, hh, qi);
         }
         const int bh = b * p.Hq + head0 + hh;
+        const int tq = VARLEN ? head0 + hh : bh;
         const int st = t % QS;
         if (!mbar_wait(bar_qempty + st, ((t / QS) & 1) ^ 1, abort_flag, p.status, WB_QEMPTY))
           break;
@@ -387,10 +529,13 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
         float* sd = sl + BR;
         mbar_arrive_expect_tx(bar_qfull + st, C::STAGE_BYTES);
         for (int c = 0; c < C::KCH; ++c) {
-          tma_load_bh(sq + c * BR * 128, &tmQ, bar_qfull + st, c * 64, qi * BR, bh, p.Hq);
-          tma_load_bh(sdo + c * BR * 128, &tmdO, bar_qfull + st, c * 64, qi * BR, bh, p.Hq);
+          tma_load_bh(sq + c * BR * 128, &tmQ, bar_qfull + st, c * 64, qoff + qi * BR, tq, p.Hq);
+          tma_load_bh(sdo + c * BR * 128, &tmdO, bar_qfull + st, c * 64, qoff + qi * BR, tq,
+                      p.Hq);
         }
-        const size_t ro = size_t(bh) * p.Nq_pad + size_t(qi) * BR;
+        const size_t ro = VARLEN ? size_t((head0 + hh) * p.lpad_ld + varlen_pad_start(qoff, b) +
+                                          qi * BR)
+                                 : size_t(bh) * p.Nq_pad + size_t(qi) * BR;
         bulk_load_1d(sl, p.Lpad + ro, BR * 4, bar_qfull + st);
         bulk_load_1d(sd, p.Dpad + ro, BR * 4, bar_qfull + st);
         ++issued;
@@ -519,12 +664,13 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
         mbar_arrive(bar_dqempty);
         const int q0 = qi * BR + g * 32;
         const int bh = b * p.Hq + head0 + hh;
-        float* dst = p.dqacc + (size_t(bh) * p.Nq + q0) * D + dcol0 + r;
-        if (q0 + 32 <= p.Nq) {
+        float* dst = p.dqacc + (VARLEN ? (size_t(head0 + hh) * p.total_q + qoff + q0) * D
+                                       : (size_t(bh) * p.Nq + q0) * D) + dcol0 + r;
+        if (q0 + 32 <= nq) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) atomicAdd(dst + i * D, __uint_as_float(v[i]));
         } else {
-          const int nvalid = p.Nq - q0;
+          const int nvalid = nq - q0;
 #pragma unroll
           for (int i = 0; i < 32; ++i)
             if (i < nvalid) atomicAdd(dst + i * D, __uint_as_float(v[i]));
@@ -554,8 +700,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
       const float* sd = sl + BR;
       const int qg = qi * BR + g * 32;              // first query of this group's columns
       // Columns c < cstart are masked: causal (query < key) or padding key.
-      const bool need_mask = (CAUSAL && key0 + BC - 1 > qg) || (key0 + BC > p.Nk);
-      const int cstart = key >= p.Nk ? 32 : (CAUSAL ? key - qg : 0);
+      const bool need_mask = (CAUSAL && key0 + BC - 1 > qg) || (key0 + BC > nk);
+      const int cstart = key >= nk ? 32 : (CAUSAL ? key - qg : 0);
       const uint32_t tS = tl + C::TM_S + (t & 1) * BR + g * 32;
       const uint32_t tDP = tl + C::TM_DP + g * 32;
 
@@ -665,8 +811,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
       if (n_steps > 0) {
         const int tcol = g == 0 ? C::TM_DK : C::TM_DV;
         const float mul = g == 0 ? p.scale : 1.f;
-        float* dst = (g == 0 ? p.dkacc : p.dvacc) + (size_t(bkv) * p.Nk + key) * D + dcol0;
-        const bool row_ok = key < p.Nk;
+        float* dst = (g == 0 ? p.dkacc : p.dvacc) +
+                     (VARLEN ? size_t(hkv) * p.total_k + koff + key : size_t(bkv) * p.Nk + key) *
+                         D + dcol0;
+        const bool row_ok = key < nk;
 #pragma unroll
         for (int c = 0; c < DH / 32; ++c) {
           uint32_t u[32];
@@ -687,6 +835,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
       const int tcol = g == 0 ? C::TM_DK : C::TM_DV;
       const float mul = g == 0 ? p.scale : 1.f;
       uint8_t* stage = sStage + g * (BC * DH * 2);
+      // Packed batches: a warp whose 32 key rows run past the sequence's
+      // end stores its rows directly (a TMA box would reach the next one).
+      const bool direct = VARLEN && (key0 + w * 32 + 32 > nk);
 #pragma unroll
       for (int c = 0; c < DH / 32; ++c) {
         uint32_t u[32];
@@ -701,6 +852,17 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i)
           pk[i] = pack_bf16(__uint_as_float(u[2 * i]) * mul, __uint_as_float(u[2 * i + 1]) * mul);
+        if (direct) {
+          if (key < nk) {
+            const Strides& so = g == 0 ? p.sdk : p.sdv;
+            uint4* dst = reinterpret_cast<uint4*>((g == 0 ? p.dk : p.dv) + hkv * so.h +
+                                                  (long long)(koff + key) * so.n + dcol0 + c * 32);
+#pragma unroll
+            for (int u4 = 0; u4 < 4; ++u4)
+              dst[u4] = make_uint4(pk[4 * u4], pk[4 * u4 + 1], pk[4 * u4 + 2], pk[4 * u4 + 3]);
+          }
+          continue;
+        }
         uint8_t* box = stage + ((c >> 1) * 4 + w) * 4096 + lane * 128;
 #pragma unroll
         for (int u4 = 0; u4 < 4; ++u4) {
@@ -711,10 +873,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0 && key0 + w * 32 < p.Nk) {
+      if (lane == 0 && !direct && key0 + w * 32 < nk) {
         const CUtensorMap* tm = g == 0 ? &tmdK : &tmdV;
         for (int c = 0; c < DH / 64; ++c)
-          tma_store_bh(tm, stage + (c * 4 + w) * 4096, dcol0 + c * 64, key0 + w * 32, bkv, p.Hkv);
+          tma_store_bh(tm, stage + (c * 4 + w) * 4096, dcol0 + c * 64, koff + key0 + w * 32, tkv,
+                       p.Hkv);
         bulk_commit();
         bulk_wait0();
       }
@@ -733,13 +896,24 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
 bool make_map_bf16(CUtensorMap* m, const void* base, int d, int rows, int heads, int batch,
                    const Strides& st, int box_rows);
 
+// A packed variable-length batch: B sequences with cumulative offsets
+// cu_q / cu_k (device int32 [B + 1]) into [total_q, Hq, d] / [total_k, Hkv, d]
+// tensors.  Nq / Nk passed alongside are the longest lengths.
+struct Varlen {
+  const int* cu_q;
+  const int* cu_k;
+  int total_q, total_k;
+};
+
 template <int D, bool CAUSAL>
 int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const void* o,
                  const float* lse, const void* dO, void* dq, void* dk, void* dv,
                  const Strides* st, int B, int Hq, int Hkv, int Nq, int Nk, float scale,
-                 const uint8_t* mask, void* workspace, DevStatus* status, cudaStream_t stream) {
+                 const uint8_t* mask, const Varlen* vl, void* workspace, DevStatus* status,
+                 cudaStream_t stream) {
   using C = BwdCfg<D>;
-  const BwdWorkspace w = bwd_workspace_layout(B, Hq, Hkv, Nq, Nk, D);
+  const BwdWorkspace w = vl ? bwd_workspace_layout_varlen(B, Hq, Hkv, vl->total_q, vl->total_k, D)
+                            : bwd_workspace_layout(B, Hq, Hkv, Nq, Nk, D);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* dqacc = reinterpret_cast<float*>(ws + w.dq_off);
   float* Dpad = reinterpret_cast<float*>(ws + w.d_off);
@@ -749,6 +923,10 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
   const int bhq = B * Hq;
   const int group = Hq / Hkv;
   const int n_kblocks = (Nk + C::BC - 1) / C::BC;
+  // Rows and batch entries the tensor maps and the convert kernels see:
+  // packed batches are one batch entry of total_q / total_k rows.
+  const int rows_q = vl ? vl->total_q : Nq, rows_k = vl ? vl->total_k : Nk;
+  const int map_b = vl ? 1 : B;
   // Split a kv group's query heads over several CTAs when the key blocks
   // alone would leave SMs idle: the smallest divisor of the group that
   // gives at least two CTAs per SM (same choice in every stage call).
@@ -765,26 +943,38 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
 
   CUtensorMap mq, mk, mv, mdo, mdk, mdv;
   // strides: q, k, v, o, dO, dq, dk, dv
-  if ((stages & 2) && (!make_map_bf16(&mq, q, D, Nq, Hq, B, st[0], C::BR) ||
-      !make_map_bf16(&mk, k, D, Nk, Hkv, B, st[1], C::BC) ||
-      !make_map_bf16(&mv, v, D, Nk, Hkv, B, st[2], C::BC) ||
-      !make_map_bf16(&mdo, dO, D, Nq, Hq, B, st[4], C::BR) ||
-      !make_map_bf16(&mdk, dk, D, Nk, Hkv, B, st[6], 32) ||
-      !make_map_bf16(&mdv, dv, D, Nk, Hkv, B, st[7], 32)))
+  if ((stages & 2) && (!make_map_bf16(&mq, q, D, rows_q, Hq, map_b, st[0], C::BR) ||
+      !make_map_bf16(&mk, k, D, rows_k, Hkv, map_b, st[1], C::BC) ||
+      !make_map_bf16(&mv, v, D, rows_k, Hkv, map_b, st[2], C::BC) ||
+      !make_map_bf16(&mdo, dO, D, rows_q, Hq, map_b, st[4], C::BR) ||
+      !make_map_bf16(&mdk, dk, D, rows_k, Hkv, map_b, st[6], 32) ||
+      !make_map_bf16(&mdv, dv, D, rows_k, Hkv, map_b, st[7], 32)))
     return 5;
+  const long long kv_n4 = gsplit > 1 ? (long long)(2 * w.kv_elems / 4) : 0LL;
 
   if (stages & 1) {
     constexpr int RPB = 256 / (D / 8);
-    const long long rows = (long long)bhq * Nq_pad;
-    const long long blocks = std::min<long long>((rows + RPB - 1) / RPB, 148LL * 16);
-    fa_bwd_pre_kernel<D><<<unsigned(blocks), 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, dqacc,
-        Dpad, Lpad, bhq, Hq, Nq, Nq_pad, st[3], st[4], kvacc,
-        gsplit > 1 ? (long long)(2 * w.kv_elems / 4) : 0LL);
+    if (vl) {
+      const long long rows = (long long)Hq * vl->total_q;
+      const long long blocks = std::max<long long>(
+          1, std::min<long long>((rows + RPB - 1) / RPB, 148LL * 16));
+      fa_bwd_pre_varlen_kernel<D><<<unsigned(blocks), 256, 0, stream>>>(
+          static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, dqacc,
+          Dpad, Lpad, vl->cu_q, B, Hq, vl->total_q, varlen_lpad_ld(B, vl->total_q), st[3], st[4],
+          kvacc, kv_n4);
+    } else {
+      const long long rows = (long long)bhq * Nq_pad;
+      const long long blocks = std::min<long long>((rows + RPB - 1) / RPB, 148LL * 16);
+      fa_bwd_pre_kernel<D><<<unsigned(blocks), 256, 0, stream>>>(
+          static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, dqacc,
+          Dpad, Lpad, bhq, Hq, Nq, Nq_pad, st[3], st[4], kvacc, kv_n4);
+    }
     if (cudaGetLastError() != cudaSuccess) return 5;
   }
   if (stages & 2) {
-    auto kern = mask ? fa_bwd_main_kernel<D, CAUSAL, true> : fa_bwd_main_kernel<D, CAUSAL, false>;
+    auto kern = vl     ? fa_bwd_main_kernel<D, CAUSAL, BMODE_VARLEN>
+                : mask ? fa_bwd_main_kernel<D, CAUSAL, BMODE_SPARSE>
+                       : fa_bwd_main_kernel<D, CAUSAL, BMODE_DENSE>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
         cudaSuccess)
       return 5;
@@ -810,22 +1000,32 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
     p.status = status;
     p.mask = mask;
     p.mask_ld = (Nk + MASK_BLOCK - 1) / MASK_BLOCK;
+    p.cu_q = vl ? vl->cu_q : nullptr;
+    p.cu_k = vl ? vl->cu_k : nullptr;
+    p.total_q = rows_q;
+    p.total_k = rows_k;
+    p.lpad_ld = vl ? varlen_lpad_ld(B, vl->total_q) : 0;
+    p.dk = static_cast<__nv_bfloat16*>(dk);
+    p.dv = static_cast<__nv_bfloat16*>(dv);
+    p.sdk = st[6];
+    p.sdv = st[7];
     const unsigned grid = unsigned(p.n_kblocks) * unsigned(B * Hkv) * C::NSPLIT * gsplit;
     kern<<<grid, C::NTHREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdk, mdv, p);
     if (cudaGetLastError() != cudaSuccess) return 5;
   }
   if (stages & 4) {
-    const long long n8 = (long long)bhq * Nq * D / 8;
-    const long long blocks = std::min<long long>((n8 + 255) / 256, 148LL * 16);
+    const long long n8 = (long long)Hq * map_b * rows_q * D / 8;
+    const long long blocks = std::max<long long>(1, std::min<long long>((n8 + 255) / 256,
+                                                                        148LL * 16));
     fa_bwd_dq_kernel<D><<<unsigned(blocks), 256, 0, stream>>>(
-        dqacc, static_cast<__nv_bfloat16*>(dq), n8, scale, Hq, Nq, st[5]);
+        dqacc, static_cast<__nv_bfloat16*>(dq), n8, scale, Hq, rows_q, st[5]);
     if (cudaGetLastError() != cudaSuccess) return 5;
     if (gsplit > 1) {
       const long long kv8 = (long long)w.kv_elems / 8;
       const long long kblocks = std::min<long long>((2 * kv8 + 255) / 256, 148LL * 16);
       fa_bwd_kv_kernel<D><<<unsigned(kblocks), 256, 0, stream>>>(
-          kvacc, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), kv8, Hkv, Nk,
-          st[6], st[7]);
+          kvacc, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), kv8, Hkv,
+          rows_k, st[6], st[7]);
       if (cudaGetLastError() != cudaSuccess) return 5;
     }
   }
@@ -833,18 +1033,21 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
 }
 
 // stages: bit 0 = preprocess, bit 1 = main, bit 2 = dq convert.  mask: the
-// block mask of block-sparse attention, or null.
+// block mask of block-sparse attention, or null; vl: a packed
+// variable-length batch, or null.
 inline int launch_bwd(int stages, const void* q, const void* k, const void* v, const void* o,
                       const float* lse, const void* dO, void* dq, void* dk, void* dv,
                       const Strides* st, int B, int Hq, int Hkv, int Nq, int Nk, int d,
-                      int causal, float scale, const uint8_t* mask, void* workspace,
-                      DevStatus* status, cudaStream_t stream) {
+                      int causal, float scale, const uint8_t* mask, const Varlen* vl,
+                      void* workspace, DevStatus* status, cudaStream_t stream) {
 #define FA_BWD_CASE(DD)                                                                          \
   if (d == DD)                                                                                   \
     return causal ? launch_bwd_t<DD, true>(stages, q, k, v, o, lse, dO, dq, dk, dv, st, B, Hq,  \
-                                           Hkv, Nq, Nk, scale, mask, workspace, status, stream) \
+                                           Hkv, Nq, Nk, scale, mask, vl, workspace, status,     \
+                                           stream)                                               \
                   : launch_bwd_t<DD, false>(stages, q, k, v, o, lse, dO, dq, dk, dv, st, B, Hq, \
-                                            Hkv, Nq, Nk, scale, mask, workspace, status, stream);
+                                            Hkv, Nq, Nk, scale, mask, vl, workspace, status,    \
+                                            stream);
   FA_BWD_CASE(64)
   FA_BWD_CASE(128)
   FA_BWD_CASE(256)

@@ -56,18 +56,70 @@ struct FwdParams {
   int mask_ld;        // ceil(Nk / 128)
   __nv_bfloat16* o;
   long long o_sb, o_sh, o_sn;
+  // Variable-length batches only: B sequences packed back to back, q / o as
+  // [total_q, Hq, d], k / v as [total_k, Hkv, d], lse as [Hq, total_q];
+  // sequence b is rows cu_q[b] .. cu_q[b+1] (cu_k for keys).  Nq and Nk are
+  // then the longest lengths, which size the grid.
+  const int* cu_q;
+  const int* cu_k;
+  int total_q, total_k;
 };
 
-// A query row that sees no key at all (every block of its mask row is
-// zero): O = 0 and LSE = -inf, the limits of an empty softmax.
-template <int D>
-__device__ __forceinline__ void write_empty_row(const FwdParams& p, int bh, int grow) {
-  if (grow >= p.Nq) return;
+// Kernel variants: fixed-length batch, block-sparse, variable-length batch.
+enum : int { MODE_DENSE = 0, MODE_SPARSE = 1, MODE_VARLEN = 2 };
+
+// Where one (batch, head)'s rows live.  Fixed-length batches: rows [0, Nq)
+// of the (b, h) slice of the 4-D tensor maps.  Variable-length batches: rows
+// [qoff, qoff + nq) of the packed tensors, whose maps have a single batch
+// entry; the offsets are clamped to the packed totals, so no access leaves
+// the tensors whatever the offsets hold.
+struct SeqGeo {
+  int nq, nk;          // sequence lengths
+  int qoff, koff;      // first packed row (0 for fixed-length batches)
+  int tq, tkv;         // TMA "bh" coordinates of q / o and of k / v
+  float* lse;          // LSE of the sequence's row 0 at this head
+  __nv_bfloat16* o;    // O of row 0 at this head (direct row stores)
+};
+
+template <bool VARLEN>
+__device__ __forceinline__ SeqGeo seq_geo(const FwdParams& p, int bh) {
   const int b = bh / p.Hq, h = bh - b * p.Hq;
-  uint4* dst = reinterpret_cast<uint4*>(p.o + b * p.o_sb + h * p.o_sh + (long long)grow * p.o_sn);
+  SeqGeo g;
+  if constexpr (VARLEN) {
+    const int q0 = min(max(__ldg(p.cu_q + b), 0), p.total_q);
+    const int q1 = min(max(__ldg(p.cu_q + b + 1), q0), p.total_q);
+    const int k0 = min(max(__ldg(p.cu_k + b), 0), p.total_k);
+    const int k1 = min(max(__ldg(p.cu_k + b + 1), k0), p.total_k);
+    g.nq = q1 - q0;
+    g.nk = k1 - k0;
+    g.qoff = q0;
+    g.koff = k0;
+    g.tq = h;
+    g.tkv = h / p.group;
+    g.lse = p.lse + size_t(h) * p.total_q + q0;
+    g.o = p.o + h * p.o_sh + (long long)q0 * p.o_sn;
+  } else {
+    g.nq = p.Nq;
+    g.nk = p.Nk;
+    g.qoff = g.koff = 0;
+    g.tq = bh;
+    g.tkv = b * p.Hkv + h / p.group;
+    g.lse = p.lse + size_t(bh) * p.Nq;
+    g.o = p.o + b * p.o_sb + h * p.o_sh;
+  }
+  return g;
+}
+
+// A query row that sees no key at all (every block of its mask row is
+// zero, or its sequence has no keys): O = 0 and LSE = -inf, the limits of
+// an empty softmax.
+template <int D>
+__device__ __forceinline__ void write_empty_row(const FwdParams& p, const SeqGeo& g, int grow) {
+  if (grow >= g.nq) return;
+  uint4* dst = reinterpret_cast<uint4*>(g.o + (long long)grow * p.o_sn);
 #pragma unroll
   for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
-  p.lse[size_t(bh) * p.Nq + grow] = -INFINITY;
+  g.lse[grow] = -INFINITY;
 }
 
 // Wait codes recorded on a timeout.
@@ -192,13 +244,17 @@ __device__ __forceinline__ bool softmax_block(RowState& st, uint32_t tS, uint32_
 
 // After the tile's last P V: O / lr to bf16, staged in `stage` (the tile's
 // free Q buffer) in the 128-byte swizzled layout, one 4 KiB box per warp and
-// 64 columns, TMA-stored by lane 0 of each warp; then the log-sum-exp.
-template <int D>
+// 64 columns, TMA-stored by lane 0 of each warp; then the log-sum-exp.  In
+// a packed variable-length batch a warp whose 32 rows run past its
+// sequence's end stores its rows directly instead (a TMA box would spill
+// into the next sequence).
+template <int D, bool VARLEN>
 __device__ __forceinline__ void softmax_finish(const RowState& st, uint32_t tO, uint8_t* stage,
                                                int w, int lane, const CUtensorMap* tmO,
-                                               int q_tile, int Nq, int bh, int H, float* lse,
-                                               int grow) {
+                                               int q_tile, const SeqGeo& g, long long o_sn,
+                                               int H, int grow) {
   const float inv = 1.0f / st.lr;
+  const bool direct = VARLEN && (q_tile + w * 32 + 32 > g.nq);   // warp-uniform
 #pragma unroll
   for (int c = 0; c < D / 32; ++c) {
     uint32_t r[32];
@@ -208,6 +264,15 @@ __device__ __forceinline__ void softmax_finish(const RowState& st, uint32_t tO, 
 #pragma unroll
     for (int i = 0; i < 16; ++i)
       pk2[i] = pack_bf16(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
+    if (direct) {
+      if (grow < g.nq) {
+        uint4* dst = reinterpret_cast<uint4*>(g.o + (long long)grow * o_sn + c * 32);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          dst[u] = make_uint4(pk2[4 * u], pk2[4 * u + 1], pk2[4 * u + 2], pk2[4 * u + 3]);
+      }
+      continue;
+    }
     uint8_t* box = stage + ((c >> 1) * 4 + w) * 4096 + lane * 128;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -218,13 +283,13 @@ __device__ __forceinline__ void softmax_finish(const RowState& st, uint32_t tO, 
   }
   fence_proxy_async_smem();
   __syncwarp();
-  if (lane == 0 && q_tile + w * 32 < Nq) {
+  if (lane == 0 && !direct && q_tile + w * 32 < g.nq) {
     for (int c = 0; c < D / 64; ++c)
-      tma_store_bh(tmO, stage + (c * 4 + w) * 4096, c * 64, q_tile + w * 32, bh, H);
+      tma_store_bh(tmO, stage + (c * 4 + w) * 4096, c * 64, g.qoff + q_tile + w * 32, g.tq, H);
     bulk_commit();
     bulk_wait0();
   }
-  if (grow < Nq) lse[size_t(bh) * Nq + grow] = (st.m + __log2f(st.l)) * 0.69314718055994531f;
+  if (grow < g.nq) g.lse[grow] = (st.m + __log2f(st.l)) * 0.69314718055994531f;
 }
 
 // ------------------------------------------------------------------ tile pairs (d = 64, 128)
@@ -262,7 +327,7 @@ enum : uint32_t { KV_T0 = 1, KV_T1 = 2, KV_LAST = 4, KV_EMPTY = 8, KV_ACT0 = 16,
 // Block-sparse (SPARSE): a unit's K/V stream is the union of the key blocks
 // its two tiles see; a tile takes part in the blocks its own mask row keeps,
 // and a tile that sees none is written out as empty rows.
-template <int D, bool CAUSAL, bool SPARSE>
+template <int D, bool CAUSAL, int MODE>
 __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
     fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
@@ -270,6 +335,7 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
                        const __grid_constant__ CUtensorMap tmO, const FwdParams p) {
   using C = FwdPairCfg<D>;
   constexpr int BR = C::BR, BC = C::BC, NS = C::NS;
+  constexpr bool SPARSE = MODE == MODE_SPARSE, VARLEN = MODE == MODE_VARLEN;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -305,7 +371,7 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
   // longest pair down, and the k-th round of units is dealt to the CTAs in
   // alternating direction (CTA c gets slot c, then grid-1-c, ...), which
   // evens out the total work per CTA.
-  auto unit = [&](int u, int& bh, int& q0, int* nt) {
+  auto unit = [&](int u, int& bh, int& q0, int* nt, SeqGeo& sg) {
     int pu;
     if (CAUSAL) {
       const int g = gridDim.x;
@@ -319,11 +385,12 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
       pu = u - bh * p.n_units;
     }
     q0 = pu * 2 * BR;
+    sg = seq_geo<VARLEN>(p, bh);
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
       const int qt = q0 + t * BR;
-      const int kv_end = CAUSAL ? min(p.Nk, qt + BR) : p.Nk;
-      nt[t] = (qt < p.Nq) ? (kv_end + BC - 1) / BC : 0;   // tile 1 may lie past Nq
+      const int kv_end = CAUSAL ? min(sg.nk, qt + BR) : sg.nk;
+      nt[t] = (qt < sg.nq) ? (kv_end + BC - 1) / BC : 0;   // tile 1 may lie past Nq
     }
   };
   if (threadIdx.x == 0) {
@@ -365,8 +432,8 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
       bool ok = !p.status->stall_kv;   // test control: withhold K/V (see fa_debug_inject)
       for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
         int bh, q0, nt[2];
-        unit(u, bh, q0, nt);
-        const int bkv = (bh / p.Hq) * p.Hkv + (bh % p.Hq) / p.group;
+        SeqGeo sg;
+        unit(u, bh, q0, nt, sg);
         // Ring order = MMA consumption order: K0, V0, K1, V1, ... over the
         // unit's (union of) key blocks.  The first ring items of a unit go
         // out before its Q loads, which wait for the previous unit's
@@ -413,7 +480,8 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
           uint8_t* dst = sKV + slot * C::KV_BYTES;
           const CUtensorMap* tm = (item & 1) ? &tmV : &tmK;
           for (int c = 0; c < C::KCH; ++c)
-            tma_load_bh(dst + c * BC * 128, tm, bar_kv_full + slot, c * 64, jc * BC, bkv, p.Hkv);
+            tma_load_bh(dst + c * BC * 128, tm, bar_kv_full + slot, c * 64, sg.koff + jc * BC,
+                        sg.tkv, p.Hkv);
           ++cnt;
           return true;
         };
@@ -427,7 +495,7 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
           mbar_arrive_expect_tx(bar_q + t, C::Q_BYTES);
           for (int c = 0; c < C::KCH; ++c)
             tma_load_bh(sQ + t * C::Q_BYTES + c * BR * 128, &tmQ, bar_q + t, c * 64,
-                        q0 + t * BR, bh, p.Hq);
+                        sg.qoff + q0 + t * BR, sg.tq, p.Hq);
           ++uses[t];
         }
         for (int it = early; it < items && ok; ++it) ok = ring(it);
@@ -495,10 +563,12 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
       };
       for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
         int bh, q0, nt[2];
-        unit(u, bh, q0, nt);
+        SeqGeo sg;
+        unit(u, bh, q0, nt, sg);
         int sK = 0, sV = 0;
         if constexpr (!SPARSE) {
           const int nmax = max(nt[0], nt[1]);
+          if (VARLEN && nmax == 0) continue;         // past its sequence, or no keys
           if (!(ok = acquire(sK))) break;
           for (int t = 0; t < 2 && ok; ++t) {
             if (nt[t] == 0) continue;
@@ -595,8 +665,14 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
     bool ok = true;
     for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
       int bh, q0, nt[2];
-      unit(u, bh, q0, nt);
-      if (nt[t] == 0) continue;                     // tile past Nq
+      SeqGeo sg;
+      unit(u, bh, q0, nt, sg);
+      if (nt[t] == 0) {
+        // tile past its sequence's end, or (packed batches) a sequence with
+        // queries but no keys
+        if (VARLEN && q0 + t * BR < sg.nq) write_empty_row<D>(p, sg, q0 + t * BR + row);
+        continue;
+      }
       int n = nt[t];
       bool last_kept = true;
       if constexpr (SPARSE) {
@@ -608,7 +684,7 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
       const int grow = q_tile + row;
       if constexpr (SPARSE) {
         if (n == 0) {                               // sees no key
-          write_empty_row<D>(p, bh, grow);
+          write_empty_row<D>(p, sg, grow);
           continue;
         }
       }
@@ -619,7 +695,7 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
           if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
           tc_fence_after();
           ok = softmax_block<BC, D, CAUSAL>(st, tl, tl + 128, j, j == 0, gb + j, q_tile, grow,
-                                            p.Nk, p.scale_log2, o_done, abort_flag, p.status);
+                                            sg.nk, p.scale_log2, o_done, abort_flag, p.status);
           if (!ok) break;
           mbar_arrive(bar_p_full + t);
         }
@@ -635,7 +711,7 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
           if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
           tc_fence_after();
           ok = softmax_block<BC, D, CAUSAL>(st, tl, tl + 128, j, l == 0, gb + l, q_tile, grow,
-                                            p.Nk, p.scale_log2, o_done, abort_flag, p.status);
+                                            sg.nk, p.scale_log2, o_done, abort_flag, p.status);
           if (!ok) break;
           mbar_arrive(bar_p_full + t);
         }
@@ -645,8 +721,8 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
       ok = mbar_wait(o_done + (jl & 1), (jl >> 1) & 1, abort_flag, p.status, W_O_DONE);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
-      softmax_finish<D>(st, tl + 128, sQ + t * C::Q_BYTES, w, lane, &tmO, q_tile, p.Nq, bh, p.Hq,
-                        p.lse, grow);
+      softmax_finish<D, VARLEN>(st, tl + 128, sQ + t * C::Q_BYTES, w, lane, &tmO, q_tile, sg,
+                                p.o_sn, p.Hq, grow);
       tc_fence_before();
       mbar_arrive(bar_o_free + t);                  // O has been read out of TMEM
       if (lane == 0) mbar_arrive(bar_q_free + t);   // this warp's staging boxes were stored
@@ -683,13 +759,14 @@ struct FwdCfg {
 // Block-sparse (SPARSE): the tile walks only the key blocks its mask row
 // keeps (two 64-key blocks per mask block); the MMA issuer sees just the
 // sequence, the producer and softmax map it back to key blocks.
-template <int D, bool CAUSAL, bool SPARSE>
+template <int D, bool CAUSAL, int MODE>
 __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                   const FwdParams p) {
   using C = FwdCfg<D>;
   constexpr int BR = C::BR, BC = C::BC, NS = C::NS;
+  constexpr bool SPARSE = MODE == MODE_SPARSE, VARLEN = MODE == MODE_VARLEN;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -713,11 +790,11 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
   const int bh = blockIdx.x / p.n_units;
   int qb = blockIdx.x - bh * p.n_units;
   if (CAUSAL) qb = p.n_units - 1 - qb;
-  const int b = bh / p.Hq;
-  const int h = bh - b * p.Hq;
-  const int bkv = b * p.Hkv + h / p.group;
+  const SeqGeo sg = seq_geo<VARLEN>(p, bh);
   const int q_row0 = qb * BR;
-  const int kv_end = CAUSAL ? min(p.Nk, q_row0 + BR) : p.Nk;
+  // A tile past its (packed) sequence's end has nothing to do.
+  if (VARLEN && q_row0 >= sg.nq) return;
+  const int kv_end = CAUSAL ? min(sg.nk, q_row0 + BR) : sg.nk;
   const int n_kv = (kv_end + BC - 1) / BC;             // key blocks in range
   constexpr int SUB = MASK_BLOCK / BC;                 // key blocks per mask block
   // Block-sparse: walks over the kept key blocks (one mask entry covers SUB
@@ -771,7 +848,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
       prefetch_tmap(&tmV);
       mbar_arrive_expect_tx(bar_q, C::Q_BYTES);
       for (int c = 0; c < C::KCH; ++c)
-        tma_load_bh(sQ + c * BR * 128, &tmQ, bar_q, c * 64, q_row0, bh, p.Hq);
+        tma_load_bh(sQ + c * BR * 128, &tmQ, bar_q, c * 64, sg.qoff + q_row0, sg.tq, p.Hq);
       int cnt = 0;
       bool ok = !p.status->stall_kv;   // test control: withhold K/V (see fa_debug_inject)
       auto load = [&](const CUtensorMap* tm, int j) {
@@ -784,7 +861,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
         mbar_arrive_expect_tx(bar_kv_full + slot, C::KV_BYTES);
         uint8_t* dst = sKV + slot * C::KV_BYTES;
         for (int c = 0; c < C::KCH; ++c)
-          tma_load_bh(dst + c * BC * 128, tm, bar_kv_full + slot, c * 64, j * BC, bkv, p.Hkv);
+          tma_load_bh(dst + c * BC * 128, tm, bar_kv_full + slot, c * 64, sg.koff + j * BC,
+                      sg.tkv, p.Hkv);
         ++cnt;
       };
       // Ring order = MMA consumption order: K0, K1, V0, K2, V1, ... over the
@@ -885,7 +963,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
     RowState st{-INFINITY, 0.f, 0.f};
     bool ok = true;
     if (n_blocks == 0) {                                 // sees no key (sparse)
-      write_empty_row<D>(p, bh, grow);
+      write_empty_row<D>(p, sg, grow);
       ok = false;
     }
     RowWalk rm;
@@ -895,7 +973,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
       ok = softmax_block<BC, D, CAUSAL>(st, tl + C::TM_S + (j & 1) * BC, tl + C::TM_O, jb, j == 0,
-                                        j, q_row0, grow, p.Nk, p.scale_log2, bar_o_done,
+                                        j, q_row0, grow, sg.nk, p.scale_log2, bar_o_done,
                                         abort_flag, p.status);
       if (!ok) break;
       mbar_arrive(bar_p_full + (j & 1));
@@ -905,8 +983,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
       ok = mbar_wait(bar_o_done + (jl & 1), (jl >> 1) & 1, abort_flag, p.status, W_O_DONE);
       if (__all_sync(0xffffffffu, ok)) {
         tc_fence_after();
-        softmax_finish<D>(st, tl + C::TM_O, sQ, warp, lane, &tmO, q_row0, p.Nq, bh, p.Hq, p.lse,
-                          grow);
+        softmax_finish<D, VARLEN>(st, tl + C::TM_O, sQ, warp, lane, &tmO, q_row0, sg, p.o_sn,
+                                  p.Hq, grow);
       }
     }
   }

@@ -119,3 +119,31 @@ def make_inputs(wl: Workload, device="cpu", with_do: bool = True):
     if not with_do:
         out.append(None)
     return tuple(out)
+
+
+def make_varlen_lengths(B: int, lo: int, hi: int, seed: int):
+    """Seeded sequence lengths, uniform integers in [lo, hi]."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    return torch.randint(lo, hi + 1, (B,), generator=g).tolist()
+
+
+def cu_seqlens(lengths):
+    """Cumulative offsets [0, l0, l0 + l1, ...] as int32 (CPU)."""
+    out = [0]
+    for n in lengths:
+        out.append(out[-1] + int(n))
+    return torch.tensor(out, dtype=torch.int32)
+
+
+def make_varlen_inputs(lengths_q, lengths_k, Hq: int, Hkv: int, d: int, seed: int):
+    """Packed bf16 q [total_q, Hq, d], k, v [total_k, Hkv, d], dO like q,
+    iid N(0, 1) drawn in that order from ``manual_seed(seed)``, plus the
+    int32 cumulative offsets of both sides (all on the CPU)."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    tq, tk = int(sum(lengths_q)), int(sum(lengths_k))
+    q = torch.randn(tq, Hq, d, generator=g)
+    k = torch.randn(tk, Hkv, d, generator=g)
+    v = torch.randn(tk, Hkv, d, generator=g)
+    do = torch.randn(tq, Hq, d, generator=g)
+    q, k, v, do = (t.to(torch.bfloat16) for t in (q, k, v, do))
+    return q, k, v, do, cu_seqlens(lengths_q), cu_seqlens(lengths_k)

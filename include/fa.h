@@ -147,6 +147,40 @@ int fa_bwd_block_sparse(const void* q, const void* k, const void* v, const void*
                         int Hkv, int Nq, int Nk, int d, int causal, float scale, void* workspace,
                         size_t workspace_bytes, cudaStream_t stream);
 
+/*
+ * Variable-length batches: B sequences of different lengths packed back to
+ * back, with no padding.  The pages do not name this; it serves the
+ * small-batch, long-sequence case that the FA2 article's section on
+ * parallelising over the sequence length addresses.
+ *   q, o, dO, dq  [total_q, Hq, d] bf16, contiguous (row n, head h at
+ *                 (n * Hq + h) * d)
+ *   k, v, dk, dv  [total_k, Hkv, d] bf16, contiguous
+ *   lse           [Hq, total_q] fp32
+ *   cu_seqlens_q, cu_seqlens_k  device int32 [B + 1]: sequence b is rows
+ *                 cu_seqlens_q[b] .. cu_seqlens_q[b+1] of q (and likewise of
+ *                 k, v); non-decreasing, starting at 0 and ending at total_q
+ *                 (total_k).  Read on the device only; out-of-range offsets
+ *                 are clamped to [0, total], never followed.
+ *   max_seqlen_q, max_seqlen_k  at least the longest sequence (they size the
+ *                 grid; rows beyond them are not computed).
+ * Attention stays within each sequence; causal masking is top-left aligned
+ * within the sequence.  A sequence with queries but no keys gets O = 0 and
+ * lse = -inf.  Other conventions as for fa_fwd / fa_bwd.
+ */
+int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                  const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int max_seqlen_q,
+                  int max_seqlen_k, int total_q, int total_k, int Hq, int Hkv, int d, int causal,
+                  float scale, cudaStream_t stream);
+
+/* Bytes of workspace fa_bwd_varlen needs (0 for invalid sizes). */
+size_t fa_bwd_varlen_workspace_size(int B, int total_q, int total_k, int Hq, int Hkv, int d);
+
+int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                  const void* dO, void* dq, void* dk, void* dv, const int* cu_seqlens_q,
+                  const int* cu_seqlens_k, int B, int max_seqlen_q, int max_seqlen_k,
+                  int total_q, int total_k, int Hq, int Hkv, int d, int causal, float scale,
+                  void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* Stages of fa_bwd, for callers that time or schedule them separately. */
 typedef enum {
   FA_BWD_ALL = 0,   /* the whole backward pass (same as fa_bwd) */

@@ -142,3 +142,24 @@ def test_block_sparse_rejects_bad_arguments():
                                   0.125, None, 0, None) == 4
     assert fa.fa_fwd_block_sparse(A, A, A, A, A, None, A, 0, 2, 2, 128, 128, 64, 0, 0.125,
                                   None) == 1
+
+
+def test_varlen_rejects_bad_arguments():
+    def fwd(**kw):
+        a = dict(q=A, k=A, v=A, o=A, lse=A, cu_q=A, cu_k=A, B=2, max_q=100, max_k=100,
+                 total_q=150, total_k=150, Hq=4, Hkv=2, d=64, causal=0, scale=0.125, stream=None)
+        a.update(kw)
+        return fa.fa_fwd_varlen(**a)
+    assert fwd(cu_q=None) == 1 and fwd(cu_k=None) == 1 and fwd(q=None) == 1
+    assert fwd(total_q=0) == 1 and fwd(B=0) == 1 and fwd(max_k=0) == 1
+    assert fwd(Hq=3) == 1 and fwd(scale=0.0) == 1 and fwd(d=80) == 2
+    assert fwd(cu_q=A + 2) == 3 and fwd(q=A + 8) == 3 and fwd(lse=A + 1) == 3
+    a = dict(q=A, k=A, v=A, o=A, lse=A, dO=A, dq=A, dk=A, dv=A, cu_q=A, cu_k=A, B=2, max_q=100,
+             max_k=100, total_q=150, total_k=150, Hq=4, Hkv=2, d=64, causal=0, scale=0.125,
+             workspace=A, workspace_bytes=1 << 40, stream=None)
+    assert fa.fa_bwd_varlen(**dict(a, workspace=None)) == 4
+    assert fa.fa_bwd_varlen(**dict(a, workspace_bytes=64)) == 4
+    assert fa.fa_bwd_varlen(**dict(a, dk=A + 8)) == 3
+    assert fa.fa_bwd_varlen(**dict(a, cu_k=None)) == 1
+    assert fa.fa_bwd_varlen_workspace_size(2, 150, 150, 4, 2, 64) > 150 * 4 * 64 * 4
+    assert fa.fa_bwd_varlen_workspace_size(2, 150, 150, 4, 3, 64) == 0
