@@ -19,6 +19,10 @@ key) block with probability P (diagonal blocks always), the step is
 fa_fwd_block_sparse + fa_bwd_block_sparse, and FLOPs count only the kept
 (query, key) pairs.
 
+``--varlen LO:HI`` measures a packed variable-length batch instead: the
+workload's B sequences get seeded lengths uniform in [LO, HI], the step is
+fa_fwd_varlen + fa_bwd_varlen, and FLOPs are summed per sequence.
+
 ``--impl reference`` times the fp64 CPU oracle instead (the only other place
 this script runs it), on a bounded sample of the same workload.
 Multi-GPU (torchrun): every rank runs an independent batch of the same shape
@@ -61,6 +65,9 @@ def parse_args(argv=None):
                     help="target CPU work for the oracle baseline sample")
     ap.add_argument("--block-density", type=float, default=None,
                     help="block-sparse attention with this fraction of 128x128 blocks kept")
+    ap.add_argument("--varlen", default=None, metavar="LO:HI",
+                    help="packed variable-length batch: the workload's B sequences get seeded "
+                         "lengths uniform in [LO, HI] (its H, d and causal flag)")
     return ap.parse_args(argv)
 
 
@@ -249,6 +256,203 @@ def time_oracle(wl, seconds: float, max_groups=None, mask=None):
               f"{'' if mask is None else ' with the same block mask'}; {t_total:.1f} s of CPU "
               f"work; rate scaled exactly by FLOPs")
     return tflops, cores, sample, t_total, done * per_group_flops
+
+
+# ----------------------------------------------------------------- packed batches
+def varlen_lengths(wl, spec, rank=0):
+    """Seeded sequence lengths of the --varlen measurement."""
+    from exact_io_aware_71_b200.inputs import make_varlen_lengths
+    lo, hi = (int(x) for x in spec.split(":"))
+    if not 1 <= lo <= hi:
+        raise ValueError("--varlen wants LO:HI with 1 <= LO <= HI")
+    return make_varlen_lengths(wl.B, lo, hi, seed=wl.seed + 1000 * rank)
+
+
+def varlen_fwd_flops(wl, lengths) -> float:
+    """Nominal forward FLOPs of a packed batch: 4*Hq*n^2*d per sequence,
+    halved when causal."""
+    f = sum(4.0 * wl.Hq * n * n * wl.d for n in lengths)
+    return f / 2 if wl.causal else f
+
+
+def time_oracle_varlen(wl, lengths, seconds: float, max_seqs=None):
+    """fp64 oracle forward + backward on whole sequences of the packed batch,
+    as many as fit in about `seconds` (shortest first, so a bounded sample
+    covers several); returns (TFLOP/s, cores, sample, seconds, FLOPs)."""
+    from threadpoolctl import threadpool_limits
+
+    import numpy as np
+
+    import oracle
+    from exact_io_aware_71_b200.inputs import make_varlen_inputs
+
+    cores = len(os.sched_getaffinity(0))
+    q, k, v, do, cq, ck = make_varlen_inputs(lengths, lengths, wl.Hq, wl.Hkv, wl.d, wl.seed)
+    order = sorted(range(len(lengths)), key=lambda b: lengths[b])
+    done, t_total, flops = 0, 0.0, 0.0
+    with threadpool_limits(limits=cores):
+        for b in order:
+            if max_seqs is not None and done >= max_seqs:
+                break
+            sl = slice(int(cq[b]), int(cq[b + 1]))
+            cu = np.array([0, lengths[b]])
+            args = [t[sl].double().numpy() for t in (q, k, v, do)]
+            t0 = time.perf_counter()
+            oracle.attention_backward_varlen(*args, cu, cu, wl.causal, wl.scale)
+            t_total += time.perf_counter() - t0
+            flops += 3.5 * varlen_fwd_flops(wl, [lengths[b]])
+            done += 1
+            if max_seqs is None and t_total >= seconds and done >= 2:
+                break
+    sample = (f"fp64 NumPy oracle fwd+bwd on {done} of {len(lengths)} sequences (shortest "
+              f"first) of the packed batch; {t_total:.1f} s of CPU work; rate scaled by FLOPs")
+    return flops / t_total / 1e12, cores, sample, t_total, flops
+
+
+def run_ours_varlen(args, rank, world, local_rank):
+    """The --varlen step: fa_fwd_varlen + fa_bwd_varlen on packed inputs."""
+    import torch
+
+    from exact_io_aware_71_b200 import binding as fa
+    from exact_io_aware_71_b200.inputs import make_varlen_inputs, workloads
+
+    wl = workloads()[args.workload]
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    fa.load()
+    lengths = varlen_lengths(wl, args.varlen, rank if world > 1 else 0)
+    q, k, v, do, cq, ck = (t.to(dev) for t in make_varlen_inputs(
+        lengths, lengths, wl.Hq, wl.Hkv, wl.d, wl.seed + (1000 * rank if world > 1 else 0)))
+    B, tq, mx = len(lengths), q.shape[0], max(lengths)
+    o = torch.empty_like(q)
+    lse = torch.empty(wl.Hq, tq, dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    wsb = fa.fa_bwd_varlen_workspace_size(B, tq, tq, wl.Hq, wl.Hkv, wl.d)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    geo = (cq.data_ptr(), ck.data_ptr(), B, mx, mx, tq, tq, wl.Hq, wl.Hkv, wl.d, int(wl.causal),
+           wl.scale)
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        st = fa.fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                              lse.data_ptr(), *geo, sh)
+        if st:
+            raise fa.FaError(st, "fa_fwd_varlen")
+        if evs:
+            evs[1].record(stream)
+        st = fa.fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                              lse.data_ptr(), do.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                              dv.data_ptr(), *geo, ws.data_ptr(), wsb, sh)
+        if st:
+            raise fa.FaError(st, "fa_bwd_varlen")
+        if evs:
+            evs[2].record(stream)
+
+    dist = torch.distributed if world > 1 else None
+
+    def reduce_max(x):
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    st, where = fa.fa_device_status(sh)
+    if st:
+        raise RuntimeError(f"device status {st} at wait {where} during warm-up")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    e0.record(stream)
+    for s_ in range(args.steps):
+        step(evs[s_])
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop()
+    per_ms = [sum(evs[s_][i].elapsed_time(evs[s_][i + 1]) for s_ in range(args.steps))
+              / args.steps for i in range(2)]
+    st, where = fa.fa_device_status(sh)
+    if st:
+        raise RuntimeError(f"device status {st} at wait {where} in the timed region")
+    fwd_flops = varlen_fwd_flops(wl, lengths)
+    bwd_flops = 2.5 * fwd_flops
+    t_ms, fps = aggregate(e0.elapsed_time(e1), args.steps * (fwd_flops + bwd_flops), world,
+                          reduce_max)
+    peaks, peak_src = load_peaks()
+    names = ["fa_fwd_pair_kernel (packed)", "fa_bwd (pre, main, dq; packed)"]
+    dom = 0 if per_ms[0] >= per_ms[1] else 1
+    achieved = (fwd_flops, bwd_flops)[dom] / (per_ms[dom] / 1e3) / 1e12
+    roof = {"bound": "tensor", "kernel": names[dom], "achieved": round(achieved, 2),
+            "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": round(achieved / peaks["bf16_tflops"], 4),
+            "peak_source": f"{peak_src} bf16 cuBLAS burst (MEASURED_PEAKS.json)"
+            if peak_src == "measured" else "fallback 1.59 PFLOP/s", "traffic": None}
+
+    # end to end: pinned host inputs in, outputs back, through the torch-level binding
+    hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, do))
+    outs_h = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (o, lse, dq, dk, dv)]
+    dev_in = [torch.empty_like(t) for t in (q, k, v, do)]
+
+    def e2e_step():
+        for dst, src in zip(dev_in, (hq, hk, hv, hdo)):
+            dst.copy_(src, non_blocking=True)
+        o_, l_ = fa.forward_varlen(dev_in[0], dev_in[1], dev_in[2], cq, ck, mx, mx, wl.causal,
+                                   wl.scale, out=o, lse=lse)
+        g = fa.backward_varlen(dev_in[0], dev_in[1], dev_in[2], o_, l_, dev_in[3], cq, ck, mx,
+                               mx, wl.causal, wl.scale, workspace=ws)
+        for dst, src in zip(outs_h, (o_, l_) + g):
+            dst.copy_(src, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    a1.record(stream)
+    torch.cuda.synchronize(dev)
+    e_ms, e_fps = aggregate(a0.elapsed_time(a1), args.e2e_steps * 3.5 * fwd_flops, world,
+                            reduce_max)
+    e2e = {"value": round(e_fps / 1e12, 2), "unit": "TFLOP/s",
+           "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo)),
+           "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in outs_h),
+           "steps": args.e2e_steps, "ms_per_step": round(e_ms / args.e2e_steps, 3)}
+    fwd_tf = fwd_flops / (per_ms[0] / 1e3) / 1e12
+    bwd_tf = bwd_flops / (per_ms[1] / 1e3) / 1e12
+    return {
+        "metric": METRIC, "value": round(fps / 1e12, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(3, args.warmup),
+        "ms_per_step": round(t_ms / args.steps, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded iid N(0,1), bf16)",
+        "config": {"workload": f"{wl.name}_varlen{args.varlen}", "B": B, "Hq": wl.Hq,
+                   "Hkv": wl.Hkv, "d": wl.d, "causal": wl.causal, "total_tokens": tq,
+                   "max_seqlen": mx, "lengths_seed": wl.seed,
+                   "step": "fa_fwd_varlen + fa_bwd_varlen (packed [total, H, d])",
+                   "parallelism": f"{world} independent replica(s), no collective",
+                   "l2": "inputs larger than L2, no flush" if 4 * q.numel() * 2 > 126e6
+                   else "inputs smaller than L2: re-read from L2 between steps",
+                   "flops": "sum over sequences of 4*Hq*n^2*d (x1/2 causal), x3.5 per step"},
+        "fwd_tflops": round(fwd_tf, 2), "bwd_tflops": round(bwd_tf, 2),
+        "fwd_frac_of_peak": round(fwd_tf / peaks["bf16_tflops"], 4),
+        "bwd_frac_of_peak": round(bwd_tf / peaks["bf16_tflops"], 4),
+        "per_kernel_ms": {n: round(t, 4) for n, t in zip(names, per_ms)},
+        "roofline": roof, "e2e": e2e, "clocks": clk,
+        "gpu_launches": launches_per_step(wl, torch.cuda.get_device_properties(dev)
+                                          .multi_processor_count) * args.steps,
+    }
 
 
 # ----------------------------------------------------------------- our arm
@@ -464,12 +668,18 @@ def run_reference(args):
     from exact_io_aware_71_b200.inputs import workloads
     wl = workloads()[args.workload]
     mask = block_mask_for(wl, args.block_density)
+    lengths = varlen_lengths(wl, args.varlen) if args.varlen else None
+
+    def sample_step():
+        if lengths is not None:
+            return time_oracle_varlen(wl, lengths, 0.0, max_seqs=1)
+        return time_oracle(wl, 0.0, max_groups=1, mask=mask)
     for _ in range(args.warmup):
-        time_oracle(wl, 0.0, max_groups=1, mask=mask)
+        sample_step()
     t_all, f_all = 0.0, 0.0
     cores = len(os.sched_getaffinity(0))
     for _ in range(args.steps):
-        _, cores, sample, t, f = time_oracle(wl, 0.0, max_groups=1, mask=mask)
+        _, cores, sample, t, f = sample_step()
         t_all += t
         f_all += f
     value = f_all / t_all / 1e12
@@ -480,7 +690,8 @@ def run_reference(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded iid N(0,1), bf16 inputs upcast to fp64)",
         "config": {"workload": wl.name + ("" if mask is None
-                                          else f"_blocksparse{args.block_density:g}"),
+                                          else f"_blocksparse{args.block_density:g}")
+                   + (f"_varlen{args.varlen}" if lengths is not None else ""),
                    "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "Nq": wl.Nq,
                    "Nk": wl.Nk, "d": wl.d, "causal": wl.causal,
                    "step": "oracle fwd+bwd on one (batch, kv-head) group of the workload"},
@@ -511,12 +722,16 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        out = run_ours(args, rank, world, local_rank)
+        out = (run_ours_varlen if args.varlen else run_ours)(args, rank, world, local_rank)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             from exact_io_aware_71_b200.inputs import workloads
             wl = workloads()[args.workload]
-            tf, cores, sample, _, _ = time_oracle(wl, args.cpu_seconds,
-                                                  mask=block_mask_for(wl, args.block_density))
+            if args.varlen:
+                tf, cores, sample, _, _ = time_oracle_varlen(wl, varlen_lengths(wl, args.varlen),
+                                                             args.cpu_seconds)
+            else:
+                tf, cores, sample, _, _ = time_oracle(wl, args.cpu_seconds,
+                                                      mask=block_mask_for(wl, args.block_density))
             out["cpu_baseline"] = {"value": round(tf, 6), "unit": "TFLOP/s", "cores": cores,
                                    "kind": "oracle", "sample": sample}
         if rank == 0:

@@ -112,3 +112,22 @@ def test_launches_per_step():
     assert bench.launches_per_step(w["long_gqa_hkv1_n16384_d128_causal"], 148) == 5
     # 8 kv heads x 128 key blocks = 1024 CTAs: no split
     assert bench.launches_per_step(w["long_gqa_hkv8_n16384_d128_causal"], 148) == 4
+
+
+def test_varlen_lengths_and_flops():
+    from exact_io_aware_71_b200.inputs import workloads
+    wl = workloads()["train_b8h16n2048d128_causal"]
+    L = bench.varlen_lengths(wl, "100:300")
+    assert len(L) == wl.B and all(100 <= n <= 300 for n in L)
+    assert L == bench.varlen_lengths(wl, "100:300")          # seeded
+    assert bench.varlen_fwd_flops(wl, [wl.Nq] * wl.B) == pytest.approx(wl.fwd_flops())
+    with pytest.raises(ValueError):
+        bench.varlen_lengths(wl, "0:10")
+
+
+def test_reference_arm_varlen_runs_on_cpu():
+    out = bench.run_reference(bench.parse_args(["--impl", "reference", "--workload",
+                                                "tiny_b1h2n128d64_full", "--varlen", "20:60",
+                                                "--steps", "1", "--warmup", "1"]))
+    assert out["impl"] == "reference" and out["value"] > 0
+    assert out["config"]["workload"].endswith("_varlen20:60")
