@@ -23,15 +23,16 @@
 //                   then dK_j * scale and dV_j are written as bf16
 //   fa_bwd_dq       dq = bf16(scale * dQacc)              (HBM-bound)
 //
-// fa_bwd_main roles (384 threads): warpgroups 0 and 1 are compute warps
+// fa_bwd_main roles (512 threads): warpgroups 0 and 1 are compute warps
 // (TMEM lane = key row); warpgroup w owns query columns [32w, 32w+32) of
 // every step, and writes its P^T (hi, lo) and dS^T only over its own S^T /
 // dP^T columns, so neither group can overwrite scores the other has not yet
-// read.  Warp 8 issues the TMA loads, warp 9 the MMAs (10, 11 idle).
+// read.  Warp 8 issues the TMA loads, warp 9 the MMAs (10, 11 idle), and
+// warpgroup 3 reads dQ^T out of TMEM and reduce-adds it into the fp32
+// accumulator, so those global reductions overlap the compute warps' work.
 // TMEM (512 columns): S^T x2 | dP^T | dQ^T | dK | dV.  S^T is double-buffered
 // so S^T of step t+1 is computed while step t's dS is formed; per step the
-// MMA order is dV_t, S_{t+1}, dK_t, dQ_t, dP_{t+1}, and the compute warps
-// read out dQ_{t-1} between P_t and dS_t.  For d = 256 the dK / dV
+// MMA order is dV_t, S_{t+1}, dK_t, dQ_t, dP_{t+1}.  For d = 256 the dK / dV
 // accumulators alone would fill TMEM, so two CTAs share a key block, each
 // owning one 128-wide half of d for dK, dV and dQ (both recompute S and dP).
 #pragma once
@@ -53,15 +54,29 @@ struct BwdCfg {
   static constexpr int STAGE_BYTES = 2 * QT_BYTES + 2 * BR * 4;
   static constexpr int STAGE_STRIDE = (STAGE_BYTES + 1023) / 1024 * 1024;
   static constexpr int DS_BYTES = BC * BR * 2;          // dS^T: [BC keys][BR queries] bf16
-  static constexpr int TM_S = 0;                        // two S^T buffers of BR columns
+  // d <= 128: K is copied into TMEM once per CTA and is the A operand of
+  // S^T = K Q^T (no shared-memory reads for it); S^T then has one buffer,
+  // which costs nothing because S^T_{t+1} is issued after dV_t has read P_t.
+  // d = 256: K stays in shared memory and S^T is double-buffered.
+  static constexpr bool KTM = D <= 128;
+  static constexpr int TM_S = 0;                        // S^T buffers of BR columns
+  static constexpr int TM_K = BR;                       // K as bf16 pairs (D / 2 columns)
   static constexpr int TM_DP = 2 * BR;
   static constexpr int TM_DQ = 3 * BR;
   static constexpr int TM_DK = 4 * BR;
   static constexpr int TM_DV = 4 * BR + DH;
   static constexpr int TMEM_COLS = 512;
-  static constexpr int NTHREADS = 384;
+  static constexpr int NTHREADS = 512;
+  // setmaxnreg split of the 512 threads' registers: compute warpgroups 0-1,
+  // producer / MMA warpgroup 2, dQ read-out warpgroup 3.
+  static constexpr int REGS_COMPUTE = 168;
+  static constexpr int REGS_OTHER = 88;
+  static constexpr int REGS_READ = 80;
+  static constexpr int REGS_NEEDED = 256 * REGS_COMPUTE + 128 * REGS_OTHER + 128 * REGS_READ;
+  static_assert(REGS_NEEDED <= 65536, "register split");
   static constexpr int SMEM_BYTES = 2 * K_BYTES + QS * STAGE_STRIDE + DS_BYTES + 1024 + 1024;
   static_assert(TM_DV + DH <= TMEM_COLS, "TMEM budget");
+  static_assert(!KTM || TM_K + D / 2 <= TM_DP, "K fits in the second S^T buffer's columns");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
   static_assert(QS * STAGE_STRIDE >= 2 * BC * DH * 2, "dK/dV staging fits in the Q/dO stages");
 };
@@ -92,11 +107,11 @@ inline size_t bwd_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d)
 }
 
 // Packed variable-length batch of B sequences: dQacc fp32 [Hq, total_q, d] |
-// Dpad, Lpad fp32 [Hq, ld] with ld = round_up(total_q, 4) + 128 (B + 1),
+// Dpad, Lpad fp32 [Hq, ld] with ld = round_up(total_q, 4) + 256 (B + 1),
 // each sequence's rows starting at varlen_pad_start | (GQA/MQA only)
 // dKacc, dVacc fp32 [Hkv, total_k, d].
 inline long long varlen_lpad_ld(int B, int total_q) {
-  return (long long)((total_q + 3) & ~3) + 128LL * (B + 1);
+  return (long long)((total_q + 3) & ~3) + 256LL * (B + 1);
 }
 inline BwdWorkspace bwd_workspace_layout_varlen(int B, int Hq, int Hkv, int total_q, int total_k,
                                                 int d) {
@@ -122,15 +137,15 @@ struct Strides {
 
 // Packed-batch helpers: sequence b's rows clamped to [0, total], and where
 // its padded fp32 row vectors (D, LSE) start in a head's workspace row:
-// 16-byte aligned, with room for ceil(n / 64) * 64 entries before the next
-// sequence (each sequence adds 128 entries of slack).
+// 16-byte aligned, with room for ceil(n / 128) * 128 entries before the next
+// sequence (each sequence adds 256 entries of slack).
 __device__ __forceinline__ void varlen_rows(const int* cu, int b, int total, int& off, int& n) {
   const int a = min(max(__ldg(cu + b), 0), total);
   n = min(max(__ldg(cu + b + 1), a), total) - a;
   off = a;
 }
 __device__ __forceinline__ long long varlen_pad_start(int off, int b) {
-  return (long long)((off + 3) & ~3) + 128LL * b;
+  return (long long)((off + 3) & ~3) + 256LL * b;
 }
 
 template <int D>
@@ -189,7 +204,7 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(
 // [Hq, total_q, d].  Row n of the packed tensors belongs to the sequence b
 // with cu_q[b] <= n < cu_q[b+1] (found by bisection); its D and LSE*log2(e)
 // go to h * ld + varlen_pad_start(cu_q[b], b) + (n - cu_q[b]).  Afterwards
-// the entries from each sequence's length up to the next multiple of 64
+// the entries from each sequence's length up to the next multiple of 128
 // are padding: D = 0, LSE = +inf, so the main kernel's P is 0 there.
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_pre_varlen_kernel(
@@ -247,15 +262,15 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_varlen_kernel(
     }
   }
   // padding entries of every (head, sequence)
-  const long long npad = (long long)Hq * B * 64;
+  const long long npad = (long long)Hq * B * 128;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < npad;
        i += (long long)gridDim.x * blockDim.x) {
-    const int e = int(i % 64);
-    const int bb = int((i / 64) % B);
-    const int h = int(i / (64LL * B));
+    const int e = int(i % 128);
+    const int bb = int((i / 128) % B);
+    const int h = int(i / (128LL * B));
     const int off = start(bb);
     const int len = min(max(__ldg(cu_q + bb + 1), off), total_q) - off;
-    if (len + e < ((len + 63) & ~63)) {
+    if (len + e < ((len + 127) & ~127)) {
       const long long pi = h * ld + varlen_pad_start(off, bb) + len + e;
       Dpad[pi] = 0.f;
       Lpad[pi] = INFINITY;
@@ -395,7 +410,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
   uint64_t* bar_dqfull = bars + 6 + 2 * QS;
   uint64_t* bar_dqempty = bars + 7 + 2 * QS;
   uint64_t* bar_final = bars + 8 + 2 * QS;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 9 + 2 * QS);
+  uint64_t* bar_ktm = bars + 9 + 2 * QS;                // K copied into TMEM (d <= 128)
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 10 + 2 * QS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   int* sparse_ni = reinterpret_cast<int*>(tmem_holder + 2);
 
@@ -472,8 +488,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
     mbar_init(bar_p, 256);
     mbar_init(bar_ds, 256);
     mbar_init(bar_dqfull, 1);
-    mbar_init(bar_dqempty, 256);
+    mbar_init(bar_dqempty, 128);
     mbar_init(bar_final, 1);
+    mbar_init(bar_ktm, 128);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -496,6 +513,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
   if constexpr (SPARSE) n_i = *sparse_ni;
   const int n_steps = p.hps * n_i;
 
+  if (warp >= 8 && warp < 12) {
+    regs_dec<C::REGS_OTHER>();
   if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && n_steps > 0) {
@@ -559,7 +578,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
       // group kk/2 wrote queries [32(kk/2), +32) packed into its own columns.
       auto pcol = [](int kk) { return uint32_t((kk >> 1) * 32 + (kk & 1) * 8); };
       auto mma_sdp = [&](uint32_t d_tm, uint32_t a_base, uint32_t b_base) {
-#pragma unroll
+#pragma unroll (D == 256 ? 4 : D / 16)
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ko = (kk >> 2) * BC * 128 + (kk & 3) * 32;
           const uint32_t qo = (kk >> 2) * BR * 128 + (kk & 3) * 32;
@@ -568,11 +587,26 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
         }
       };
       auto stage_q = [&](int t) { return aS0 + (t % QS) * C::STAGE_STRIDE; };
+      // S^T of step t: A = K from TMEM (d <= 128) or shared memory.
+      auto mma_s = [&](int t) {
+        const uint32_t d_tm = tmem + C::TM_S + (C::KTM ? 0 : (t & 1) * BR);
+        if constexpr (C::KTM) {
+          const uint32_t bq = stage_q(t);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            umma_ts(d_tm, tmem + C::TM_K + kk * 8,
+                    sdesc_sw128(bq + (kk >> 2) * BR * 128 + (kk & 3) * 32, 16, 1024), ID_S,
+                    kk > 0);
+        } else {
+          mma_sdp(d_tm, aK, stage_q(t));
+        }
+      };
       bool ok = mbar_wait(bar_kv, 0, abort_flag, p.status, WB_KV) &&
-                mbar_wait(bar_qfull + 0, 0, abort_flag, p.status, WB_QFULL);
+                mbar_wait(bar_qfull + 0, 0, abort_flag, p.status, WB_QFULL) &&
+                (!C::KTM || mbar_wait(bar_ktm, 0, abort_flag, p.status, WB_KV));
       tc_fence_after();
       if (ok) {
-        mma_sdp(tmem + C::TM_S, aK, stage_q(0));
+        mma_s(0);
         umma_commit(bar_s + 0);
         mma_sdp(tmem + C::TM_DP, aV, stage_q(0) + C::QT_BYTES);
         umma_commit(bar_dp);
@@ -581,7 +615,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
         const int st = t % QS;
         const uint32_t aQ = stage_q(t);
         const uint32_t adO = aQ + C::QT_BYTES;
-        const uint32_t tS = tmem + C::TM_S + (t & 1) * BR;
+        const uint32_t tS = tmem + C::TM_S + (C::KTM ? 0 : (t & 1) * BR);
         // dV += P^T dO  (hi then lo half of P)
         if (!(ok = mbar_wait(bar_p, t & 1, abort_flag, p.status, WB_P))) break;
         tc_fence_after();
@@ -602,7 +636,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
                          WB_QFULL))
             return false;
           tc_fence_after();
-          mma_sdp(tmem + C::TM_S + ((t + 1) & 1) * BR, aK, stage_q(t + 1));
+          mma_s(t + 1);
           umma_commit(bar_s + ((t + 1) & 1));
           return true;
         };
@@ -640,7 +674,59 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
       volatile int no_abort = 0;
       mbar_wait(bar_final, 0, &no_abort, nullptr, WB_DRAIN);
     }
-  } else if (warp < 8) {
+  }
+    // warps 10 and 11 have no role
+  } else if (warp >= 12) {
+    regs_dec<C::REGS_READ>();
+    // ------------------------------------------------------------ dQ read-out
+    // Warp 12 + w reads TMEM lane quarter w of dQ^T (lanes = d rows, all 64
+    // query columns of the step) and reduce-adds it into the fp32
+    // accumulator, coalesced over d, while the compute warps form the next
+    // step's P and dS.
+    const int w = warp - 12;
+    const int r = w * 32 + lane;                   // d row
+    const uint32_t tl = tmem + (uint32_t(w * 32) << 16);
+    Seq sq;
+    if constexpr (SPARSE) seq_begin(sq);
+    for (int u = 0; u < n_steps; ++u) {
+      int hh, qi;
+      if constexpr (SPARSE) {
+        hh = sq.hh;
+        qi = sq.qi;
+        seq_next(sq);
+      } else {
+        step_q(u, hh, qi);
+      }
+      const bool okk = mbar_wait(bar_dqfull, u & 1, abort_flag, p.status, WB_DQFULL);
+      if (!__all_sync(0xffffffffu, okk)) break;
+      tc_fence_after();
+      if (r < DH) {
+        uint32_t v[64];
+        FA_TMEM_LD32(tl + C::TM_DQ, v);
+        FA_TMEM_LD32(tl + C::TM_DQ + 32, (v + 32));
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar_dqempty);
+        const int q0 = qi * BR;
+        const int bh = b * p.Hq + head0 + hh;
+        float* dst = p.dqacc + (VARLEN ? (size_t(head0 + hh) * p.total_q + qoff + q0) * D
+                                       : (size_t(bh) * p.Nq + q0) * D) + dcol0 + r;
+        if (q0 + BR <= nq) {
+#pragma unroll
+          for (int i = 0; i < BR; ++i) atomicAdd(dst + i * D, __uint_as_float(v[i]));
+        } else {
+          const int nvalid = nq - q0;
+#pragma unroll
+          for (int i = 0; i < BR; ++i)
+            if (i < nvalid) atomicAdd(dst + i * D, __uint_as_float(v[i]));
+        }
+      } else {
+        tc_fence_before();
+        mbar_arrive(bar_dqempty);
+      }
+    }
+  } else {
+    regs_inc<C::REGS_COMPUTE>();
     // ------------------------------------------------------------ compute warps
     const int g = warp >> 2;                       // compute group: query columns [32g, 32g+32)
     const int w = warp & 3;                        // TMEM lane quarter
@@ -650,42 +736,35 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
     const float sl2 = p.scale_log2;
     bool ok = true;
 
-    // Read out dQ^T of step u (lanes = d, columns = this group's 32 queries)
-    // and reduce-add it into the fp32 accumulator (coalesced over d).
-    auto dq_readout = [&](int u, int hh, int qi) -> bool {
-      bool okk = mbar_wait(bar_dqfull, u & 1, abort_flag, p.status, WB_DQFULL);
-      if (!__all_sync(0xffffffffu, okk)) return false;
-      tc_fence_after();
-      if (r < DH) {
-        uint32_t v[32];
-        FA_TMEM_LD32(tl + C::TM_DQ + g * 32, v);
-        tmem_wait_ld();
+    // d <= 128: group 0 copies its key row of K (swizzled shared tile) into
+    // TMEM as bf16 pairs, the A operand layout of S^T = K Q^T.
+    if (C::KTM && g == 0 && n_steps > 0) {
+      ok = mbar_wait(bar_kv, 0, abort_flag, p.status, WB_KV);
+      if (__all_sync(0xffffffffu, ok)) {
+        uint32_t kr[D / 2];
+#pragma unroll
+        for (int c = 0; c < C::KCH; ++c)
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const uint4 x = *reinterpret_cast<const uint4*>(sK + c * BC * 128 + r * 128 +
+                                                            ((u ^ (r & 7)) << 4));
+            kr[32 * c + 4 * u + 0] = x.x;
+            kr[32 * c + 4 * u + 1] = x.y;
+            kr[32 * c + 4 * u + 2] = x.z;
+            kr[32 * c + 4 * u + 3] = x.w;
+          }
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) FA_TMEM_ST32(tl + C::TM_K + c * 32, (kr + c * 32));
+        tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar_dqempty);
-        const int q0 = qi * BR + g * 32;
-        const int bh = b * p.Hq + head0 + hh;
-        float* dst = p.dqacc + (VARLEN ? (size_t(head0 + hh) * p.total_q + qoff + q0) * D
-                                       : (size_t(bh) * p.Nq + q0) * D) + dcol0 + r;
-        if (q0 + 32 <= nq) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) atomicAdd(dst + i * D, __uint_as_float(v[i]));
-        } else {
-          const int nvalid = nq - q0;
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (i < nvalid) atomicAdd(dst + i * D, __uint_as_float(v[i]));
-        }
+        mbar_arrive(bar_ktm);
       } else {
-        tc_fence_before();
-        mbar_arrive(bar_dqempty);
+        ok = false;
       }
-      return true;
-    };
-
-    int prev_hh = 0, prev_qi = 0;                   // query block of step t - 1
+    }
     Seq sq;
     if constexpr (SPARSE) seq_begin(sq);
-    for (int t = 0; t < n_steps; ++t) {
+    for (int t = 0; t < n_steps && ok; ++t) {
       int hh, qi;
       if constexpr (SPARSE) {
         hh = sq.hh;
@@ -702,7 +781,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
       // Columns c < cstart are masked: causal (query < key) or padding key.
       const bool need_mask = (CAUSAL && key0 + BC - 1 > qg) || (key0 + BC > nk);
       const int cstart = key >= nk ? 32 : (CAUSAL ? key - qg : 0);
-      const uint32_t tS = tl + C::TM_S + (t & 1) * BR + g * 32;
+      const uint32_t tS = tl + C::TM_S + (C::KTM ? 0 : (t & 1) * BR) + g * 32;
       const uint32_t tDP = tl + C::TM_DP + g * 32;
 
       ok = mbar_wait(bar_qfull + st, (t / QS) & 1, abort_flag, p.status, WB_QFULL) &&
@@ -754,9 +833,6 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
       tc_fence_before();
       mbar_arrive(bar_p);
 
-      // ---- dQ of the previous step (its MMA ran while P was formed)
-      if (t > 0 && !(ok = dq_readout(t - 1, prev_hh, prev_qi))) break;
-
       // ---- dS^T = P^T o (dP^T - D)
       ok = mbar_wait(bar_dp, t & 1, abort_flag, p.status, WB_DP);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
@@ -792,10 +868,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar_ds);
-      prev_hh = hh;
-      prev_qi = qi;
     }
-    if (ok && n_steps > 0) ok = dq_readout(n_steps - 1, prev_hh, prev_qi);
 
     // ---- epilogue: group 0 writes dK = scale * dK_acc, group 1 writes dV,
     // bf16 through the (now free) Q/dO stages, one 4 KiB box per warp and
@@ -892,6 +965,12 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
   }
 }
 
+}  // namespace fa
+
+#include "fa_bwd128.cuh"
+
+namespace fa {
+
 // ------------------------------------------------------------------ launch
 bool make_map_bf16(CUtensorMap* m, const void* base, int d, int rows, int heads, int batch,
                    const Strides& st, int box_rows);
@@ -943,10 +1022,14 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
 
   CUtensorMap mq, mk, mv, mdo, mdk, mdv;
   // strides: q, k, v, o, dO, dq, dk, dv
-  if ((stages & 2) && (!make_map_bf16(&mq, q, D, rows_q, Hq, map_b, st[0], C::BR) ||
+  // d <= 128 runs the 128-query-step kernel (fa_bwd128.cuh); d = 256 the
+  // general one with 64-query steps.
+  constexpr bool STEP128 = D <= 128;
+  constexpr int BRK = STEP128 ? 128 : C::BR;
+  if ((stages & 2) && (!make_map_bf16(&mq, q, D, rows_q, Hq, map_b, st[0], BRK) ||
       !make_map_bf16(&mk, k, D, rows_k, Hkv, map_b, st[1], C::BC) ||
       !make_map_bf16(&mv, v, D, rows_k, Hkv, map_b, st[2], C::BC) ||
-      !make_map_bf16(&mdo, dO, D, rows_q, Hq, map_b, st[4], C::BR) ||
+      !make_map_bf16(&mdo, dO, D, rows_q, Hq, map_b, st[4], BRK) ||
       !make_map_bf16(&mdk, dk, D, rows_k, Hkv, map_b, st[6], 32) ||
       !make_map_bf16(&mdv, dv, D, rows_k, Hkv, map_b, st[7], 32)))
     return 5;
@@ -972,12 +1055,21 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
     if (cudaGetLastError() != cudaSuccess) return 5;
   }
   if (stages & 2) {
-    auto kern = vl     ? fa_bwd_main_kernel<D, CAUSAL, BMODE_VARLEN>
-                : mask ? fa_bwd_main_kernel<D, CAUSAL, BMODE_SPARSE>
-                       : fa_bwd_main_kernel<D, CAUSAL, BMODE_DENSE>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+    using C2 = typename std::conditional<STEP128, Bwd128Cfg<(D <= 128 ? D : 128)>, C>::type;
+    auto kern = STEP128 ? (vl     ? fa_bwd_main128_kernel<(D <= 128 ? D : 128), CAUSAL, BMODE_VARLEN>
+                           : mask ? fa_bwd_main128_kernel<(D <= 128 ? D : 128), CAUSAL, BMODE_SPARSE>
+                                  : fa_bwd_main128_kernel<(D <= 128 ? D : 128), CAUSAL, BMODE_DENSE>)
+                        : (vl     ? fa_bwd_main_kernel<D, CAUSAL, BMODE_VARLEN>
+                           : mask ? fa_bwd_main_kernel<D, CAUSAL, BMODE_SPARSE>
+                                  : fa_bwd_main_kernel<D, CAUSAL, BMODE_DENSE>);
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C2::SMEM_BYTES) !=
         cudaSuccess)
       return 5;
+    // The warpgroups' setmaxnreg split must fit in the registers the block
+    // is launched with, or a setmaxnreg.inc would wait forever: refuse.
+    cudaFuncAttributes fattr;
+    if (cudaFuncGetAttributes(&fattr, kern) != cudaSuccess) return 5;
+    if (fattr.numRegs * C2::NTHREADS < C2::REGS_NEEDED) return 2;
     BwdParams p;
     p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Nq = Nq; p.Nk = Nk; p.Nq_pad = Nq_pad;
     p.group = group;
@@ -991,7 +1083,7 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
     p.hps = group / gsplit;
     p.dkacc = kvacc;
     p.dvacc = kvacc + w.kv_elems;
-    p.n_qblocks = (Nq + C::BR - 1) / C::BR;
+    p.n_qblocks = (Nq + BRK - 1) / BRK;
     p.scale = scale;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.Dpad = Dpad;
@@ -1010,7 +1102,7 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
     p.sdk = st[6];
     p.sdv = st[7];
     const unsigned grid = unsigned(p.n_kblocks) * unsigned(B * Hkv) * C::NSPLIT * gsplit;
-    kern<<<grid, C::NTHREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdk, mdv, p);
+    kern<<<grid, C2::NTHREADS, C2::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdk, mdv, p);
     if (cudaGetLastError() != cudaSuccess) return 5;
   }
   if (stages & 4) {

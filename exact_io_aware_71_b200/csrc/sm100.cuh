@@ -190,6 +190,14 @@ template <int N>
 __device__ __forceinline__ void regs_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
+// Move a warpgroup from the launch count L to N registers per thread
+// (setmaxnreg.inc may only raise the count and .dec only lower it).
+template <int N, int L>
+__device__ __forceinline__ void regs_to() {
+  static_assert(N % 8 == 0 && N >= 24 && N <= 256, "setmaxnreg range");
+  if constexpr (N > L) regs_inc<N>();
+  else if constexpr (N < L) regs_dec<N>();
+}
 
 // ---------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
@@ -278,6 +286,22 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
         "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),       \
         "=r"(r[31])                                                                         \
       : "r"(taddr))
+
+#define FA_TMEM_LD16(taddr, r)                                                              \
+  asm volatile(                                                                             \
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "                                             \
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"                    \
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), \
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),          \
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])                                               \
+      : "r"(taddr))
+
+#define FA_TMEM_ST8(taddr, r)                                                             \
+  asm volatile(                                                                           \
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), \
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),        \
+      "r"(r[7])                                                                           \
+      : "memory")
 
 #define FA_TMEM_ST16(taddr, r)                                                            \
   asm volatile(                                                                           \
