@@ -54,13 +54,7 @@ struct BwdCfg {
   static constexpr int STAGE_BYTES = 2 * QT_BYTES + 2 * BR * 4;
   static constexpr int STAGE_STRIDE = (STAGE_BYTES + 1023) / 1024 * 1024;
   static constexpr int DS_BYTES = BC * BR * 2;          // dS^T: [BC keys][BR queries] bf16
-  // d <= 128: K is copied into TMEM once per CTA and is the A operand of
-  // S^T = K Q^T (no shared-memory reads for it); S^T then has one buffer,
-  // which costs nothing because S^T_{t+1} is issued after dV_t has read P_t.
-  // d = 256: K stays in shared memory and S^T is double-buffered.
-  static constexpr bool KTM = D <= 128;
-  static constexpr int TM_S = 0;                        // S^T buffers of BR columns
-  static constexpr int TM_K = BR;                       // K as bf16 pairs (D / 2 columns)
+  static constexpr int TM_S = 0;                        // two S^T buffers of BR columns
   static constexpr int TM_DP = 2 * BR;
   static constexpr int TM_DQ = 3 * BR;
   static constexpr int TM_DK = 4 * BR;
@@ -76,7 +70,6 @@ struct BwdCfg {
   static_assert(REGS_NEEDED <= 65536, "register split");
   static constexpr int SMEM_BYTES = 2 * K_BYTES + QS * STAGE_STRIDE + DS_BYTES + 1024 + 1024;
   static_assert(TM_DV + DH <= TMEM_COLS, "TMEM budget");
-  static_assert(!KTM || TM_K + D / 2 <= TM_DP, "K fits in the second S^T buffer's columns");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
   static_assert(QS * STAGE_STRIDE >= 2 * BC * DH * 2, "dK/dV staging fits in the Q/dO stages");
 };
@@ -410,8 +403,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
   uint64_t* bar_dqfull = bars + 6 + 2 * QS;
   uint64_t* bar_dqempty = bars + 7 + 2 * QS;
   uint64_t* bar_final = bars + 8 + 2 * QS;
-  uint64_t* bar_ktm = bars + 9 + 2 * QS;                // K copied into TMEM (d <= 128)
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 10 + 2 * QS);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 9 + 2 * QS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   int* sparse_ni = reinterpret_cast<int*>(tmem_holder + 2);
 
@@ -490,7 +482,6 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
     mbar_init(bar_dqfull, 1);
     mbar_init(bar_dqempty, 128);
     mbar_init(bar_final, 1);
-    mbar_init(bar_ktm, 128);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -587,23 +578,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
         }
       };
       auto stage_q = [&](int t) { return aS0 + (t % QS) * C::STAGE_STRIDE; };
-      // S^T of step t: A = K from TMEM (d <= 128) or shared memory.
-      auto mma_s = [&](int t) {
-        const uint32_t d_tm = tmem + C::TM_S + (C::KTM ? 0 : (t & 1) * BR);
-        if constexpr (C::KTM) {
-          const uint32_t bq = stage_q(t);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            umma_ts(d_tm, tmem + C::TM_K + kk * 8,
-                    sdesc_sw128(bq + (kk >> 2) * BR * 128 + (kk & 3) * 32, 16, 1024), ID_S,
-                    kk > 0);
-        } else {
-          mma_sdp(d_tm, aK, stage_q(t));
-        }
-      };
+      // S^T of step t into buffer t mod 2
+      auto mma_s = [&](int t) { mma_sdp(tmem + C::TM_S + (t & 1) * BR, aK, stage_q(t)); };
       bool ok = mbar_wait(bar_kv, 0, abort_flag, p.status, WB_KV) &&
-                mbar_wait(bar_qfull + 0, 0, abort_flag, p.status, WB_QFULL) &&
-                (!C::KTM || mbar_wait(bar_ktm, 0, abort_flag, p.status, WB_KV));
+                mbar_wait(bar_qfull + 0, 0, abort_flag, p.status, WB_QFULL);
       tc_fence_after();
       if (ok) {
         mma_s(0);
@@ -615,7 +593,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
         const int st = t % QS;
         const uint32_t aQ = stage_q(t);
         const uint32_t adO = aQ + C::QT_BYTES;
-        const uint32_t tS = tmem + C::TM_S + (C::KTM ? 0 : (t & 1) * BR);
+        const uint32_t tS = tmem + C::TM_S + (t & 1) * BR;
         // dV += P^T dO  (hi then lo half of P)
         if (!(ok = mbar_wait(bar_p, t & 1, abort_flag, p.status, WB_P))) break;
         tc_fence_after();
@@ -736,32 +714,6 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
     const float sl2 = p.scale_log2;
     bool ok = true;
 
-    // d <= 128: group 0 copies its key row of K (swizzled shared tile) into
-    // TMEM as bf16 pairs, the A operand layout of S^T = K Q^T.
-    if (C::KTM && g == 0 && n_steps > 0) {
-      ok = mbar_wait(bar_kv, 0, abort_flag, p.status, WB_KV);
-      if (__all_sync(0xffffffffu, ok)) {
-        uint32_t kr[D / 2];
-#pragma unroll
-        for (int c = 0; c < C::KCH; ++c)
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const uint4 x = *reinterpret_cast<const uint4*>(sK + c * BC * 128 + r * 128 +
-                                                            ((u ^ (r & 7)) << 4));
-            kr[32 * c + 4 * u + 0] = x.x;
-            kr[32 * c + 4 * u + 1] = x.y;
-            kr[32 * c + 4 * u + 2] = x.z;
-            kr[32 * c + 4 * u + 3] = x.w;
-          }
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c) FA_TMEM_ST32(tl + C::TM_K + c * 32, (kr + c * 32));
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bar_ktm);
-      } else {
-        ok = false;
-      }
-    }
     Seq sq;
     if constexpr (SPARSE) seq_begin(sq);
     for (int t = 0; t < n_steps && ok; ++t) {
@@ -781,7 +733,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
       // Columns c < cstart are masked: causal (query < key) or padding key.
       const bool need_mask = (CAUSAL && key0 + BC - 1 > qg) || (key0 + BC > nk);
       const int cstart = key >= nk ? 32 : (CAUSAL ? key - qg : 0);
-      const uint32_t tS = tl + C::TM_S + (C::KTM ? 0 : (t & 1) * BR) + g * 32;
+      const uint32_t tS = tl + C::TM_S + (t & 1) * BR + g * 32;
       const uint32_t tDP = tl + C::TM_DP + g * 32;
 
       ok = mbar_wait(bar_qfull + st, (t / QS) & 1, abort_flag, p.status, WB_QFULL) &&
@@ -1056,12 +1008,17 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
   }
   if (stages & 2) {
     using C2 = typename std::conditional<STEP128, Bwd128Cfg<(D <= 128 ? D : 128)>, C>::type;
-    auto kern = STEP128 ? (vl     ? fa_bwd_main128_kernel<(D <= 128 ? D : 128), CAUSAL, BMODE_VARLEN>
-                           : mask ? fa_bwd_main128_kernel<(D <= 128 ? D : 128), CAUSAL, BMODE_SPARSE>
-                                  : fa_bwd_main128_kernel<(D <= 128 ? D : 128), CAUSAL, BMODE_DENSE>)
-                        : (vl     ? fa_bwd_main_kernel<D, CAUSAL, BMODE_VARLEN>
-                           : mask ? fa_bwd_main_kernel<D, CAUSAL, BMODE_SPARSE>
-                                  : fa_bwd_main_kernel<D, CAUSAL, BMODE_DENSE>);
+    auto pick = [&]() {
+      if constexpr (STEP128)
+        return vl ? fa_bwd_main128_kernel<D, CAUSAL, BMODE_VARLEN>
+               : mask ? fa_bwd_main128_kernel<D, CAUSAL, BMODE_SPARSE>
+                      : fa_bwd_main128_kernel<D, CAUSAL, BMODE_DENSE>;
+      else
+        return vl ? fa_bwd_main_kernel<D, CAUSAL, BMODE_VARLEN>
+               : mask ? fa_bwd_main_kernel<D, CAUSAL, BMODE_SPARSE>
+                      : fa_bwd_main_kernel<D, CAUSAL, BMODE_DENSE>;
+    };
+    auto kern = pick();
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C2::SMEM_BYTES) !=
         cudaSuccess)
       return 5;
