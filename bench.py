@@ -48,7 +48,8 @@ if ROOT not in sys.path:
 DEFAULT_WORKLOAD = "train_b8h16n2048d128_full"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = ["exact_io_aware_71_b200/csrc/sm100.cuh", "exact_io_aware_71_b200/csrc/fa_fwd.cuh",
-                  "exact_io_aware_71_b200/csrc/fa_bwd.cuh", "exact_io_aware_71_b200/csrc/fa_mask.cuh"]
+                  "exact_io_aware_71_b200/csrc/fa_bwd.cuh", "exact_io_aware_71_b200/csrc/fa_mask.cuh",
+                  "exact_io_aware_71_b200/csrc/fa_bwd128.cuh"]
 METRIC = "attention fwd / fwd+bwd TFLOP/s (bf16, 1×B200) and % of dense BF16 peak"
 
 
