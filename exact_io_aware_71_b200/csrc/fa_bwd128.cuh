@@ -21,10 +21,10 @@
 // frees DP for dP_{t+1}.  Waiting for dP_t also proves that dQ_{t-1}, which
 // reads the shared dS^T tile, has finished before dS_t overwrites it.
 //
-// P is formed as bf16 hi + lo (lo = P - hi): both go to TMEM for dV (hi,
-// plus lo when the precision rule asks for it: GQA/MQA groups) and stay in
-// the thread's registers for dS, because S^T_{t+1} overwrites the P^T
-// columns while dS_t is being formed.  The LSE
+// P goes to TMEM as bf16 hi (plus lo = P - hi when the precision rule asks
+// for it: GQA/MQA groups) for dV, and stays in the thread's registers in
+// fp32 for dS, because S^T_{t+1} overwrites the P^T columns while dS_t is
+// being formed.  The LSE
 // and D rows are read straight from the workspace (L1-resident broadcast
 // loads) rather than staged, which keeps shared memory within 227 KB.
 #pragma once
@@ -379,7 +379,8 @@ __global__ void __launch_bounds__(Bwd128Cfg<D>::NTHREADS, 1)
       ok = mbar_wait(bar_s, t & 1, abort_flag, p.status, WB_S);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
-      uint32_t hi[32], lo[32];                      // P as bf16 pairs, kept for dS
+      float pf[64];                                 // P (fp32), kept for dS
+      const bool split = p.split_p != 0;
       const float2 sl22 = make_float2(sl2, sl2);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
@@ -403,20 +404,23 @@ __global__ void __launch_bounds__(Bwd128Cfg<D>::NTHREADS, 1)
             for (int e = 0; e < 4; ++e) pv[e] = (i + e < cstart) ? 0.f : pv[e];
           }
 #pragma unroll
-          for (int e = 0; e < 4; ++e) u[i + e] = __float_as_uint(pv[e]);
+          for (int e = 0; e < 4; ++e) pf[c * 32 + i + e] = pv[e];
         }
+        uint32_t hi[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float a = __uint_as_float(u[2 * i]), bb = __uint_as_float(u[2 * i + 1]);
-          const uint32_t h = pack_bf16(a, bb);
-          const float2 rem = fadd2(make_float2(a, bb),
-                                   make_float2(-__uint_as_float(h << 16),
-                                               -__uint_as_float(h & 0xFFFF0000u)));
-          hi[c * 16 + i] = h;
-          lo[c * 16 + i] = pack_bf16(rem.x, rem.y);
+        for (int i = 0; i < 16; ++i) hi[i] = pack_bf16(pf[c * 32 + 2 * i], pf[c * 32 + 2 * i + 1]);
+        FA_TMEM_ST16(tSP + c * 32, hi);
+        if (split) {                                 // lo = P - hi, for dV of GQA/MQA groups
+          uint32_t lo[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float2 rem = fadd2(make_float2(pf[c * 32 + 2 * i], pf[c * 32 + 2 * i + 1]),
+                                     make_float2(-__uint_as_float(hi[i] << 16),
+                                                 -__uint_as_float(hi[i] & 0xFFFF0000u)));
+            lo[i] = pack_bf16(rem.x, rem.y);
+          }
+          FA_TMEM_ST16(tSP + c * 32 + 16, lo);
         }
-        FA_TMEM_ST16(tSP + c * 32, (hi + c * 16));
-        FA_TMEM_ST16(tSP + c * 32 + 16, (lo + c * 16));
       }
       tmem_wait_st();
       tc_fence_before();
@@ -438,11 +442,7 @@ __global__ void __launch_bounds__(Bwd128Cfg<D>::NTHREADS, 1)
           const float dsub[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const uint32_t h = hi[c * 8 + i + e], l = lo[c * 8 + i + e];
-            const float2 pp = fadd2(make_float2(__uint_as_float(h << 16),
-                                                __uint_as_float(h & 0xFFFF0000u)),
-                                    make_float2(__uint_as_float(l << 16),
-                                                __uint_as_float(l & 0xFFFF0000u)));
+            const float2 pp = make_float2(pf[c * 16 + 2 * (i + e)], pf[c * 16 + 2 * (i + e) + 1]);
             const float2 x = fadd2(make_float2(__uint_as_float(dpv[2 * (i + e)]),
                                                __uint_as_float(dpv[2 * (i + e) + 1])),
                                    make_float2(-dsub[2 * e], -dsub[2 * e + 1]));
