@@ -304,14 +304,16 @@ def forward_varlen(q, k, v, cu_q, cu_k, max_q, max_k, causal: bool, scale: float
 
 
 def backward_varlen(q, k, v, o, lse, do, cu_q, cu_k, max_q, max_k, causal: bool, scale: float,
-                    workspace=None):
-    """dQ, dK, dV (packed, bf16) of a variable-length batch."""
+                    workspace=None, grads=None):
+    """dQ, dK, dV (packed, bf16) of a variable-length batch; `grads` may
+    give contiguous output tensors shaped like q, k, v."""
     import torch
     B, tq, tk, Hq, Hkv, d = _varlen_dims(q, k, cu_q, cu_k)
     need = fa_bwd_varlen_workspace_size(B, tq, tk, Hq, Hkv, d)
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dq, dk, dv = grads if grads is not None else (torch.empty_like(q), torch.empty_like(k),
+                                                  torch.empty_like(v))
     st = fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                        do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
                        cu_q.data_ptr(), cu_k.data_ptr(), B, int(max_q), int(max_k), tq, tk, Hq,
