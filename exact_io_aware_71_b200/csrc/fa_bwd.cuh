@@ -563,48 +563,54 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
       constexpr uint32_t ID_S = idesc_bf16_f32(128, BR, 0, 0);    // S^T, dP^T: K-major both
       constexpr uint32_t ID_KV = idesc_bf16_f32(128, DH, 0, 1);   // dV, dK: B MN-major
       constexpr uint32_t ID_DQ = idesc_bf16_f32(128, BR, 1, 1);   // dQ^T: A, B MN-major
-      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aS0 = smem_u32(sStage);
-      const uint32_t adS = smem_u32(sdS);
+      // Descriptor low words: K-major (S^T, dP^T operands) and MN-major (the
+      // B operands of dV, dK and both operands of dQ^T).
+      const uint32_t kK = sdesc_sw128_lo(smem_u32(sK), 16);
+      const uint32_t mK = sdesc_sw128_lo(smem_u32(sK), BC * 128);
+      const uint32_t kV = sdesc_sw128_lo(smem_u32(sV), 16);
+      const uint32_t kS0 = sdesc_sw128_lo(smem_u32(sStage), 16);
+      const uint32_t mS0 = sdesc_sw128_lo(smem_u32(sStage), BR * 128);
+      const uint32_t mdS = sdesc_sw128_lo(smem_u32(sdS), BC * 128);
+      constexpr uint32_t STG = C::STAGE_STRIDE >> 4, QT = C::QT_BYTES >> 4;
       // A-operand column (within a P^T / dS^T buffer) of k-step kk: compute
       // group kk/2 wrote queries [32(kk/2), +32) packed into its own columns.
       auto pcol = [](int kk) { return uint32_t((kk >> 1) * 32 + (kk & 1) * 8); };
-      auto mma_sdp = [&](uint32_t d_tm, uint32_t a_base, uint32_t b_base) {
+      auto mma_sdp = [&](uint32_t d_tm, uint32_t a_lo, uint32_t b_lo) {
 #pragma unroll (D == 256 ? 4 : D / 16)
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ko = (kk >> 2) * BC * 128 + (kk & 3) * 32;
-          const uint32_t qo = (kk >> 2) * BR * 128 + (kk & 3) * 32;
-          umma_ss(d_tm, sdesc_sw128(a_base + ko, 16, 1024), sdesc_sw128(b_base + qo, 16, 1024),
-                  ID_S, kk > 0);
+          const uint32_t ko = ((kk >> 2) * BC * 128 + (kk & 3) * 32) >> 4;
+          const uint32_t qo = ((kk >> 2) * BR * 128 + (kk & 3) * 32) >> 4;
+          umma_ss_lo(d_tm, a_lo + ko, b_lo + qo, ID_S, kk > 0);
         }
       };
-      auto stage_q = [&](int t) { return aS0 + (t % QS) * C::STAGE_STRIDE; };
+      auto kst = [&](int t) { return kS0 + uint32_t(t % QS) * STG; };   // Q of step t, K-major
+      auto mst = [&](int t) { return mS0 + uint32_t(t % QS) * STG; };   // Q of step t, MN-major
       // S^T of step t into buffer t mod 2
-      auto mma_s = [&](int t) { mma_sdp(tmem + C::TM_S + (t & 1) * BR, aK, stage_q(t)); };
+      auto mma_s = [&](int t) { mma_sdp(tmem + C::TM_S + (t & 1) * BR, kK, kst(t)); };
+      // this CTA's 64-column share of d in the MN-major operands
+      const uint32_t dq_off = uint32_t((dcol0 / 64) * BR * 128) >> 4;
+      const uint32_t dk_off = uint32_t((dcol0 / 64) * BC * 128) >> 4;
       bool ok = mbar_wait(bar_kv, 0, abort_flag, p.status, WB_KV) &&
                 mbar_wait(bar_qfull + 0, 0, abort_flag, p.status, WB_QFULL);
       tc_fence_after();
       if (ok) {
         mma_s(0);
         umma_commit(bar_s + 0);
-        mma_sdp(tmem + C::TM_DP, aV, stage_q(0) + C::QT_BYTES);
+        mma_sdp(tmem + C::TM_DP, kV, kst(0) + QT);
         umma_commit(bar_dp);
       }
       for (int t = 0; t < n_steps && ok; ++t) {
         const int st = t % QS;
-        const uint32_t aQ = stage_q(t);
-        const uint32_t adO = aQ + C::QT_BYTES;
+        const uint32_t mQ = mst(t) + dq_off, mdO = mQ + QT;
         const uint32_t tS = tmem + C::TM_S + (t & 1) * BR;
         // dV += P^T dO  (hi then lo half of P)
         if (!(ok = mbar_wait(bar_p, t & 1, abort_flag, p.status, WB_P))) break;
         tc_fence_after();
         for (int half = 0; half < 1 + p.split_p; ++half)
 #pragma unroll
-          for (int kk = 0; kk < BR / 16; ++kk) {
-            const uint32_t bo = (dcol0 / 64) * BR * 128 + kk * 2048;
-            umma_ts(tmem + C::TM_DV, tS + pcol(kk) + half * 16,
-                    sdesc_sw128(adO + bo, BR * 128, 1024), ID_KV,
-                    (t > 0 || kk > 0 || half > 0) ? 1u : 0u);
-          }
+          for (int kk = 0; kk < BR / 16; ++kk)
+            umma_ts_lo(tmem + C::TM_DV, tS + pcol(kk) + half * 16, mdO + kk * 128, ID_KV,
+                       (t > 0 || kk > 0 || half > 0) ? 1u : 0u);
         // S^T of the next step into the other buffer.  With one Q/dO stage
         // the next Q only arrives after this step's dK releases the stage,
         // so S^T_{t+1} then waits until after dQ_t (below).
@@ -623,11 +629,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
         if (!(ok = mbar_wait(bar_ds, t & 1, abort_flag, p.status, WB_DS))) break;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < BR / 16; ++kk) {
-          const uint32_t bo = (dcol0 / 64) * BR * 128 + kk * 2048;
-          umma_ts(tmem + C::TM_DK, tmem + C::TM_DP + pcol(kk),
-                  sdesc_sw128(aQ + bo, BR * 128, 1024), ID_KV, (t > 0 || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < BR / 16; ++kk)
+          umma_ts_lo(tmem + C::TM_DK, tmem + C::TM_DP + pcol(kk), mQ + kk * 128, ID_KV,
+                     (t > 0 || kk > 0) ? 1u : 0u);
         umma_commit(bar_qempty + st);
         // dQ^T = K^T dS^T  (M = 128 rows of d, N = BR queries, K = 128 keys).
         // For d = 64 the upper 64 rows of M read the V tile and are ignored.
@@ -635,16 +639,13 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
           break;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < BC / 16; ++kk) {
-          const uint32_t ao = (dcol0 / 64) * BC * 128 + kk * 2048;
-          umma_ss(tmem + C::TM_DQ, sdesc_sw128(aK + ao, BC * 128, 1024),
-                  sdesc_sw128(adS + kk * 2048, BC * 128, 1024), ID_DQ, kk > 0);
-        }
+        for (int kk = 0; kk < BC / 16; ++kk)
+          umma_ss_lo(tmem + C::TM_DQ, mK + dk_off + kk * 128, mdS + kk * 128, ID_DQ, kk > 0);
         umma_commit(bar_dqfull);
         if (QS == 1 && !(ok = next_s())) break;
         // dP^T of the next step (overwrites dS^T_t, read by dK_t above)
         if (t + 1 < n_steps) {
-          mma_sdp(tmem + C::TM_DP, aV, stage_q(t + 1) + C::QT_BYTES);
+          mma_sdp(tmem + C::TM_DP, kV, kst(t + 1) + QT);
           umma_commit(bar_dp);
         }
       }

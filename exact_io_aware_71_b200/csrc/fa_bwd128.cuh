@@ -6,15 +6,17 @@
 // N = 128 one, so the 64-query steps of the general kernel leave half of
 // the tensor pipe unused on S^T, dP^T and dQ^T.
 //
-// TMEM (512 columns) cannot hold S^T, dP^T, dQ^T, dK and dV of a 128-query
-// step side by side, so regions are reused within a step:
+// At d = 128, TMEM (512 columns) cannot hold S^T, dP^T, dQ^T, dK and dV of
+// a 128-query step side by side, so regions are reused within a step:
 //   SP  [0, 128)    S^T (fp32)  -> P^T as bf16 hi | lo pairs (per group)
 //   DP  [128, 256)  dP^T (fp32) -> dS^T as bf16 pairs -> dQ^T (fp32)
 //   DK  [256, 256 + d), DV [256 + d, 256 + 2d)
+// At d = 64, dQ^T has its own columns [384, 512).
 // MMA order per step t (one issuing thread; tcgen05 MMAs run in issue
 // order, so a later MMA never overwrites a region an earlier one reads):
 //   S_0, dP_0, then per step: [P_t] dV_t, S_{t+1}, [dS_t] dK_t, dQ_t,
 //   [dQ_t read out] dP_{t+1}
+// (d = 64: [dQ_{t-1} read out] dQ_t, then dP_{t+1} without a wait).
 // The compute warps form P_t while dP_t runs and dS_t while dV_t and
 // S_{t+1} run; the read-out warpgroup empties dQ^T_t from TMEM right away
 // (then reduce-adds it into the fp32 accumulator from registers), which
@@ -47,6 +49,9 @@ struct Bwd128Cfg {
   static constexpr int TM_DP = 128;
   static constexpr int TM_DK = 256;
   static constexpr int TM_DV = 256 + DH;
+  // dQ^T: its own columns when d = 64 leaves them free, else the DP region.
+  static constexpr bool DQ_OWN = (D == 64);
+  static constexpr int TM_DQ = DQ_OWN ? TM_DV + DH : TM_DP;
   static constexpr int TMEM_COLS = 512;
   static constexpr int NTHREADS = 512;
   static constexpr int REGS_COMPUTE = 144;              // warpgroups 0-1
@@ -57,6 +62,7 @@ struct Bwd128Cfg {
   static constexpr int SMEM_BYTES = 2 * K_BYTES + QS * STAGE_BYTES + DS_BYTES + 1024 + 1024;
   static_assert(REGS_NEEDED <= 65536, "register split");
   static_assert(TM_DV + DH <= TMEM_COLS, "TMEM budget");
+  static_assert(!DQ_OWN || TM_DQ + BR <= TMEM_COLS, "TMEM budget (dQ^T)");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
   static_assert(QS * STAGE_BYTES >= 2 * BC * DH * 2, "dK/dV staging fits in the Q/dO stages");
 };
@@ -235,74 +241,87 @@ __global__ void __launch_bounds__(Bwd128Cfg<D>::NTHREADS, 1)
       constexpr uint32_t ID_S = idesc_bf16_f32(128, BR, 0, 0);    // S^T, dP^T: K-major both
       constexpr uint32_t ID_KV = idesc_bf16_f32(128, DH, 0, 1);   // dV, dK: B MN-major
       constexpr uint32_t ID_DQ = idesc_bf16_f32(128, BR, 1, 1);   // dQ^T: A, B MN-major
-      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aS0 = smem_u32(sStage);
-      const uint32_t adS = smem_u32(sdS);
+      // Descriptor low words: K-major (S^T, dP^T operands) and MN-major (the
+      // B operands of dV, dK and both operands of dQ^T).
+      const uint32_t kK = sdesc_sw128_lo(smem_u32(sK), 16);
+      const uint32_t mK = sdesc_sw128_lo(smem_u32(sK), BC * 128);
+      const uint32_t kV = sdesc_sw128_lo(smem_u32(sV), 16);
+      const uint32_t kS0 = sdesc_sw128_lo(smem_u32(sStage), 16);
+      const uint32_t mS0 = sdesc_sw128_lo(smem_u32(sStage), BR * 128);
+      const uint32_t mdS = sdesc_sw128_lo(smem_u32(sdS), BC * 128);
+      constexpr uint32_t STG = C::STAGE_BYTES >> 4, QT = C::QT_BYTES >> 4;
       // A-operand column of k-step kk (16 queries) within a P^T / dS^T
       // region: each 32-query chunk (32 columns of S^T / dP^T) holds its
       // queries' bf16 pairs in its first 16 columns (P lo in the next 16).
       auto pcol = [](int kk) { return uint32_t((kk >> 1) * 32 + (kk & 1) * 8); };
-      auto stage_q = [&](int t) { return aS0 + (t % QS) * C::STAGE_BYTES; };
-      auto mma_kq = [&](uint32_t d_tm, uint32_t a_base, uint32_t b_base) {
-#pragma unroll 2
+      auto kst = [&](int t) { return kS0 + uint32_t(t % QS) * STG; };   // Q of step t, K-major
+      auto mst = [&](int t) { return mS0 + uint32_t(t % QS) * STG; };   // Q of step t, MN-major
+      auto mma_kq = [&](uint32_t d_tm, uint32_t a_lo, uint32_t b_lo) {
+#pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ko = (kk >> 2) * BC * 128 + (kk & 3) * 32;
-          const uint32_t qo = (kk >> 2) * BR * 128 + (kk & 3) * 32;
-          umma_ss(d_tm, sdesc_sw128(a_base + ko, 16, 1024), sdesc_sw128(b_base + qo, 16, 1024),
-                  ID_S, kk > 0);
+          const uint32_t ko = ((kk >> 2) * BC * 128 + (kk & 3) * 32) >> 4;
+          const uint32_t qo = ((kk >> 2) * BR * 128 + (kk & 3) * 32) >> 4;
+          umma_ss_lo(d_tm, a_lo + ko, b_lo + qo, ID_S, kk > 0);
         }
       };
       bool ok = mbar_wait(bar_kv, 0, abort_flag, p.status, WB_KV) &&
                 mbar_wait(bar_qfull + 0, 0, abort_flag, p.status, WB_QFULL);
       tc_fence_after();
       if (ok) {
-        mma_kq(tmem + C::TM_SP, aK, stage_q(0));
+        mma_kq(tmem + C::TM_SP, kK, kst(0));
         umma_commit(bar_s);
-        mma_kq(tmem + C::TM_DP, aV, stage_q(0) + C::QT_BYTES);
+        mma_kq(tmem + C::TM_DP, kV, kst(0) + QT);
         umma_commit(bar_dp);
       }
       for (int t = 0; t < n_steps && ok; ++t) {
         const int st = t % QS;
-        const uint32_t aQ = stage_q(t);
-        const uint32_t adO = aQ + C::QT_BYTES;
+        const uint32_t mQ = mst(t), mdO = mQ + QT;
         // dV += P^T dO  (hi, then lo when the precision rule asks for it)
         if (!(ok = mbar_wait(bar_p, t & 1, abort_flag, p.status, WB_P))) break;
         tc_fence_after();
         for (int half = 0; half < 1 + p.split_p; ++half)
-#pragma unroll 2
+#pragma unroll
           for (int kk = 0; kk < BR / 16; ++kk)
-            umma_ts(tmem + C::TM_DV, tmem + C::TM_SP + pcol(kk) + half * 16,
-                    sdesc_sw128(adO + kk * 2048, BR * 128, 1024), ID_KV,
-                    (t > 0 || kk > 0 || half > 0) ? 1u : 0u);
+            umma_ts_lo(tmem + C::TM_DV, tmem + C::TM_SP + pcol(kk) + half * 16, mdO + kk * 128,
+                       ID_KV, (t > 0 || kk > 0 || half > 0) ? 1u : 0u);
         // S^T of the next step (SP is free once dV_t has read P_t)
         if (t + 1 < n_steps) {
           if (!(ok = mbar_wait(bar_qfull + (t + 1) % QS, ((t + 1) / QS) & 1, abort_flag,
                                p.status, WB_QFULL)))
             break;
           tc_fence_after();
-          mma_kq(tmem + C::TM_SP, aK, stage_q(t + 1));
+          mma_kq(tmem + C::TM_SP, kK, kst(t + 1));
           umma_commit(bar_s);
         }
         // dK += dS^T Q
         if (!(ok = mbar_wait(bar_ds, t & 1, abort_flag, p.status, WB_DS))) break;
         tc_fence_after();
-#pragma unroll 2
+#pragma unroll
         for (int kk = 0; kk < BR / 16; ++kk)
-          umma_ts(tmem + C::TM_DK, tmem + C::TM_DP + pcol(kk),
-                  sdesc_sw128(aQ + kk * 2048, BR * 128, 1024), ID_KV, (t > 0 || kk > 0) ? 1u : 0u);
+          umma_ts_lo(tmem + C::TM_DK, tmem + C::TM_DP + pcol(kk), mQ + kk * 128, ID_KV,
+                     (t > 0 || kk > 0) ? 1u : 0u);
         umma_commit(bar_qempty + st);
-        // dQ^T = K^T dS^T into DP (M = 128 rows of d, N = 128 queries, K = 128
-        // keys); for d = 64 the upper 64 rows of M read the V tile and are
-        // ignored.
-#pragma unroll 2
-        for (int kk = 0; kk < BC / 16; ++kk)
-          umma_ss(tmem + C::TM_DP, sdesc_sw128(aK + kk * 2048, BC * 128, 1024),
-                  sdesc_sw128(adS + kk * 2048, BC * 128, 1024), ID_DQ, kk > 0);
-        umma_commit(bar_dqfull);
-        // dP^T of the next step, once dQ^T_t has left TMEM
-        if (t + 1 < n_steps) {
-          if (!(ok = mbar_wait(bar_dqempty, t & 1, abort_flag, p.status, WB_DQEMPTY))) break;
+        // dQ^T = K^T dS^T (M = 128 rows of d, N = 128 queries, K = 128 keys);
+        // for d = 64 the upper 64 rows of M read the V tile and are ignored.
+        // In its own columns it only waits for the read-out of dQ^T_{t-1}.
+        if constexpr (C::DQ_OWN) {
+          if (t > 0 &&
+              !(ok = mbar_wait(bar_dqempty, (t - 1) & 1, abort_flag, p.status, WB_DQEMPTY)))
+            break;
           tc_fence_after();
-          mma_kq(tmem + C::TM_DP, aV, stage_q(t + 1) + C::QT_BYTES);
+        }
+#pragma unroll
+        for (int kk = 0; kk < BC / 16; ++kk)
+          umma_ss_lo(tmem + C::TM_DQ, mK + kk * 128, mdS + kk * 128, ID_DQ, kk > 0);
+        umma_commit(bar_dqfull);
+        // dP^T of the next step; in the DP region it waits until dQ^T_t has
+        // left TMEM
+        if (t + 1 < n_steps) {
+          if constexpr (!C::DQ_OWN) {
+            if (!(ok = mbar_wait(bar_dqempty, t & 1, abort_flag, p.status, WB_DQEMPTY))) break;
+            tc_fence_after();
+          }
+          mma_kq(tmem + C::TM_DP, kV, kst(t + 1) + QT);
           umma_commit(bar_dp);
         }
       }
@@ -332,7 +351,7 @@ __global__ void __launch_bounds__(Bwd128Cfg<D>::NTHREADS, 1)
       uint32_t v[BR];
       if (r < DH) {
 #pragma unroll
-        for (int c = 0; c < BR / 32; ++c) FA_TMEM_LD32(tl + C::TM_DP + c * 32, (v + c * 32));
+        for (int c = 0; c < BR / 32; ++c) FA_TMEM_LD32(tl + C::TM_DQ + c * 32, (v + c * 32));
         tmem_wait_ld();
       }
       tc_fence_before();

@@ -272,6 +272,38 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   return d;
 }
 
+// The same descriptor as two 32-bit words.  For 128-byte swizzled operands
+// with a 1024-byte stride between 8-row groups the high word is a constant;
+// the low word holds the start address (16-byte units, bits 0-13) and the
+// leading byte offset (bits 16-29).  Adding (byte offset / 16) to the low word
+// moves the start address: shared-memory addresses stay below 2^18 bytes, so
+// the address field never carries into the offset field.
+constexpr uint32_t SDESC_SW128_HI = (1024u >> 4) | (1u << 14) | (2u << 29);
+__device__ __forceinline__ uint32_t sdesc_sw128_lo(uint32_t saddr, uint32_t lbo) {
+  return ((saddr >> 4) & 0x3FFFu) | (((lbo >> 4) & 0x3FFFu) << 16);
+}
+__device__ __forceinline__ void umma_ss_lo(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .b64 da, db;\n\t.reg .pred p;\n\t"
+      "mov.b64 da, {%1, %3};\n\t"
+      "mov.b64 db, {%2, %3};\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_lo), "r"(b_lo), "r"(SDESC_SW128_HI), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void umma_ts_lo(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .b64 db;\n\t.reg .pred p;\n\t"
+      "mov.b64 db, {%2, %3};\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(SDESC_SW128_HI), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // ---- TMEM <-> registers, 32 lanes x 32-bit shape: thread t of the warp
 // owns TMEM lane (warp quarter * 32 + t); .xN moves N consecutive columns.
 #define FA_TMEM_LD32(taddr, r)                                                              \
