@@ -262,14 +262,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, in
 
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version bits.
 // lbo/sbo in bytes.
-__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  uint64_t d = 0;
-  d |= uint64_t((saddr >> 4) & 0x3FFFu);
-  d |= uint64_t((lbo >> 4) & 0x3FFFu) << 16;
-  d |= uint64_t((sbo >> 4) & 0x3FFFu) << 32;
-  d |= uint64_t(1) << 46;   // descriptor version for sm_100
-  d |= uint64_t(2) << 61;   // SWIZZLE_128B
-  return d;
+__host__ __device__ __forceinline__ constexpr uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo,
+                                                                  uint32_t sbo) {
+  return uint64_t((saddr >> 4) & 0x3FFFu)              //
+         | (uint64_t((lbo >> 4) & 0x3FFFu) << 16)      //
+         | (uint64_t((sbo >> 4) & 0x3FFFu) << 32)      //
+         | (uint64_t(1) << 46)                         // descriptor version for sm_100
+         | (uint64_t(2) << 61);                        // SWIZZLE_128B
 }
 
 // The same descriptor as two 32-bit words.  For 128-byte swizzled operands
@@ -279,9 +278,21 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
 // moves the start address: shared-memory addresses stay below 2^18 bytes, so
 // the address field never carries into the offset field.
 constexpr uint32_t SDESC_SW128_HI = (1024u >> 4) | (1u << 14) | (2u << 29);
-__device__ __forceinline__ uint32_t sdesc_sw128_lo(uint32_t saddr, uint32_t lbo) {
+__host__ __device__ __forceinline__ constexpr uint32_t sdesc_sw128_lo(uint32_t saddr,
+                                                                     uint32_t lbo) {
   return ((saddr >> 4) & 0x3FFFu) | (((lbo >> 4) & 0x3FFFu) << 16);
 }
+// The split form is the full descriptor, and a k-step's offset added to the
+// low word equals the descriptor of the offset address (largest shared
+// address and offsets used by the kernels).
+static_assert((uint64_t(SDESC_SW128_HI) << 32 | sdesc_sw128_lo(0x1F000u, 16)) ==
+                  sdesc_sw128(0x1F000u, 16, 1024), "descriptor words (K-major)");
+static_assert((uint64_t(SDESC_SW128_HI) << 32 | sdesc_sw128_lo(0x8400u, 128 * 128)) ==
+                  sdesc_sw128(0x8400u, 128 * 128, 1024), "descriptor words (MN-major)");
+static_assert((uint64_t(SDESC_SW128_HI) << 32 |
+               (sdesc_sw128_lo(0x30000u, 16) + ((0x4000u + 96) >> 4))) ==
+                  sdesc_sw128(0x30000u + 0x4000u + 96, 16, 1024),
+              "descriptor low-word offset");
 __device__ __forceinline__ void umma_ss_lo(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
                                            uint32_t idesc, uint32_t accumulate) {
   asm volatile(
