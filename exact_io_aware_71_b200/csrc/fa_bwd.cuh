@@ -587,7 +587,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
       auto mst = [&](int t) { return mS0 + uint32_t(t % QS) * STG; };   // Q of step t, MN-major
       // S^T of step t into buffer t mod 2
       auto mma_s = [&](int t) { mma_sdp(tmem + C::TM_S + (t & 1) * BR, kK, kst(t)); };
-      // this CTA's 64-column share of d in the MN-major operands
+      // start of this CTA's share of d (DH columns, whole 64-column chunks) in
+      // the MN-major operands
       const uint32_t dq_off = uint32_t((dcol0 / 64) * BR * 128) >> 4;
       const uint32_t dk_off = uint32_t((dcol0 / 64) * BC * 128) >> 4;
       bool ok = mbar_wait(bar_kv, 0, abort_flag, p.status, WB_KV) &&
