@@ -131,3 +131,25 @@ def test_reference_arm_varlen_runs_on_cpu():
                                                 "--steps", "1", "--warmup", "1"]))
     assert out["impl"] == "reference" and out["value"] > 0
     assert out["config"]["workload"].endswith("_varlen20:60")
+
+
+@pytest.mark.parametrize("extra", [[], ["--block-density", "0.5"]])
+def test_reference_arm_line_keeps_the_contract(extra):
+    """The oracle arm's JSON line carries every key of the bench contract,
+    with its e2e and cpu_baseline describing the same CPU run."""
+    out = bench.run_reference(bench.parse_args(["--impl", "reference", "--workload",
+                                                "tiny_b1h2n128d64_full", "--steps", "1",
+                                                "--warmup", "1"] + extra))
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in out, key
+    assert out["impl"] == "reference" and out["higher_is_better"] is True
+    assert out["value"] > 0 and out["unit"] == "TFLOP/s" and out["n_gpus"] == 1
+    assert out["vs_baseline"] is None
+    cb = out["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == out["value"]
+    e2e = out["e2e"]
+    assert e2e["value"] == out["value"] and e2e["unit"] == out["unit"]
+    assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+    assert out["config"]["workload"].startswith("tiny_b1h2n128d64_full")
