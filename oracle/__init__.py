@@ -12,6 +12,7 @@ from .attention import (  # noqa: F401
     attention_forward_varlen,
     attention_backward,
     attention_backward_dq_rows,
+    attention_backward_kv_rows,
     attention_forward,
     attention_forward_rows,
     kv_head,

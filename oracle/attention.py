@@ -71,6 +71,7 @@ __all__ = [
     "attention_forward_rows",
     "attention_backward",
     "attention_backward_dq_rows",
+    "attention_backward_kv_rows",
 ]
 
 # Rows of S per chunk are chosen so one chunk of S holds at most this many
@@ -96,13 +97,15 @@ BLOCK = 128
 
 
 def scores(q_rows: np.ndarray, k: np.ndarray, scale: float, causal: bool,
-           row_index: np.ndarray, block_mask=None) -> np.ndarray:
+           row_index: np.ndarray, block_mask=None, col_index=None) -> np.ndarray:
     """Scaled, masked score rows S[r, j] for the query rows ``row_index``.
 
-    q_rows: [R, d] (the rows themselves), k: [Nk, d], row_index: [R] absolute
-    query positions (needed for the causal and block masks)."""
+    q_rows: [R, d] (the rows themselves), k: [C, d] (the key rows), row_index:
+    [R] absolute query positions, col_index: [C] absolute key positions of the
+    rows of ``k`` (default 0..C-1; both are needed for the causal and block
+    masks)."""
     s = scale * (q_rows @ k.T)
-    j = np.arange(k.shape[0])[None, :]
+    j = (np.arange(k.shape[0]) if col_index is None else np.asarray(col_index))[None, :]
     if causal:
         s = np.where(j > row_index[:, None], -np.inf, s)
     if block_mask is not None:
@@ -236,6 +239,62 @@ def attention_backward_dq_rows(q, k, v, do, causal: bool, scale: float, b: int, 
     d_row = (p * dp).sum(axis=1)
     ds = p * (dp - d_row[:, None])
     return scale * (ds @ kk)
+
+
+def attention_backward_kv_rows(q, k, v, do, causal: bool, scale: float, b: int, kvh: int,
+                               keys, heads=None, block_mask=None):
+    """dK and dV of selected key rows of one (batch, kv head).
+
+    Key row j of dK and dV sums over every query row i of every query head
+    of the kv group (the GQA/MQA sum of the FA2 article, section "具体实现"):
+
+        dV_j = sum_h sum_i P_ij dO_i
+        dK_j = scale * sum_h sum_i P_ij (dP_ij - D_i) q_i,  dP_ij = dO_i . v_j
+
+    Each term needs row i's LSE_i (for P_ij = exp(S_ij - LSE_i)) and
+    D_i = sum_j' P_ij' dP_ij', which are sums over the whole row.  So the
+    function first takes every row of each query head in chunks (exact:
+    rows are independent) to get LSE and D, exactly as attention_backward
+    does, and then forms the columns of P, dP and dS of the selected keys
+    only.  Under the causal mask a row chunk's scores are formed only for
+    the keys up to its last row; the keys beyond are masked for every row of
+    the chunk and add exp(-inf) = 0 to its sums.
+
+    heads: the query heads of the group to sum over (default: all of them;
+    a subset gives that subset's share of the sum).
+    Returns (dK [K, d], dV [K, d]) in fp64."""
+    q, k, v, do = _as64(q), _as64(k), _as64(v), _as64(do)
+    hq, nq = q.shape[1], q.shape[2]
+    hkv, nk = k.shape[1], k.shape[2]
+    g = hq // hkv
+    keys = np.asarray(keys, dtype=np.int64)
+    kk, vv = k[b, kvh], v[b, kvh]
+    heads = range(kvh * g, (kvh + 1) * g) if heads is None else heads
+    dk = np.zeros((len(keys), q.shape[3]))
+    dv = np.zeros((len(keys), q.shape[3]))
+    step = _chunk_rows(nq, nk)
+    for h in heads:
+        if kv_head(h, hq, hkv) != kvh:
+            raise ValueError(f"query head {h} does not read kv head {kvh}")
+        lse = np.empty(nq)
+        dd = np.empty(nq)
+        for r0 in range(0, nq, step):
+            rows = np.arange(r0, min(nq, r0 + step))
+            kmax = min(nk, int(rows[-1]) + 1) if causal else nk
+            s = scores(q[b, h, rows], kk[:kmax], scale, causal, rows, block_mask)
+            l_, p = _softmax_stats(s)
+            dp = do[b, h, rows] @ vv[:kmax].T
+            lse[rows] = l_
+            dd[rows] = (p * dp).sum(axis=1)
+        rows = np.arange(nq)
+        s = scores(q[b, h], kk[keys], scale, causal, rows, block_mask, col_index=keys)
+        empty = np.isneginf(lse)
+        p = np.where(empty[:, None], 0.0, np.exp(s - np.where(empty, 0.0, lse)[:, None]))
+        dp = do[b, h] @ vv[keys].T
+        ds = p * (dp - dd[:, None])
+        dv += p.T @ do[b, h]
+        dk += scale * (ds.T @ q[b, h])
+    return dk, dv
 
 
 # ------------------------------------------------------------------ variable-length batches

@@ -315,6 +315,51 @@ def test_dq_rows_match_full_backward():
         np.testing.assert_allclose(got, dq[1, 3, rows], atol=1e-14)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("hq,hkv,nq,nk", [(4, 2, 21, 21), (4, 1, 30, 17), (4, 4, 13, 29),
+                                          (8, 1, 40, 40)])
+def test_kv_rows_match_full_backward(monkeypatch, causal, hq, hkv, nq, nk):
+    """dK / dV of sampled key rows equal the full backward's rows; small row
+    chunks make the per-chunk causal key horizon cut across the rows."""
+    import oracle.attention as oa
+    monkeypatch.setattr(oa, "_MAX_CHUNK_ELEMS", 7 * nk)
+    q = rnd((2, hq, nq, 8), 70)
+    k = rnd((2, hkv, nk, 8), 71)
+    v = rnd((2, hkv, nk, 8), 72)
+    do = rnd((2, hq, nq, 8), 73)
+    _, dk, dv = oracle.attention_backward(q, k, v, do, causal, 0.4)
+    keys = [0, 1, nk // 2, nk - 1]
+    for kvh in range(hkv):
+        gk, gv = oracle.attention_backward_kv_rows(q, k, v, do, causal, 0.4, 1, kvh, keys)
+        np.testing.assert_allclose(gk, dk[1, kvh, keys], atol=1e-13)
+        np.testing.assert_allclose(gv, dv[1, kvh, keys], atol=1e-13)
+    # a subset of the group's heads gives that subset's share; the shares add up
+    g = hq // hkv
+    parts = [oracle.attention_backward_kv_rows(q, k, v, do, causal, 0.4, 0, 0, keys, heads=[h])
+             for h in range(g)]
+    np.testing.assert_allclose(sum(p_[0] for p_ in parts), dk[0, 0, keys], atol=1e-13)
+    np.testing.assert_allclose(sum(p_[1] for p_ in parts), dv[0, 0, keys], atol=1e-13)
+    if hkv > 1:                      # a head of another group is refused
+        with pytest.raises(ValueError):
+            oracle.attention_backward_kv_rows(q, k, v, do, causal, 0.4, 0, 0, keys,
+                                              heads=[hq - 1])
+
+
+def test_kv_rows_with_block_mask_and_empty_rows():
+    q = rnd((1, 2, 300, 8), 74)
+    k = rnd((1, 1, 260, 8), 75)
+    v = rnd((1, 1, 260, 8), 76)
+    do = rnd((1, 2, 300, 8), 77)
+    mask = np.array([[1, 0, 1], [0, 0, 0], [1, 1, 0]], np.uint8)   # query block 1 sees nothing
+    for causal in (False, True):
+        _, dk, dv = oracle.attention_backward(q, k, v, do, causal, 0.3, block_mask=mask)
+        keys = [0, 127, 128, 200, 259]
+        gk, gv = oracle.attention_backward_kv_rows(q, k, v, do, causal, 0.3, 0, 0, keys,
+                                                   block_mask=mask)
+        np.testing.assert_allclose(gk, dk[0, 0, keys], atol=1e-13)
+        np.testing.assert_allclose(gv, dv[0, 0, keys], atol=1e-13)
+
+
 def test_backward_group_subset():
     q = rnd((2, 4, 10, 4), 43)
     k = rnd((2, 2, 10, 4), 44)
