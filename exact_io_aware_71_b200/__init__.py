@@ -14,6 +14,8 @@ from .binding import (  # noqa: F401
     fa_fwd_strided,
     fa_fwd_block_sparse,
     fa_bwd_block_sparse,
+    fa_fwd_residual,
+    fa_bwd_residual,
     MASK_BLOCK,
     fa_fwd_varlen,
     fa_bwd_varlen,

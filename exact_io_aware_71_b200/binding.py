@@ -25,7 +25,8 @@ STATUS_NAMES = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED",
 SYMBOLS = ("fa_fwd", "fa_bwd", "fa_bwd_stage", "fa_bwd_workspace_size", "fa_status_string",
            "fa_device_status", "fa_bwd_noalloc", "fa_debug_inject", "fa_fwd_strided",
            "fa_bwd_strided", "fa_fwd_block_sparse", "fa_bwd_block_sparse", "fa_fwd_varlen",
-           "fa_bwd_varlen", "fa_bwd_varlen_workspace_size")
+           "fa_bwd_varlen", "fa_bwd_varlen_workspace_size", "fa_fwd_residual",
+           "fa_bwd_residual")
 
 # Rows / keys per block-mask entry (FA_MASK_BLOCK).
 MASK_BLOCK = 128
@@ -89,6 +90,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fa_bwd_varlen.restype = i
     lib.fa_bwd_varlen_workspace_size.argtypes = [i] * 6
     lib.fa_bwd_varlen_workspace_size.restype = sz
+    lib.fa_fwd_residual.argtypes = [vp] * 6 + [sp] + [i] * 7 + [f, vp]
+    lib.fa_fwd_residual.restype = i
+    lib.fa_bwd_residual.argtypes = [vp] * 10 + [sp] + [i] * 7 + [f, vp, sz, vp]
+    lib.fa_bwd_residual.restype = i
     lib.fa_bwd_noalloc.argtypes = lib.fa_bwd.argtypes[:17] + [vp]
     lib.fa_bwd_noalloc.restype = i
     lib.fa_bwd_workspace_size.argtypes = [i, i, i, i, i, i, i]
@@ -120,6 +125,21 @@ def fa_bwd_strided(q, k, v, o, lse, dO, dq, dk, dv, strides, B, Hq, Hkv, Nq, Nk,
     arr = (FaStrides * 8)(*strides) if strides is not None else None
     return load().fa_bwd_strided(q, k, v, o, lse, dO, dq, dk, dv, arr, B, Hq, Hkv, Nq, Nk, d,
                                  int(causal), float(scale), workspace, workspace_bytes, stream)
+
+
+def fa_fwd_residual(q, k, v, o, o_res, lse, strides, B, Hq, Hkv, Nq, Nk, d, causal, scale,
+                    stream) -> int:
+    arr = (FaStrides * 4)(*strides) if strides is not None else None
+    return load().fa_fwd_residual(q, k, v, o, o_res, lse, arr, B, Hq, Hkv, Nq, Nk, d,
+                                  int(causal), float(scale), stream)
+
+
+def fa_bwd_residual(q, k, v, o, o_res, lse, dO, dq, dk, dv, strides, B, Hq, Hkv, Nq, Nk, d,
+                    causal, scale, workspace, workspace_bytes, stream) -> int:
+    arr = (FaStrides * 8)(*strides) if strides is not None else None
+    return load().fa_bwd_residual(q, k, v, o, o_res, lse, dO, dq, dk, dv, arr, B, Hq, Hkv, Nq,
+                                  Nk, d, int(causal), float(scale), workspace, workspace_bytes,
+                                  stream)
 
 
 def fa_fwd_block_sparse(q, k, v, o, lse, strides, block_mask, B, Hq, Hkv, Nq, Nk, d, causal,
@@ -217,10 +237,13 @@ def _mask_ptr(block_mask, Nq, Nk):
     return block_mask.data_ptr()
 
 
-def forward(q, k, v, causal: bool, scale: float, out=None, lse=None, block_mask=None):
+def forward(q, k, v, causal: bool, scale: float, out=None, lse=None, block_mask=None,
+            o_res=None):
     """O, LSE for bf16 CUDA tensors q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d] (any
     strides with a contiguous last axis, e.g. permuted [B,N,H,d] storage).
-    block_mask: optional block-sparse mask, [ceil(Nq/128), ceil(Nk/128)]."""
+    block_mask: optional block-sparse mask, [ceil(Nq/128), ceil(Nk/128)].
+    o_res: optional tensor shaped and strided like the output that receives
+    its rounding residual (fa_fwd_residual; not with a block mask)."""
     import torch
     B, Hq, Hkv, Nq, Nk, d = _dims(q, k)
     if out is None:
@@ -229,7 +252,13 @@ def forward(q, k, v, causal: bool, scale: float, out=None, lse=None, block_mask=
         lse = torch.empty(B, Hq, Nq, dtype=torch.float32, device=q.device)
     ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr())
     strides = [strides_of(t) for t in (q, k, v, out)]
-    if block_mask is None:
+    if o_res is not None:
+        if block_mask is not None or o_res.stride() != out.stride() or o_res.shape != out.shape:
+            raise ValueError("o_res must be shaped and strided like the output, without a mask")
+        st = fa_fwd_residual(*ptrs[:4], o_res.data_ptr(), ptrs[4], strides, B, Hq, Hkv, Nq, Nk, d,
+                             causal, scale, _stream_handle())
+        what = "fa_fwd_residual"
+    elif block_mask is None:
         st = fa_fwd_strided(*ptrs, strides, B, Hq, Hkv, Nq, Nk, d, causal, scale,
                             _stream_handle())
         what = "fa_fwd_strided"
@@ -243,10 +272,11 @@ def forward(q, k, v, causal: bool, scale: float, out=None, lse=None, block_mask=
 
 
 def backward(q, k, v, o, lse, do, causal: bool, scale: float, workspace=None, grads=None,
-             block_mask=None):
+             block_mask=None, o_res=None):
     """dQ, dK, dV (bf16) for the forward inputs/outputs and dO; gradients
     take the strides of q, k, v unless `grads` gives the output tensors.
-    block_mask: the forward pass's block-sparse mask, if it had one."""
+    block_mask: the forward pass's block-sparse mask, if it had one.
+    o_res: the forward's residual output (fa_bwd_residual), if kept."""
     import torch
     B, Hq, Hkv, Nq, Nk, d = _dims(q, k)
     need = fa_bwd_workspace_size(B, Hq, Hkv, Nq, Nk, d, causal)
@@ -257,7 +287,14 @@ def backward(q, k, v, o, lse, do, causal: bool, scale: float, workspace=None, gr
     ts = (q, k, v, o, do, dq, dk, dv)
     ptrs = (*(t.data_ptr() for t in ts[:4]), lse.data_ptr(), *(t.data_ptr() for t in ts[4:]))
     strides = [strides_of(t) for t in ts]
-    if block_mask is None:
+    if o_res is not None:
+        if block_mask is not None or o_res.stride() != o.stride() or o_res.shape != o.shape:
+            raise ValueError("o_res must be shaped and strided like o, without a mask")
+        st = fa_bwd_residual(*ptrs[:4], o_res.data_ptr(), *ptrs[4:], strides, B, Hq, Hkv, Nq, Nk,
+                             d, causal, scale, workspace.data_ptr(), workspace.numel(),
+                             _stream_handle())
+        what = "fa_bwd_residual"
+    elif block_mask is None:
         st = fa_bwd_strided(*ptrs, strides, B, Hq, Hkv, Nq, Nk, d, causal, scale,
                             workspace.data_ptr(), workspace.numel(), _stream_handle())
         what = "fa_bwd_strided"

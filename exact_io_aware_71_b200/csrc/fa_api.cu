@@ -100,21 +100,16 @@ namespace {
 
 // Scratch of fa_bwd_noalloc (see fa.h).  In host code this name is only a
 // host-side stand-in for the array; its device address comes from
-// cudaGetSymbolAddress, looked up once per device with that device current.
+// cudaGetSymbolAddress, looked up on every call with the caller's device and
+// context current.  The lookup allocates nothing, and it is not cached: after
+// a device reset, or in another context, the module (and the array) can sit
+// at another address.
 __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
 
 void* noalloc_scratch() {
-  static std::mutex mu;
-  static void* addr[128] = {};
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
-    addr[dev] = p;
-  }
-  return addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+  return p;
 }
 
 DevStatus* status_ptr() {
@@ -137,13 +132,14 @@ int launch_kernel(KernelT kern, int smem, int threads, unsigned grid, const CUte
 
 // d = 64 / 128: two query tiles per CTA; d = 256: one.  MODE: dense,
 // block-sparse (p.mask) or packed variable-length batch (p.cu_q, p.cu_k).
-template <int D, bool CAUSAL, int MODE>
+// EPI: the epilogue (O and LSE, plus the residual, or D only).
+template <int D, bool CAUSAL, int MODE, int EPI>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                const CUtensorMap& mo, FwdParams p, cudaStream_t stream) {
   if constexpr (D == 256) {
     using C = FwdCfg<D>;
     p.n_units = p.n_qblocks;
-    return launch_kernel(fa_fwd_kernel<D, CAUSAL, MODE>, C::SMEM_BYTES, C::NTHREADS,
+    return launch_kernel(fa_fwd_kernel<D, CAUSAL, MODE, EPI>, C::SMEM_BYTES, C::NTHREADS,
                          unsigned(p.n_units) * unsigned(p.B * p.Hq), mq, mk, mv, mo, p, stream);
   } else {
     using C = FwdPairCfg<D>;
@@ -152,12 +148,13 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
     static int regs = -1;
     if (regs < 0) {
       cudaFuncAttributes fattr;
-      if (cudaFuncGetAttributes(&fattr, fa_fwd_pair_kernel<D, CAUSAL, MODE>) != cudaSuccess)
+      if (cudaFuncGetAttributes(&fattr, fa_fwd_pair_kernel<D, CAUSAL, MODE, EPI>) != cudaSuccess)
         return FA_ERR_CUDA;
       regs = fattr.numRegs;
     }
     if (regs * C::NTHREADS < C::REGS_NEEDED) return FA_ERR_UNSUPPORTED;
     p.n_units = (p.n_qblocks + 1) / 2;
+
     // Persistent (one CTA per SM, each walking a strided unit list) for short
     // rows, where unit boundaries are frequent, and for causal rows up to 16k,
     // whose units differ in length; one CTA per unit otherwise (measured
@@ -170,17 +167,29 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
     const long long units = (long long)p.n_units * p.B * p.Hq;
     const bool persistent = p.Nk <= 4096 || (CAUSAL && p.Nk <= 16384);
     const unsigned grid = unsigned(persistent ? std::min<long long>(units, sms) : units);
-    return launch_kernel(fa_fwd_pair_kernel<D, CAUSAL, MODE>, C::SMEM_BYTES, C::NTHREADS, grid,
-                         mq, mk, mv, mo, p, stream);
+    return launch_kernel(fa_fwd_pair_kernel<D, CAUSAL, MODE, EPI>, C::SMEM_BYTES, C::NTHREADS,
+                         grid, mq, mk, mv, mo, p, stream);
   }
+}
+
+// The residual output exists for fixed-length batches without a block mask;
+// the D epilogue for every mode.
+template <int D, bool CAUSAL, int MODE>
+int launch_fwd_epi(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                   const CUtensorMap& mo, const FwdParams& p, cudaStream_t stream) {
+  if (p.d_out) return launch_fwd<D, CAUSAL, MODE, EPI_D>(mq, mk, mv, mo, p, stream);
+  if constexpr (MODE == MODE_DENSE) {
+    if (p.o_res) return launch_fwd<D, CAUSAL, MODE, EPI_RES>(mq, mk, mv, mo, p, stream);
+  }
+  return launch_fwd<D, CAUSAL, MODE, EPI_O>(mq, mk, mv, mo, p, stream);
 }
 
 template <int D, bool CAUSAL>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                const CUtensorMap& mo, const FwdParams& p, cudaStream_t stream) {
-  return p.cu_q ? launch_fwd<D, CAUSAL, MODE_VARLEN>(mq, mk, mv, mo, p, stream)
-         : p.mask ? launch_fwd<D, CAUSAL, MODE_SPARSE>(mq, mk, mv, mo, p, stream)
-                  : launch_fwd<D, CAUSAL, MODE_DENSE>(mq, mk, mv, mo, p, stream);
+  return p.cu_q ? launch_fwd_epi<D, CAUSAL, MODE_VARLEN>(mq, mk, mv, mo, p, stream)
+         : p.mask ? launch_fwd_epi<D, CAUSAL, MODE_SPARSE>(mq, mk, mv, mo, p, stream)
+                  : launch_fwd_epi<D, CAUSAL, MODE_DENSE>(mq, mk, mv, mo, p, stream);
 }
 
 int launch_fwd_any(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
@@ -195,14 +204,16 @@ int launch_fwd_any(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorM
 }
 
 // The forward pass on strided tensors, with an optional block mask.
+// o_res: optional residual output at o's strides (null: none).
 int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse,
              const fa_strides* strides, const unsigned char* mask, int B, int Hq, int Hkv,
-             int Nq, int Nk, int d, int causal, float scale, cudaStream_t stream) {
+             int Nq, int Nk, int d, int causal, float scale, cudaStream_t stream,
+             void* o_res = nullptr) {
   if (!q || !k || !v || !o || !lse || !strides) return FA_ERR_INVALID_ARG;
   int st = check_sizes(B, Hq, Hkv, Nq, Nk, d, causal, scale);
   if (st != FA_OK) return st;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(lse) ||
-      !strides_ok(strides, 4))
+      !strides_ok(strides, 4) || (o_res && !aligned16(o_res)) || (mask && !aligned16(mask)))
     return FA_ERR_MISALIGNED;
   Strides sq{strides[0].batch, strides[0].head, strides[0].row};
   Strides sk{strides[1].batch, strides[1].head, strides[1].row};
@@ -233,6 +244,11 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse,
   p.cu_q = p.cu_k = nullptr;
   p.total_q = Nq;
   p.total_k = Nk;
+  p.o_res = static_cast<__nv_bfloat16*>(o_res);
+  p.d_out = nullptr;
+  p.d_ld = 0;
+  p.dO = nullptr;
+  p.do_sb = p.do_sh = p.do_sn = 0;
   return launch_fwd_any(mq, mk, mv, mo, p, d, causal, stream);
 }
 
@@ -288,6 +304,56 @@ int fwd_varlen_impl(const void* q, const void* k, const void* v, void* o, float*
   p.cu_k = cu_k;
   p.total_q = total_q;
   p.total_k = total_k;
+  p.o_res = nullptr;
+  p.d_out = nullptr;
+  p.d_ld = 0;
+  p.dO = nullptr;
+  p.do_sb = p.do_sh = p.do_sn = 0;
+  return launch_fwd_any(mq, mk, mv, mo, p, d, causal, stream);
+}
+
+// Exact D for the backward of a wide GQA / MQA group: the forward pass runs
+// again with the D epilogue and overwrites the workspace's D rows (written
+// from the bf16 O by the preprocess) with D = rowsum(dO o O), O in fp32.
+// st: strides of q, k, v, o, dO (fixed-length) as [B, H, N, d] views; vl:
+// packed batch or null; mask: block mask or null.  O and the LSE are read
+// by nobody here and written by nobody.
+int recompute_d(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                const void* dO, const Strides* st, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                int causal, float scale, const unsigned char* mask, const Varlen* vl,
+                void* workspace, DevStatus* status, cudaStream_t stream) {
+  const int rows_q = vl ? vl->total_q : Nq, rows_k = vl ? vl->total_k : Nk;
+  const int map_b = vl ? 1 : B;
+  const int bc = (d == 256) ? 64 : 128;
+  CUtensorMap mq, mk, mv, mo;
+  if (!make_map_bf16(&mq, q, d, rows_q, Hq, map_b, st[0], 128) ||
+      !make_map_bf16(&mk, k, d, rows_k, Hkv, map_b, st[1], bc) ||
+      !make_map_bf16(&mv, v, d, rows_k, Hkv, map_b, st[2], bc) ||
+      !make_map_bf16(&mo, o, d, rows_q, Hq, map_b, st[3], 32))
+    return FA_ERR_CUDA;
+  const BwdWorkspace w = vl ? bwd_workspace_layout_varlen(B, Hq, Hkv, vl->total_q, vl->total_k, d)
+                            : bwd_workspace_layout(B, Hq, Hkv, Nq, Nk, d);
+  FwdParams p;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Nq = Nq; p.Nk = Nk;
+  p.group = Hq / Hkv;
+  p.n_qblocks = (Nq + 127) / 128;
+  p.causal = causal;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.lse = const_cast<float*>(lse);
+  p.status = status;
+  p.mask = mask;
+  p.mask_ld = (Nk + MASK_BLOCK - 1) / MASK_BLOCK;
+  p.o = static_cast<__nv_bfloat16*>(const_cast<void*>(o));
+  p.o_sb = st[3].b; p.o_sh = st[3].h; p.o_sn = st[3].n;
+  p.cu_q = vl ? vl->cu_q : nullptr;
+  p.cu_k = vl ? vl->cu_k : nullptr;
+  p.total_q = rows_q;
+  p.total_k = rows_k;
+  p.o_res = nullptr;
+  p.d_out = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.d_off);
+  p.d_ld = vl ? varlen_lpad_ld(B, vl->total_q) : (long long)round_up(Nq, 128);
+  p.dO = static_cast<const __nv_bfloat16*>(dO);
+  p.do_sb = st[4].b; p.do_sh = st[4].h; p.do_sn = st[4].n;
   return launch_fwd_any(mq, mk, mv, mo, p, d, causal, stream);
 }
 
@@ -362,7 +428,8 @@ int bwd_impl(int stage, const void* q, const void* k, const void* v, const void*
              const float* lse, const void* dO, void* dq, void* dk, void* dv,
              const fa_strides* strides, int B, int Hq, int Hkv, int Nq, int Nk, int d,
              int causal, float scale, void* workspace, size_t workspace_bytes,
-             cudaStream_t stream, const unsigned char* mask = nullptr) {
+             cudaStream_t stream, const unsigned char* mask = nullptr,
+             const void* o_res = nullptr) {
   int stages;
   switch (stage) {
     case FA_BWD_ALL: stages = 7; break;
@@ -377,7 +444,7 @@ int bwd_impl(int stage, const void* q, const void* k, const void* v, const void*
   if (st != FA_OK) return st;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(lse) ||
       !aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
-      !strides_ok(strides, 8))
+      !strides_ok(strides, 8) || (o_res && !aligned16(o_res)) || (mask && !aligned16(mask)))
     return FA_ERR_MISALIGNED;
   const size_t need = bwd_workspace_bytes(B, Hq, Hkv, Nq, Nk, d);
   if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
@@ -386,8 +453,20 @@ int bwd_impl(int stage, const void* q, const void* k, const void* v, const void*
   if (!sp) return FA_ERR_CUDA;
   Strides s8[8];
   for (int i = 0; i < 8; ++i) s8[i] = Strides{strides[i].batch, strides[i].head, strides[i].row};
-  return launch_bwd(stages, q, k, v, o, lse, dO, dq, dk, dv, s8, B, Hq, Hkv, Nq, Nk, d, causal,
-                    scale, mask, nullptr, workspace, sp, stream);
+  if (stages & 1) {
+    int r = launch_bwd(1, q, k, v, o, o_res, lse, dO, dq, dk, dv, s8, B, Hq, Hkv, Nq, Nk, d,
+                       causal, scale, mask, nullptr, workspace, sp, stream);
+    if (r != FA_OK) return r;
+    // Wide groups without the forward's residual: exact D by recomputation.
+    if (!o_res && exact_dk(Hq / Hkv, d)) {
+      r = recompute_d(q, k, v, o, lse, dO, s8, B, Hq, Hkv, Nq, Nk, d, causal, scale, mask,
+                      nullptr, workspace, sp, stream);
+      if (r != FA_OK) return r;
+    }
+  }
+  if (!(stages & 6)) return FA_OK;
+  return launch_bwd(stages & 6, q, k, v, o, o_res, lse, dO, dq, dk, dv, s8, B, Hq, Hkv, Nq, Nk,
+                    d, causal, scale, mask, nullptr, workspace, sp, stream);
 }
 
 void contiguous8(fa_strides* s, int Hq, int Hkv, int Nq, int Nk, int d) {
@@ -444,6 +523,36 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
                       scale, workspace, workspace_bytes, stream);
 }
 
+int fa_fwd_residual(const void* q, const void* k, const void* v, void* o, void* o_res,
+                    float* lse, const fa_strides* strides, int B, int Hq, int Hkv, int Nq,
+                    int Nk, int d, int causal, float scale, cudaStream_t stream) {
+  if (!o_res) return FA_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1) return FA_ERR_INVALID_ARG;
+  fa_strides s[4];
+  if (!strides) {
+    contiguous4(s, Hq, Hkv, Nq, Nk, d);
+    strides = s;
+  }
+  return fwd_impl(q, k, v, o, lse, strides, nullptr, B, Hq, Hkv, Nq, Nk, d, causal, scale, stream,
+                  o_res);
+}
+
+int fa_bwd_residual(const void* q, const void* k, const void* v, const void* o,
+                    const void* o_res, const float* lse, const void* dO, void* dq, void* dk,
+                    void* dv, const fa_strides* strides, int B, int Hq, int Hkv, int Nq, int Nk,
+                    int d, int causal, float scale, void* workspace, size_t workspace_bytes,
+                    cudaStream_t stream) {
+  if (!o_res) return FA_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1) return FA_ERR_INVALID_ARG;
+  fa_strides s[8];
+  if (!strides) {
+    contiguous8(s, Hq, Hkv, Nq, Nk, d);
+    strides = s;
+  }
+  return bwd_impl(FA_BWD_ALL, q, k, v, o, lse, dO, dq, dk, dv, strides, B, Hq, Hkv, Nq, Nk, d,
+                  causal, scale, workspace, workspace_bytes, stream, nullptr, o_res);
+}
+
 int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
                    const void* dO, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq,
                    int Nk, int d, int causal, float scale, cudaStream_t stream) {
@@ -492,7 +601,15 @@ int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, co
   const Strides a = packed(Hq, total_q, d), b = packed(Hkv, total_k, d);
   const Strides s8[8] = {a, b, b, a, a, a, b, b};   // q, k, v, o, dO, dq, dk, dv
   const Varlen vl{cu_seqlens_q, cu_seqlens_k, total_q, total_k};
-  return launch_bwd(7, q, k, v, o, lse, dO, dq, dk, dv, s8, B, Hq, Hkv, max_seqlen_q,
+  int r = launch_bwd(1, q, k, v, o, nullptr, lse, dO, dq, dk, dv, s8, B, Hq, Hkv, max_seqlen_q,
+                     max_seqlen_k, d, causal, scale, nullptr, &vl, workspace, sp, stream);
+  if (r != FA_OK) return r;
+  if (exact_dk(Hq / Hkv, d)) {   // wide groups: exact D by recomputation
+    r = recompute_d(q, k, v, o, lse, dO, s8, B, Hq, Hkv, max_seqlen_q, max_seqlen_k, d, causal,
+                    scale, nullptr, &vl, workspace, sp, stream);
+    if (r != FA_OK) return r;
+  }
+  return launch_bwd(6, q, k, v, o, nullptr, lse, dO, dq, dk, dv, s8, B, Hq, Hkv, max_seqlen_q,
                     max_seqlen_k, d, causal, scale, nullptr, &vl, workspace, sp, stream);
 }
 

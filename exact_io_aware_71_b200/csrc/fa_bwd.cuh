@@ -38,6 +38,9 @@
 #pragma once
 #include "sm100.cuh"
 #include "fa_mask.cuh"
+#include "fa_rows.cuh"
+
+#include <type_traits>
 
 namespace fa {
 
@@ -75,6 +78,16 @@ struct BwdCfg {
 };
 
 inline int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+// Groups whose dK the backward computes from dS as bf16 hi + lo and from an
+// exact D (the forward's residual output, or D recomputed by a forward pass
+// with the D epilogue): the errors of a bf16 dS and of D from the bf16 O add
+// up over every query row of the group.  From 16 query heads per kv head
+// on at d <= 128; at d = 256, whose dK carries more of that error (measured
+// 2.1e-2 on a packed batch with 4 query heads per kv head), for every GQA /
+// MQA group.
+constexpr int kExactGroup = 16;
+inline bool exact_dk(int group, int d) { return group >= kExactGroup || (d == 256 && group > 1); }
 
 // Workspace: dQacc fp32 [B*Hq, Nq, d] | Dpad fp32 [B*Hq, Nq_pad] |
 // Lpad fp32 [B*Hq, Nq_pad] | (GQA/MQA only) dKacc, dVacc fp32 [B*Hkv, Nk, d]
@@ -128,22 +141,21 @@ struct Strides {
   long long b, h, n;
 };
 
-// Packed-batch helpers: sequence b's rows clamped to [0, total], and where
-// its padded fp32 row vectors (D, LSE) start in a head's workspace row:
-// 16-byte aligned, with room for ceil(n / 128) * 128 entries before the next
-// sequence (each sequence adds 256 entries of slack).
+// Packed-batch helper: sequence b's rows clamped to [0, total] (its padded
+// fp32 row vectors start at varlen_pad_start, fa_rows.cuh: 16-byte aligned,
+// with room for ceil(n / 128) * 128 entries before the next sequence).
 __device__ __forceinline__ void varlen_rows(const int* cu, int b, int total, int& off, int& n) {
   const int a = min(max(__ldg(cu + b), 0), total);
   n = min(max(__ldg(cu + b + 1), a), total) - a;
   off = a;
 }
-__device__ __forceinline__ long long varlen_pad_start(int off, int b) {
-  return (long long)((off + 3) & ~3) + 256LL * b;
-}
 
+// ores (optional, at o's strides): the forward's residual bf16(O - bf16(O));
+// D then uses o + ores, the fp32 output to 16 bits.
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(
-    const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
+    const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ ores,
+    const __nv_bfloat16* __restrict__ dO,
     const float* __restrict__ lse, float* __restrict__ dqacc, float* __restrict__ Dpad,
     float* __restrict__ Lpad, int rows_bh, int Hq, int Nq, int Nq_pad, Strides so, Strides sdo,
     float* __restrict__ kvacc, long long kv_n4) {
@@ -161,18 +173,21 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(
     if (valid) {
       const size_t e = (size_t(bh) * Nq + q) * D + sub * 8;
       const long long bb = bh / Hq, hh = bh - bb * Hq;
-      const uint4 ov = *reinterpret_cast<const uint4*>(o + bb * so.b + hh * so.h + q * so.n +
-                                                       sub * 8);
+      const long long oi = bb * so.b + hh * so.h + q * so.n + sub * 8;
+      const uint4 ov = *reinterpret_cast<const uint4*>(o + oi);
+      const uint4 rv = ores ? *reinterpret_cast<const uint4*>(ores + oi) : make_uint4(0u, 0u, 0u, 0u);
       const uint4 dv = *reinterpret_cast<const uint4*>(dO + bb * sdo.b + hh * sdo.h +
                                                        q * sdo.n + sub * 8);
       const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
+      const __nv_bfloat162* r2 = reinterpret_cast<const __nv_bfloat162*>(&rv);
       const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const float2 a = __bfloat1622float2(o2[i]);
+        const float2 r = __bfloat1622float2(r2[i]);
         const float2 b = __bfloat1622float2(d2[i]);
-        acc = fmaf(a.x, b.x, acc);
-        acc = fmaf(a.y, b.y, acc);
+        acc = fmaf(a.x + r.x, b.x, acc);
+        acc = fmaf(a.y + r.y, b.y, acc);
       }
       float4* z = reinterpret_cast<float4*>(dqacc + e);
       z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -372,7 +387,7 @@ __device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_
 
 // Block-sparse (SPARSE): a key block visits only the query blocks whose mask
 // entry for it is set, in the same cyclic order for every role.
-template <int D, bool CAUSAL, int MODE>
+template <int D, bool CAUSAL, int MODE, bool SPLIT_DS>
 __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
@@ -630,9 +645,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
         if (!(ok = mbar_wait(bar_ds, t & 1, abort_flag, p.status, WB_DS))) break;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < BR / 16; ++kk)
-          umma_ts_lo(tmem + C::TM_DK, tmem + C::TM_DP + pcol(kk), mQ + kk * 128, ID_KV,
-                     (t > 0 || kk > 0) ? 1u : 0u);
+        for (int half = 0; half < 1 + int(SPLIT_DS); ++half)
+#pragma unroll
+          for (int kk = 0; kk < BR / 16; ++kk)
+            umma_ts_lo(tmem + C::TM_DK, tmem + C::TM_DP + pcol(kk) + half * 16, mQ + kk * 128,
+                       ID_KV, (t > 0 || kk > 0 || half > 0) ? 1u : 0u);
         umma_commit(bar_qempty + st);
         // dQ^T = K^T dS^T  (M = 128 rows of d, N = BR queries, K = 128 keys).
         // For d = 64 the upper 64 rows of M read the V tile and are ignored.
@@ -799,7 +816,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
         for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4*>(dd + i) =
             *reinterpret_cast<const float4*>(sd + i);
         tmem_wait_ld();
-        uint32_t pk[16];
+        uint32_t pk[16], lo[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const float2 x = fadd2(make_float2(__uint_as_float(u[2 * i]),
@@ -807,8 +824,13 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
                                  make_float2(-dd[2 * i], -dd[2 * i + 1]));
           const float2 y = fmul2(make_float2(P[2 * i], P[2 * i + 1]), x);
           pk[i] = pack_bf16(y.x, y.y);
+          if constexpr (SPLIT_DS)
+            lo[i] = pack_bf16(y.x - __uint_as_float(pk[i] << 16),
+                              y.y - __uint_as_float(pk[i] & 0xFFFF0000u));
         }
         FA_TMEM_ST16(tDP, pk);
+        // dS lo over the group's other 16 columns (all 32 were read above)
+        if constexpr (SPLIT_DS) FA_TMEM_ST16(tDP + 16, lo);
         // dS^T row r, queries 32g..32g+31: half of a 128-byte swizzled row
         uint8_t* row = sdS + r * 128;
 #pragma unroll
@@ -940,7 +962,7 @@ struct Varlen {
 
 template <int D, bool CAUSAL>
 int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const void* o,
-                 const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                 const void* ores, const float* lse, const void* dO, void* dq, void* dk, void* dv,
                  const Strides* st, int B, int Hq, int Hkv, int Nq, int Nk, float scale,
                  const uint8_t* mask, const Varlen* vl, void* workspace, DevStatus* status,
                  cudaStream_t stream) {
@@ -1003,24 +1025,30 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
       const long long rows = (long long)bhq * Nq_pad;
       const long long blocks = std::min<long long>((rows + RPB - 1) / RPB, 148LL * 16);
       fa_bwd_pre_kernel<D><<<unsigned(blocks), 256, 0, stream>>>(
-          static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, dqacc,
+          static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(ores),
+          static_cast<const __nv_bfloat16*>(dO), lse, dqacc,
           Dpad, Lpad, bhq, Hq, Nq, Nq_pad, st[3], st[4], kvacc, kv_n4);
     }
     if (cudaGetLastError() != cudaSuccess) return 5;
   }
   if (stages & 2) {
     using C2 = typename std::conditional<STEP128, Bwd128Cfg<(D <= 128 ? D : 128)>, C>::type;
-    auto pick = [&]() {
+    // dK sums dS^T Q over every query row of the kv group: for wide groups
+    // rounding dS to bf16 alone moves dK by about 2e-2 (causal, N = 4096),
+    // so dS also goes in as hi + lo there (exact_dk).
+    const bool split_ds = exact_dk(group, D);
+    auto pick = [&](auto split_tag) {
+      constexpr bool S = decltype(split_tag)::value;
       if constexpr (STEP128)
-        return vl ? fa_bwd_main128_kernel<D, CAUSAL, BMODE_VARLEN>
-               : mask ? fa_bwd_main128_kernel<D, CAUSAL, BMODE_SPARSE>
-                      : fa_bwd_main128_kernel<D, CAUSAL, BMODE_DENSE>;
+        return vl ? fa_bwd_main128_kernel<D, CAUSAL, BMODE_VARLEN, S>
+               : mask ? fa_bwd_main128_kernel<D, CAUSAL, BMODE_SPARSE, S>
+                      : fa_bwd_main128_kernel<D, CAUSAL, BMODE_DENSE, S>;
       else
-        return vl ? fa_bwd_main_kernel<D, CAUSAL, BMODE_VARLEN>
-               : mask ? fa_bwd_main_kernel<D, CAUSAL, BMODE_SPARSE>
-                      : fa_bwd_main_kernel<D, CAUSAL, BMODE_DENSE>;
+        return vl ? fa_bwd_main_kernel<D, CAUSAL, BMODE_VARLEN, S>
+               : mask ? fa_bwd_main_kernel<D, CAUSAL, BMODE_SPARSE, S>
+                      : fa_bwd_main_kernel<D, CAUSAL, BMODE_DENSE, S>;
     };
-    auto kern = pick();
+    auto kern = split_ds ? pick(std::true_type{}) : pick(std::false_type{});
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C2::SMEM_BYTES) !=
         cudaSuccess)
       return 5;
@@ -1086,19 +1114,20 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
 // stages: bit 0 = preprocess, bit 1 = main, bit 2 = dq convert.  mask: the
 // block mask of block-sparse attention, or null; vl: a packed
 // variable-length batch, or null.
+// ores: the forward's residual output (o's strides), or null.
 inline int launch_bwd(int stages, const void* q, const void* k, const void* v, const void* o,
-                      const float* lse, const void* dO, void* dq, void* dk, void* dv,
-                      const Strides* st, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                      const void* ores, const float* lse, const void* dO, void* dq, void* dk,
+                      void* dv, const Strides* st, int B, int Hq, int Hkv, int Nq, int Nk, int d,
                       int causal, float scale, const uint8_t* mask, const Varlen* vl,
                       void* workspace, DevStatus* status, cudaStream_t stream) {
 #define FA_BWD_CASE(DD)                                                                          \
   if (d == DD)                                                                                   \
-    return causal ? launch_bwd_t<DD, true>(stages, q, k, v, o, lse, dO, dq, dk, dv, st, B, Hq,  \
-                                           Hkv, Nq, Nk, scale, mask, vl, workspace, status,     \
+    return causal ? launch_bwd_t<DD, true>(stages, q, k, v, o, ores, lse, dO, dq, dk, dv, st, B, \
+                                           Hq, Hkv, Nq, Nk, scale, mask, vl, workspace, status,  \
                                            stream)                                               \
-                  : launch_bwd_t<DD, false>(stages, q, k, v, o, lse, dO, dq, dk, dv, st, B, Hq, \
-                                            Hkv, Nq, Nk, scale, mask, vl, workspace, status,    \
-                                            stream);
+                  : launch_bwd_t<DD, false>(stages, q, k, v, o, ores, lse, dO, dq, dk, dv, st,   \
+                                            B, Hq, Hkv, Nq, Nk, scale, mask, vl, workspace,      \
+                                            status, stream);
   FA_BWD_CASE(64)
   FA_BWD_CASE(128)
   FA_BWD_CASE(256)

@@ -67,7 +67,7 @@ struct Bwd128Cfg {
   static_assert(QS * STAGE_BYTES >= 2 * BC * DH * 2, "dK/dV staging fits in the Q/dO stages");
 };
 
-template <int D, bool CAUSAL, int MODE>
+template <int D, bool CAUSAL, int MODE, bool SPLIT_DS>
 __global__ void __launch_bounds__(Bwd128Cfg<D>::NTHREADS, 1)
     fa_bwd_main128_kernel(const __grid_constant__ CUtensorMap tmQ,
                           const __grid_constant__ CUtensorMap tmK,
@@ -297,9 +297,11 @@ __global__ void __launch_bounds__(Bwd128Cfg<D>::NTHREADS, 1)
         if (!(ok = mbar_wait(bar_ds, t & 1, abort_flag, p.status, WB_DS))) break;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < BR / 16; ++kk)
-          umma_ts_lo(tmem + C::TM_DK, tmem + C::TM_DP + pcol(kk), mQ + kk * 128, ID_KV,
-                     (t > 0 || kk > 0) ? 1u : 0u);
+        for (int half = 0; half < 1 + int(SPLIT_DS); ++half)
+#pragma unroll
+          for (int kk = 0; kk < BR / 16; ++kk)
+            umma_ts_lo(tmem + C::TM_DK, tmem + C::TM_DP + pcol(kk) + half * 16, mQ + kk * 128,
+                       ID_KV, (t > 0 || kk > 0 || half > 0) ? 1u : 0u);
         umma_commit(bar_qempty + st);
         // dQ^T = K^T dS^T (M = 128 rows of d, N = 128 queries, K = 128 keys);
         // for d = 64 the upper 64 rows of M read the V tile and are ignored.
@@ -449,36 +451,55 @@ __global__ void __launch_bounds__(Bwd128Cfg<D>::NTHREADS, 1)
       ok = mbar_wait(bar_dp, t & 1, abort_flag, p.status, WB_DP);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
+      {
+        constexpr bool SPLIT = SPLIT_DS;
+        uint32_t lo_even[8];                        // dS lo of a chunk's first 16 queries
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t dpv[16];
-        FA_TMEM_LD16(tDP + c * 16, dpv);
-        tmem_wait_ld();
-        uint32_t pk[8];
+        for (int c = 0; c < 4; ++c) {
+          uint32_t dpv[16];
+          FA_TMEM_LD16(tDP + c * 16, dpv);
+          tmem_wait_ld();
+          uint32_t pk[8], lo[8];
 #pragma unroll
-        for (int i = 0; i < 8; i += 2) {
-          const float4 d4 = __ldg(dd4 + (c * 16 + 2 * i) / 4);
-          const float dsub[4] = {d4.x, d4.y, d4.z, d4.w};
+          for (int i = 0; i < 8; i += 2) {
+            const float4 d4 = __ldg(dd4 + (c * 16 + 2 * i) / 4);
+            const float dsub[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const float2 pp = make_float2(pf[c * 16 + 2 * (i + e)], pf[c * 16 + 2 * (i + e) + 1]);
-            const float2 x = fadd2(make_float2(__uint_as_float(dpv[2 * (i + e)]),
-                                               __uint_as_float(dpv[2 * (i + e) + 1])),
-                                   make_float2(-dsub[2 * e], -dsub[2 * e + 1]));
-            const float2 y = fmul2(pp, x);
-            pk[i + e] = pack_bf16(y.x, y.y);
+            for (int e = 0; e < 2; ++e) {
+              const float2 pp =
+                  make_float2(pf[c * 16 + 2 * (i + e)], pf[c * 16 + 2 * (i + e) + 1]);
+              const float2 x = fadd2(make_float2(__uint_as_float(dpv[2 * (i + e)]),
+                                                 __uint_as_float(dpv[2 * (i + e) + 1])),
+                                     make_float2(-dsub[2 * e], -dsub[2 * e + 1]));
+              const float2 y = fmul2(pp, x);
+              pk[i + e] = pack_bf16(y.x, y.y);
+              if constexpr (SPLIT)
+                lo[i + e] = pack_bf16(y.x - __uint_as_float(pk[i + e] << 16),
+                                      y.y - __uint_as_float(pk[i + e] & 0xFFFF0000u));
+            }
           }
-        }
-        // dS^T pairs over already read dP^T columns of this 32-query chunk
-        // (the chunk's first 16 columns, 8 per 16 queries) ...
-        FA_TMEM_ST8(tDP + (c >> 1) * 32 + (c & 1) * 8, pk);
-        // ... and into the shared tile for dQ: row r, queries [64g + 16c, +16)
-        uint8_t* rowp = sdS + g * (BC * 128) + r * 128;
+          // dS^T pairs over already read dP^T columns of this 32-query chunk
+          // (the chunk's first 16 columns, 8 per 16 queries) ...
+          FA_TMEM_ST8(tDP + (c >> 1) * 32 + (c & 1) * 8, pk);
+          // ... when split, the lo pairs over the chunk's last 16 columns,
+          // which are all read only once the chunk's second half is ...
+          if constexpr (SPLIT) {
+            if ((c & 1) == 0) {
 #pragma unroll
-        for (int q4 = 0; q4 < 2; ++q4) {
-          const int unit = c * 2 + q4;
-          *reinterpret_cast<uint4*>(rowp + ((unit ^ (r & 7)) * 16)) =
-              make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+              for (int i = 0; i < 8; ++i) lo_even[i] = lo[i];
+            } else {
+              FA_TMEM_ST8(tDP + (c >> 1) * 32 + 16, lo_even);
+              FA_TMEM_ST8(tDP + (c >> 1) * 32 + 24, lo);
+            }
+          }
+          // ... and into the shared tile for dQ: row r, queries [64g + 16c, +16)
+          uint8_t* rowp = sdS + g * (BC * 128) + r * 128;
+#pragma unroll
+          for (int q4 = 0; q4 < 2; ++q4) {
+            const int unit = c * 2 + q4;
+            *reinterpret_cast<uint4*>(rowp + ((unit ^ (r & 7)) * 16)) =
+                make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+          }
         }
       }
       tmem_wait_st();

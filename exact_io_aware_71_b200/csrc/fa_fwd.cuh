@@ -30,6 +30,7 @@
 #pragma once
 #include "sm100.cuh"
 #include "fa_mask.cuh"
+#include "fa_rows.cuh"
 
 // A row's O and sums are rescaled only when its running max (log2 units)
 // grows by more than this; in between, probabilities reach at most 2^threshold.
@@ -63,10 +64,27 @@ struct FwdParams {
   const int* cu_q;
   const int* cu_k;
   int total_q, total_k;
+  // Optional residual output (null: none): o_res = bf16(O - bf16(O)) at o's
+  // strides, the part of the fp32 output that rounding O to bf16 dropped.
+  // The backward pass forms D = rowsum(dO o (o + o_res)) from it.
+  __nv_bfloat16* o_res;
+  // D epilogue (null: the normal output).  The kernel then writes neither O
+  // nor the LSE: each row's epilogue dots its fp32 output with the row of
+  // dO and stores D = sum_c dO_c O_c into the backward workspace's row
+  // vector (fa_rows.cuh: entry bh * d_ld + row, or for packed batches
+  // h * d_ld + varlen_pad_start(cu_q[b], b) + row).
+  float* d_out;
+  long long d_ld;
+  const __nv_bfloat16* dO;
+  long long do_sb, do_sh, do_sn;
 };
 
 // Kernel variants: fixed-length batch, block-sparse, variable-length batch.
 enum : int { MODE_DENSE = 0, MODE_SPARSE = 1, MODE_VARLEN = 2 };
+// Epilogues: O and the LSE; the same plus the residual output; D only (the
+// backward's exact D for wide groups).  A compile-time choice, so the plain
+// output path carries none of the others' registers.
+enum : int { EPI_O = 0, EPI_RES = 1, EPI_D = 2 };
 
 // Where one (batch, head)'s rows live.  Fixed-length batches: rows [0, Nq)
 // of the (b, h) slice of the 4-D tensor maps.  Variable-length batches: rows
@@ -79,9 +97,12 @@ struct SeqGeo {
   int tq, tkv;         // TMA "bh" coordinates of q / o and of k / v
   float* lse;          // LSE of the sequence's row 0 at this head
   __nv_bfloat16* o;    // O of row 0 at this head (direct row stores)
+  __nv_bfloat16* ores; // residual output of row 0 (null: none)
+  float* dpad;         // D epilogue: D of row 0 (null: normal output)
+  const __nv_bfloat16* dO;   // D epilogue: dO of row 0
 };
 
-template <bool VARLEN>
+template <bool VARLEN, int EPI>
 __device__ __forceinline__ SeqGeo seq_geo(const FwdParams& p, int bh) {
   const int b = bh / p.Hq, h = bh - b * p.Hq;
   SeqGeo g;
@@ -98,6 +119,9 @@ __device__ __forceinline__ SeqGeo seq_geo(const FwdParams& p, int bh) {
     g.tkv = h / p.group;
     g.lse = p.lse + size_t(h) * p.total_q + q0;
     g.o = p.o + h * p.o_sh + (long long)q0 * p.o_sn;
+    g.ores = EPI == EPI_RES ? p.o_res + h * p.o_sh + (long long)q0 * p.o_sn : nullptr;
+    g.dpad = EPI == EPI_D ? p.d_out + h * p.d_ld + varlen_pad_start(q0, b) : nullptr;
+    g.dO = EPI == EPI_D ? p.dO + h * p.do_sh + (long long)q0 * p.do_sn : nullptr;
   } else {
     g.nq = p.Nq;
     g.nk = p.Nk;
@@ -106,6 +130,9 @@ __device__ __forceinline__ SeqGeo seq_geo(const FwdParams& p, int bh) {
     g.tkv = b * p.Hkv + h / p.group;
     g.lse = p.lse + size_t(bh) * p.Nq;
     g.o = p.o + b * p.o_sb + h * p.o_sh;
+    g.ores = EPI == EPI_RES ? p.o_res + b * p.o_sb + h * p.o_sh : nullptr;
+    g.dpad = EPI == EPI_D ? p.d_out + size_t(bh) * p.d_ld : nullptr;
+    g.dO = EPI == EPI_D ? p.dO + b * p.do_sb + h * p.do_sh : nullptr;
   }
   return g;
 }
@@ -113,12 +140,19 @@ __device__ __forceinline__ SeqGeo seq_geo(const FwdParams& p, int bh) {
 // A query row that sees no key at all (every block of its mask row is
 // zero, or its sequence has no keys): O = 0 and LSE = -inf, the limits of
 // an empty softmax.
-template <int D>
+// In the D epilogue nothing is written: the backward's preprocess already
+// set D = rowsum(dO o 0) = 0 for such a row.
+template <int D, int EPI>
 __device__ __forceinline__ void write_empty_row(const FwdParams& p, const SeqGeo& g, int grow) {
-  if (grow >= g.nq) return;
+  if (EPI == EPI_D || grow >= g.nq) return;
   uint4* dst = reinterpret_cast<uint4*>(g.o + (long long)grow * p.o_sn);
 #pragma unroll
   for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+  if (EPI == EPI_RES) {
+    uint4* dr = reinterpret_cast<uint4*>(g.ores + (long long)grow * p.o_sn);
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) dr[c] = make_uint4(0u, 0u, 0u, 0u);
+  }
   g.lse[grow] = -INFINITY;
 }
 
@@ -148,12 +182,19 @@ struct RowState {
 //   o_done the two barriers that complete after P V of even / odd blocks
 // The caller has waited for S; the function waits for P_{j-1} V_{j-1} only
 // if it has to rescale O.  Returns false if that wait gave up.
-template <int BC, int D, bool CAUSAL>
+// SPLIT_P (the residual and D epilogues): P also goes to TMEM as
+// lo = bf16(P - hi) over the block's last BC/2 columns (all of S has been
+// read by then), and the MMA issuer adds P_lo V, so the fp32 output that
+// the backward's D is formed from carries no bf16 rounding of P.
+// HALVES: once the first half of the block's keys has its P in TMEM, the
+// thread arrives on p_half (the MMA issuer starts that half's P V); the
+// caller arrives on the block's P-full barrier after the function returns.
+template <int BC, int D, bool CAUSAL, bool SPLIT_P = false, bool HALVES = false>
 __device__ __forceinline__ bool softmax_block(RowState& st, uint32_t tS, uint32_t tO, int j,
                                               bool first, int gj, int q_tile, int grow, int Nk,
                                               float sl2,
                                               uint64_t* o_done, volatile int* abort,
-                                              DevStatus* status) {
+                                              DevStatus* status, uint64_t* p_half = nullptr) {
   float s[BC];
   {
     uint32_t* r = reinterpret_cast<uint32_t*>(s);
@@ -219,7 +260,7 @@ __device__ __forceinline__ bool softmax_block(RowState& st, uint32_t tS, uint32_
   const float2 sl22 = make_float2(sl2, sl2), neg2 = make_float2(neg, neg);
 #pragma unroll
   for (int c = 0; c < BC / 32; ++c) {
-    uint32_t pk[16];
+    uint32_t pk[16], lo[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const int e = c * 32 + 2 * i;
@@ -230,8 +271,18 @@ __device__ __forceinline__ bool softmax_block(RowState& st, uint32_t tS, uint32_
       ar[i & 3] = fadd2(ar[i & 3], make_float2(__uint_as_float(pr << 16),
                                                __uint_as_float(pr & 0xFFFF0000u)));
       pk[i] = pr;
+      if constexpr (SPLIT_P)
+        lo[i] = pack_bf16(pp.x - __uint_as_float(pr << 16), pp.y - __uint_as_float(pr & 0xFFFF0000u));
     }
     FA_TMEM_ST16(tS + c * 16, pk);
+    if constexpr (SPLIT_P) FA_TMEM_ST16(tS + BC / 2 + c * 16, lo);
+    if constexpr (HALVES) {
+      if (c == BC / 64 - 1) {                      // keys [0, BC/2) are in TMEM
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(p_half);
+      }
+    }
   }
   const float2 la = fadd2(fadd2(al[0], al[1]), fadd2(al[2], al[3]));
   const float2 lb = fadd2(fadd2(ar[0], ar[1]), fadd2(ar[2], ar[3]));
@@ -247,13 +298,42 @@ __device__ __forceinline__ bool softmax_block(RowState& st, uint32_t tS, uint32_
 // 64 columns, TMA-stored by lane 0 of each warp; then the log-sum-exp.  In
 // a packed variable-length batch a warp whose 32 rows run past its
 // sequence's end stores its rows directly instead (a TMA box would spill
-// into the next sequence).
-template <int D, bool VARLEN>
+// into the next sequence).  With a residual output the row's residual
+// bf16(O - bf16(O)) is stored directly as well.  In the D epilogue
+// (g.dpad set) the row's fp32 output is only dotted with its row of dO and
+// D is written; O and the LSE are left alone.
+template <int D, bool VARLEN, int EPI>
 __device__ __forceinline__ void softmax_finish(const RowState& st, uint32_t tO, uint8_t* stage,
                                                int w, int lane, const CUtensorMap* tmO,
                                                int q_tile, const SeqGeo& g, long long o_sn,
-                                               int H, int grow) {
-  const float inv = 1.0f / st.lr;
+                                               long long do_sn, int H, int grow) {
+  // The residual and D epilogues' P V used P as hi + lo: normalise by the
+  // fp32 sum of P.
+  const float inv = 1.0f / (EPI != EPI_O ? st.l : st.lr);
+  if constexpr (EPI == EPI_D) {
+    const bool row_ok = grow < g.nq;
+    const uint4* dor = reinterpret_cast<const uint4*>(g.dO + (long long)(row_ok ? grow : 0) * do_sn);
+    float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t r[32];
+      FA_TMEM_LD32(tO + c * 32, r);
+      uint4 dv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) dv[u] = row_ok ? dor[c * 4 + u] : make_uint4(0u, 0u, 0u, 0u);
+      tmem_wait_ld();
+      const uint32_t* dw = reinterpret_cast<const uint32_t*>(dv);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float2 x = fmul2(make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])),
+                               make_float2(inv, inv));
+        acc = ffma2(x, make_float2(__uint_as_float(dw[i] << 16), __uint_as_float(dw[i] & 0xFFFF0000u)),
+                    acc);
+      }
+    }
+    if (row_ok) g.dpad[grow] = acc.x + acc.y;
+    return;
+  }
   const bool direct = VARLEN && (q_tile + w * 32 + 32 > g.nq);   // warp-uniform
 #pragma unroll
   for (int c = 0; c < D / 32; ++c) {
@@ -264,6 +344,20 @@ __device__ __forceinline__ void softmax_finish(const RowState& st, uint32_t tO, 
 #pragma unroll
     for (int i = 0; i < 16; ++i)
       pk2[i] = pack_bf16(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
+    if constexpr (EPI == EPI_RES) {
+      if (grow < g.nq) {
+        uint32_t rs[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          rs[i] = pack_bf16(__uint_as_float(r[2 * i]) * inv - __uint_as_float(pk2[i] << 16),
+                            __uint_as_float(r[2 * i + 1]) * inv -
+                                __uint_as_float(pk2[i] & 0xFFFF0000u));
+        uint4* dst = reinterpret_cast<uint4*>(g.ores + (long long)grow * o_sn + c * 32);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          dst[u] = make_uint4(rs[4 * u], rs[4 * u + 1], rs[4 * u + 2], rs[4 * u + 3]);
+      }
+    }
     if (direct) {
       if (grow < g.nq) {
         uint4* dst = reinterpret_cast<uint4*>(g.o + (long long)grow * o_sn + c * 32);
@@ -301,6 +395,11 @@ struct FwdPairCfg {
   static constexpr int Q_BYTES = BR * D * 2;        // one tile
   static constexpr int KV_BYTES = BC * D * 2;
   static constexpr int NS = (D == 64) ? 8 : 5;      // K/V ring slots
+  // P handed to the MMA issuer in two halves of 64 keys (P V of the first
+  // half runs while the second half is exponentiated): measured 1-2% faster
+  // at d = 64 and 4-5% slower at d = 128, where the extra handshake costs
+  // more than the overlap gains.
+  static constexpr bool P_HALVES = D == 64;
   static constexpr int TM_TILE = 256;               // tile t: S at t*256, O at t*256 + 128
   static constexpr int TMEM_COLS = 512;
   static constexpr int NTHREADS = 384;
@@ -319,15 +418,15 @@ enum : uint32_t { KV_T0 = 1, KV_T1 = 2, KV_LAST = 4, KV_EMPTY = 8, KV_ACT0 = 16,
 // head-major so that concurrently running units share K/V in L2, and under
 // the causal mask each head's longest pair comes first.  All roles walk the
 // same list; barrier phases run on across units.  Between units of a tile,
-// "Q free" (the epilogue's TMA store has read the staging buffer) gates the
-// next Q load and "O free" (the epilogue has read O from TMEM) gates the
-// next unit's first P V, while the tensor pipe already computes the next
-// unit's first S.
+// "Q free" (the epilogue's TMA store has read the staging buffer, the tile's
+// Q buffer) gates the next Q load and "O free" (the epilogue has read O from
+// TMEM) gates the next unit's first P V, while the tensor pipe already
+// computes the next unit's first S.
 //
 // Block-sparse (SPARSE): a unit's K/V stream is the union of the key blocks
 // its two tiles see; a tile takes part in the blocks its own mask row keeps,
 // and a tile that sees none is written out as empty rows.
-template <int D, bool CAUSAL, int MODE>
+template <int D, bool CAUSAL, int MODE, int EPI>
 __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
     fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
@@ -352,7 +451,8 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
   uint64_t* bar_q_free = bars + 10 + 2 * NS;   // [2] Q/staging buffer free (4 warps)
   uint64_t* bar_o_free = bars + 12 + 2 * NS;   // [2] O read out of TMEM (128 threads)
   uint64_t* bar_drain = bars + 14 + 2 * NS;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 16 + 2 * NS);
+  uint64_t* bar_p_half = bars + 16 + 2 * NS;   // [2] per tile (P halves only): first 64 keys' P
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + (C::P_HALVES ? 18 : 16) + 2 * NS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   // Block-sparse: the producer tags each K ring item with the tiles that
   // take its block (KV_T0, KV_T1), the unit's last block (KV_LAST) and, on
@@ -385,7 +485,7 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
       pu = u - bh * p.n_units;
     }
     q0 = pu * 2 * BR;
-    sg = seq_geo<VARLEN>(p, bh);
+    sg = seq_geo<VARLEN, EPI>(p, bh);
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
       const int qt = q0 + t * BR;
@@ -398,6 +498,7 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
       mbar_init(bar_q + i, 1);
       mbar_init(bar_s_full + i, 1);
       mbar_init(bar_p_full + i, BR);
+      if (C::P_HALVES) mbar_init(bar_p_half + i, BR);
       mbar_init(bar_q_free + i, 4);
       mbar_init(bar_o_free + i, BR);
     }
@@ -567,20 +668,55 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
         if (j == 0 && uses[t] > 1 &&
             !mbar_wait(bar_o_free + t, (uses[t] - 2) & 1, abort_flag, p.status, W_O_DONE))
           return false;
-        if (!mbar_wait(bar_p_full + t, gj & 1, abort_flag, p.status, W_P_FULL)) return false;
-        tc_fence_after();
+        // the residual and D epilogues also add P_lo V (P_lo in the block's
+        // last BC/2 columns)
+        constexpr int NPH = EPI != EPI_O ? 2 : 1;
+        constexpr int NH = C::P_HALVES ? 2 : 1;         // P handed over in NH parts
+        constexpr int KH = BC / 16 / NH;                // k-steps per part
+        if constexpr (NPH == 1 && NH == 1) {
+          if (!mbar_wait(bar_p_full + t, gj & 1, abort_flag, p.status, W_P_FULL)) return false;
+          tc_fence_after();
+          const uint32_t tt = tmem + t * C::TM_TILE;
+          if constexpr (LEAN) {
+            const uint32_t b0 = vlo + uint32_t(slot * (C::KV_BYTES >> 4));
+#pragma unroll
+            for (int kk = 0; kk < BC / 16; ++kk)
+              umma_ts_lo(tt + 128, tt + kk * 8, b0 + kk * 128, IDESC_O,
+                         (j > 0 || kk > 0) ? 1u : 0u);
+          } else {
+            const uint32_t vbase = sKV_addr + slot * C::KV_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < BC / 16; ++kk)
+              umma_ts(tt + 128, tt + kk * 8, sdesc_sw128(vbase + kk * 16 * 128, BC * 128, 1024),
+                      IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(bar_o_done + t * 2 + (gj & 1));
+          return true;
+        }
         const uint32_t tt = tmem + t * C::TM_TILE;
-        if constexpr (LEAN) {
-          const uint32_t b0 = vlo + uint32_t(slot * (C::KV_BYTES >> 4));
 #pragma unroll
-          for (int kk = 0; kk < BC / 16; ++kk)
-            umma_ts_lo(tt + 128, tt + kk * 8, b0 + kk * 128, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
-        } else {
-          const uint32_t vbase = sKV_addr + slot * C::KV_BYTES;
+        for (int hf = 0; hf < NH; ++hf) {
+          uint64_t* pb = (hf + 1 < NH) ? bar_p_half + t : bar_p_full + t;
+          if (!mbar_wait(pb, gj & 1, abort_flag, p.status, W_P_FULL)) return false;
+          tc_fence_after();
+          if constexpr (LEAN) {
+            const uint32_t b0 = vlo + uint32_t(slot * (C::KV_BYTES >> 4));
 #pragma unroll
-          for (int kk = 0; kk < BC / 16; ++kk)
-            umma_ts(tt + 128, tt + kk * 8, sdesc_sw128(vbase + kk * 16 * 128, BC * 128, 1024),
-                    IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+            for (int ph = 0; ph < NPH; ++ph)
+#pragma unroll
+              for (int kk = hf * KH; kk < (hf + 1) * KH; ++kk)
+                umma_ts_lo(tt + 128, tt + ph * (BC / 2) + kk * 8, b0 + kk * 128, IDESC_O,
+                           (j > 0 || kk > 0 || ph > 0) ? 1u : 0u);
+          } else {
+            const uint32_t vbase = sKV_addr + slot * C::KV_BYTES;
+#pragma unroll
+            for (int ph = 0; ph < NPH; ++ph)
+#pragma unroll
+              for (int kk = hf * KH; kk < (hf + 1) * KH; ++kk)
+                umma_ts(tt + 128, tt + ph * (BC / 2) + kk * 8,
+                        sdesc_sw128(vbase + kk * 16 * 128, BC * 128, 1024), IDESC_O,
+                        (j > 0 || kk > 0 || ph > 0) ? 1u : 0u);
+          }
         }
         umma_commit(bar_o_done + t * 2 + (gj & 1));
         return true;
@@ -694,7 +830,7 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
       if (nt[t] == 0) {
         // tile past its sequence's end, or (packed batches) a sequence with
         // queries but no keys
-        if (VARLEN && q0 + t * BR < sg.nq) write_empty_row<D>(p, sg, q0 + t * BR + row);
+        if (VARLEN && q0 + t * BR < sg.nq) write_empty_row<D, EPI>(p, sg, q0 + t * BR + row);
         continue;
       }
       int n = nt[t];
@@ -708,7 +844,7 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
       const int grow = q_tile + row;
       if constexpr (SPARSE) {
         if (n == 0) {                               // sees no key
-          write_empty_row<D>(p, sg, grow);
+          write_empty_row<D, EPI>(p, sg, grow);
           continue;
         }
       }
@@ -718,8 +854,9 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
           ok = mbar_wait(bar_s_full + t, (gb + j) & 1, abort_flag, p.status, W_S_FULL);
           if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
           tc_fence_after();
-          ok = softmax_block<BC, D, CAUSAL>(st, tl, tl + 128, j, j == 0, gb + j, q_tile, grow,
-                                            sg.nk, p.scale_log2, o_done, abort_flag, p.status);
+          ok = softmax_block<BC, D, CAUSAL, EPI != EPI_O, C::P_HALVES>(
+              st, tl, tl + 128, j, j == 0, gb + j, q_tile, grow, sg.nk, p.scale_log2, o_done,
+              abort_flag, p.status, bar_p_half + t);
           if (!ok) break;
           mbar_arrive(bar_p_full + t);
         }
@@ -734,8 +871,9 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
           ok = mbar_wait(bar_s_full + t, (gb + l) & 1, abort_flag, p.status, W_S_FULL);
           if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
           tc_fence_after();
-          ok = softmax_block<BC, D, CAUSAL>(st, tl, tl + 128, j, l == 0, gb + l, q_tile, grow,
-                                            sg.nk, p.scale_log2, o_done, abort_flag, p.status);
+          ok = softmax_block<BC, D, CAUSAL, EPI != EPI_O, C::P_HALVES>(
+              st, tl, tl + 128, j, l == 0, gb + l, q_tile, grow, sg.nk, p.scale_log2, o_done,
+              abort_flag, p.status, bar_p_half + t);
           if (!ok) break;
           mbar_arrive(bar_p_full + t);
         }
@@ -745,11 +883,11 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
       ok = mbar_wait(o_done + (jl & 1), (jl >> 1) & 1, abort_flag, p.status, W_O_DONE);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
-      softmax_finish<D, VARLEN>(st, tl + 128, sQ + t * C::Q_BYTES, w, lane, &tmO, q_tile, sg,
-                                p.o_sn, p.Hq, grow);
+      softmax_finish<D, VARLEN, EPI>(st, tl + 128, sQ + t * C::Q_BYTES, w, lane, &tmO, q_tile,
+                                     sg, p.o_sn, p.do_sn, p.Hq, grow);
       tc_fence_before();
       mbar_arrive(bar_o_free + t);                  // O has been read out of TMEM
-      if (lane == 0) mbar_arrive(bar_q_free + t);   // this warp's staging boxes were stored
+      if (lane == 0) mbar_arrive(bar_q_free + t);   // this warp's staging boxes were read
       gb += n;
     }
   }
@@ -783,7 +921,7 @@ struct FwdCfg {
 // Block-sparse (SPARSE): the tile walks only the key blocks its mask row
 // keeps (two 64-key blocks per mask block); the MMA issuer sees just the
 // sequence, the producer and softmax map it back to key blocks.
-template <int D, bool CAUSAL, int MODE>
+template <int D, bool CAUSAL, int MODE, int EPI>
 __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -814,7 +952,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
   const int bh = blockIdx.x / p.n_units;
   int qb = blockIdx.x - bh * p.n_units;
   if (CAUSAL) qb = p.n_units - 1 - qb;
-  const SeqGeo sg = seq_geo<VARLEN>(p, bh);
+  const SeqGeo sg = seq_geo<VARLEN, EPI>(p, bh);
   const int q_row0 = qb * BR;
   // A tile past its (packed) sequence's end has nothing to do.
   if (VARLEN && q_row0 >= sg.nq) return;
@@ -959,10 +1097,13 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
         if (!acquire(slot)) { ok = false; return; }
         const uint32_t a_tm = tmem + C::TM_S + (j & 1) * BC;   // P_j (bf16 pairs)
         const uint32_t b0 = vlo + uint32_t(slot * (C::KV_BYTES >> 4));
+        constexpr int NPH = EPI != EPI_O ? 2 : 1;   // residual / D epilogues add P_lo V
 #pragma unroll
-        for (int kk = 0; kk < BC / 16; ++kk)
-          umma_ts_lo(tmem + C::TM_O, a_tm + kk * 8, b0 + kk * 128, IDESC_O,
-                     (j > 0 || kk > 0) ? 1u : 0u);
+        for (int ph = 0; ph < NPH; ++ph)
+#pragma unroll
+          for (int kk = 0; kk < BC / 16; ++kk)
+            umma_ts_lo(tmem + C::TM_O, a_tm + ph * (BC / 2) + kk * 8, b0 + kk * 128, IDESC_O,
+                       (j > 0 || kk > 0 || ph > 0) ? 1u : 0u);
         umma_commit(bar_o_done + (j & 1));
         release(slot);
       };
@@ -987,7 +1128,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
     RowState st{-INFINITY, 0.f, 0.f};
     bool ok = true;
     if (n_blocks == 0) {                                 // sees no key (sparse)
-      write_empty_row<D>(p, sg, grow);
+      write_empty_row<D, EPI>(p, sg, grow);
       ok = false;
     }
     RowWalk rm;
@@ -996,9 +1137,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
       ok = mbar_wait(bar_s_full + (j & 1), (j >> 1) & 1, abort_flag, p.status, W_S_FULL);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
-      ok = softmax_block<BC, D, CAUSAL>(st, tl + C::TM_S + (j & 1) * BC, tl + C::TM_O, jb, j == 0,
-                                        j, q_row0, grow, sg.nk, p.scale_log2, bar_o_done,
-                                        abort_flag, p.status);
+      ok = softmax_block<BC, D, CAUSAL, EPI != EPI_O>(st, tl + C::TM_S + (j & 1) * BC,
+                                                     tl + C::TM_O, jb, j == 0, j, q_row0, grow,
+                                                     sg.nk, p.scale_log2, bar_o_done,
+                                                     abort_flag, p.status);
       if (!ok) break;
       mbar_arrive(bar_p_full + (j & 1));
     }
@@ -1007,8 +1149,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::NTHREADS, 1)
       ok = mbar_wait(bar_o_done + (jl & 1), (jl >> 1) & 1, abort_flag, p.status, W_O_DONE);
       if (__all_sync(0xffffffffu, ok)) {
         tc_fence_after();
-        softmax_finish<D, VARLEN>(st, tl + C::TM_O, sQ, warp, lane, &tmO, q_row0, sg, p.o_sn,
-                                  p.Hq, grow);
+        softmax_finish<D, VARLEN, EPI>(st, tl + C::TM_O, sQ, warp, lane, &tmO, q_row0, sg, p.o_sn,
+                                  p.do_sn, p.Hq, grow);
       }
     }
   }

@@ -25,9 +25,10 @@ __device__ __forceinline__ uint32_t nonzero_bytes(uint32_t x) {
 
 // Entries [32 w, 32 w + 32) of a mask row that lie below n, one bit each.
 // The bytes are fetched as the (at most three) aligned 16-byte chunks that
-// hold them, with independent vector loads; every chunk read holds at least
-// one byte of the row, so it lies within the mask's own memory page, and
-// its other bytes are discarded.
+// hold them, with independent vector loads, and the chunks' other bytes are
+// discarded.  The mask starts on a 16-byte boundary and its allocation
+// extends to the next multiple of 16 bytes (the C ABI requires both), so
+// every chunk lies inside the caller's allocation.
 __device__ __forceinline__ uint32_t mask_word(const uint8_t* row, int w, int n) {
   const int j0 = w * 32;
   const int cnt = min(32, n - j0);                   // entries wanted

@@ -99,6 +99,12 @@ size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int 
  * dk/dv sum over the query heads of each group.  `workspace` must hold
  * fa_bwd_workspace_size(...) bytes; its contents need not be initialised
  * and are clobbered.  The same `scale` and `causal` as the forward pass.
+ * Wide groups (Hq / Hkv >= 16, e.g. MQA; at d = 256 every Hq / Hkv >= 2):
+ * dk sums dS^T q over every query row of the group, so the rounding of
+ * D = rowsum(dO * O) from the bf16 o adds up; the pass then recomputes D
+ * from the fp32 output with one more forward pass (about the forward's
+ * time).  fa_fwd_residual / fa_bwd_residual give the same precision
+ * without it.
  */
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
            const void* dO, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nk,
@@ -123,7 +129,11 @@ int fa_bwd_strided(const void* q, const void* k, const void* v, const void* o, c
  *               entry (I, J) != 0 keeps the FA_MASK_BLOCK x FA_MASK_BLOCK
  *               block of query rows [I*128, I*128+128) and keys
  *               [J*128, J*128+128) (clipped to Nq, Nk).  Read-only, owned by
- *               the caller, unchanged until the kernels have finished.
+ *               the caller, unchanged until the kernels have finished.  The
+ *               kernels read it in aligned 16-byte chunks: it must start on
+ *               a 16-byte boundary (else FA_ERR_MISALIGNED) and its
+ *               allocation must extend to the next multiple of 16 bytes
+ *               (torch and cudaMalloc allocations do).
  * A removed block's scores count as -inf: the kernels neither load its K/V
  * nor compute it, so the work shrinks with the fraction of blocks kept.
  * With causal = 1 both masks apply.  A query row left with no visible key
@@ -181,10 +191,41 @@ int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, co
                   int total_q, int total_k, int Hq, int Hkv, int d, int causal, float scale,
                   void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/*
+ * Forward pass that also writes the output's rounding residual
+ *   o_res [B, Hq, Nq, d] bf16 (out), at o's strides: bf16(O - o), the part
+ *   of the fp32 output that rounding it to bf16 dropped,
+ * so that o + o_res holds the output to about 16 bits.  To make that the
+ * exact output to 16 bits, this pass also multiplies V by P as bf16 hi + lo
+ * (one more tensor-core product per key block, so it is slower than
+ * fa_fwd; o itself is then the exact output rounded once).  fa_bwd_residual
+ * takes o_res to form D = rowsum(dO * O) without recomputing the forward
+ * pass; that matters for wide GQA / MQA groups (see fa_bwd).  The pages have no
+ * counterpart; it serves their GQA / MQA setting (QbitAI FA2 article,
+ * section "具体实现", second small change).  strides: q, k, v, o as for
+ * fa_fwd_strided, or NULL for contiguous tensors.  Otherwise as fa_fwd.
+ */
+int fa_fwd_residual(const void* q, const void* k, const void* v, void* o, void* o_res,
+                    float* lse, const fa_strides* strides, int B, int Hq, int Hkv, int Nq,
+                    int Nk, int d, int causal, float scale, cudaStream_t stream);
+
+/*
+ * Backward pass with the forward's residual o_res (from fa_fwd_residual,
+ * same strides as o): D = rowsum(dO * (o + o_res)).  strides: 8 entries as
+ * for fa_bwd_strided, or NULL for contiguous tensors.  Otherwise as fa_bwd,
+ * with the same workspace.
+ */
+int fa_bwd_residual(const void* q, const void* k, const void* v, const void* o,
+                    const void* o_res, const float* lse, const void* dO, void* dq, void* dk,
+                    void* dv, const fa_strides* strides, int B, int Hq, int Hkv, int Nq, int Nk,
+                    int d, int causal, float scale, void* workspace, size_t workspace_bytes,
+                    cudaStream_t stream);
+
 /* Stages of fa_bwd, for callers that time or schedule them separately. */
 typedef enum {
   FA_BWD_ALL = 0,   /* the whole backward pass (same as fa_bwd) */
-  FA_BWD_PRE = 1,   /* D = rowsum(dO * O), LSE copy, dQ accumulator := 0 (in the workspace) */
+  FA_BWD_PRE = 1,   /* D = rowsum(dO * O), LSE copy, dQ accumulator := 0 (in the workspace);
+                       for wide groups also the forward pass that recomputes D (see fa_bwd) */
   FA_BWD_MAIN = 2,  /* dK, dV written; dQ accumulated into the workspace */
   FA_BWD_DQ = 3     /* dq = scale * dQ accumulator, as bf16 */
 } fa_bwd_stage_t;
@@ -219,9 +260,10 @@ int fa_bwd_stage(int stage, const void* q, const void* k, const void* v, const v
  * instead.  The call allocates nothing and calls no allocating routine.
  *  - Problems whose fa_bwd_workspace_size() exceeds FA_NOALLOC_SCRATCH_BYTES
  *    are rejected with FA_ERR_TOO_LARGE before anything is launched.
- *  - The first call on a device looks up the array's device address (with
- *    that device current) and caches it; make that first call before any
- *    stream capture.
+ *  - Every call looks up the array's device address in the caller's current
+ *    device and context (nothing is cached, so a device reset or another
+ *    context is followed).  The first lookup on a device may load the
+ *    library's device code; make that first call before any stream capture.
  *  - Every call shares the one array per device, and it keeps the last
  *    call's contents; the call re-initialises every part it reads.  Calls
  *    whose kernels overlap on the GPU (e.g. on two streams, or from two host

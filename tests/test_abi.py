@@ -142,6 +142,27 @@ def test_block_sparse_rejects_bad_arguments():
                                   0.125, None, 0, None) == 4
     assert fa.fa_fwd_block_sparse(A, A, A, A, A, None, A, 0, 2, 2, 128, 128, 64, 0, 0.125,
                                   None) == 1
+    # the mask is read in aligned 16-byte chunks: it must start on a 16-byte boundary
+    assert fa.fa_fwd_block_sparse(A, A, A, A, A, None, A + 1, 1, 2, 2, 128, 128, 64, 0, 0.125,
+                                  None) == 3
+    assert fa.fa_bwd_block_sparse(A, A, A, A, A, A, A, A, A, None, A + 8, 1, 2, 2, 128, 128, 64,
+                                  0, 0.125, A, 1 << 40, None) == 3
+
+
+def test_residual_entry_points_reject_bad_arguments():
+    """fa_fwd_residual / fa_bwd_residual: the residual pointer is required
+    and 16-byte aligned; the other checks are those of fa_fwd / fa_bwd."""
+    f = lambda **kw: fa.fa_fwd_residual(**dict(dict(
+        q=A, k=A, v=A, o=A, o_res=A, lse=A, strides=None, B=1, Hq=2, Hkv=2, Nq=128, Nk=128,
+        d=64, causal=0, scale=0.125, stream=None), **kw))
+    assert f(o_res=None) == 1 and f(q=None) == 1 and f(B=0) == 1 and f(d=80) == 2
+    assert f(o_res=A + 8) == 3 and f(o=A + 2) == 3
+    b = lambda **kw: fa.fa_bwd_residual(**dict(dict(
+        q=A, k=A, v=A, o=A, o_res=A, lse=A, dO=A, dq=A, dk=A, dv=A, strides=None, B=1, Hq=2,
+        Hkv=2, Nq=128, Nk=128, d=64, causal=0, scale=0.125, workspace=A,
+        workspace_bytes=1 << 40, stream=None), **kw))
+    assert b(o_res=None) == 1 and b(dO=None) == 1 and b(Hq=3) == 1
+    assert b(o_res=A + 4) == 3 and b(workspace=None) == 4 and b(workspace_bytes=16) == 4
 
 
 def test_varlen_rejects_bad_arguments():

@@ -21,8 +21,13 @@ int use_all(void) {
                int, float, cudaStream_t) = fa_fwd;
   size_t (*f_ws)(int, int, int, int, int, int, int) = fa_bwd_workspace_size;
   const char* (*f_str)(int) = fa_status_string;
+  int (*f_res)(const void*, const void*, const void*, void*, void*, float*, const fa_strides*,
+               int, int, int, int, int, int, int, float, cudaStream_t) = fa_fwd_residual;
+  int (*f_bres)(const void*, const void*, const void*, const void*, const void*, const float*,
+                const void*, void*, void*, void*, const fa_strides*, int, int, int, int, int,
+                int, int, float, void*, size_t, cudaStream_t) = fa_bwd_residual;
   fa_strides s = {1, 2, 3};
-  (void)f_fwd; (void)f_ws; (void)f_str; (void)s;
+  (void)f_fwd; (void)f_ws; (void)f_str; (void)f_res; (void)f_bres; (void)s;
   return FA_OK + FA_MASK_BLOCK;
 }
 """
@@ -38,6 +43,18 @@ def _compile(tmp_path, compiler, std, suffix):
                         "-I", INCLUDE, "-I", CUDA_INCLUDE, str(src)],
                        capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_header_constants_match_the_binding():
+    """The binding's copies of the header's constants (mask block, the
+    no-allocation scratch size) are the header's values."""
+    import re
+    from exact_io_aware_71_b200 import binding
+    text = open(os.path.join(INCLUDE, "fa.h")).read()
+    mb = int(re.search(r"#define FA_MASK_BLOCK (\d+)", text).group(1))
+    m = re.search(r"#define FA_NOALLOC_SCRATCH_BYTES \((\d+)ull << (\d+)\)", text)
+    assert mb == binding.MASK_BLOCK
+    assert int(m.group(1)) << int(m.group(2)) == binding.NOALLOC_SCRATCH_BYTES
 
 
 def test_header_compiles_as_c99(tmp_path):

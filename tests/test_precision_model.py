@@ -1,0 +1,129 @@
+"""An exact-arithmetic model of the backward pass's bf16 rounding points, and
+what it says about dK for wide GQA / MQA groups.  CPU only.
+
+dK_j = scale * sum_h sum_i dS_ij q_i sums over every query row of every
+query head that shares the kv head, so per-element rounding that is harmless
+for one head adds up over a group.  The kernels round in three places that
+matter here (all other arithmetic is fp32, far below these):
+
+  * the forward's P V takes P as bf16: its fp32 output O_f is
+    sum bf16(p) v / sum bf16(p); the forward with the residual output and
+    the recomputation below take P as hi + lo instead, which gives the
+    output to about 16 bits;
+  * D = rowsum(dO * O) is formed from the output the backward receives:
+    bf16(O_f) for fa_bwd, o + o_res for fa_bwd_residual, or, for the
+    recomputation the library runs for wide groups, the fp32 output of a
+    forward pass with P as hi + lo;
+  * dK's product takes dS as bf16, or as hi + lo (bf16(dS) + bf16(rest)).
+
+This file emulates exactly those roundings in fp64 numpy (torch's bf16
+round-to-nearest-even) and compares dK, rounded to bf16 as the kernels store
+it, with the fp64 oracle, per element against the parity tests' bound
+(tests/parity.py).  It is the evidence for three choices of the library:
+dS goes in as hi + lo for groups of 16 or more query heads per kv head,
+D comes from the residual or the recomputation there, and the peaky stress
+inputs (Q x 4) keep the Frobenius bar for dK.  It shares no code with the
+CUDA library; it models it.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_io_aware_71_b200.inputs import Workload, make_inputs
+from tests.parity import bound, to64
+
+
+def bf(x):
+    """Round fp64 values to bf16 (round to nearest even), back to fp64."""
+    return torch.from_numpy(np.ascontiguousarray(x)).to(torch.bfloat16).to(torch.float64).numpy()
+
+
+SCHEMES = ("plain", "split_only", "residual_bf16p", "residual", "recompute")
+
+
+def model_dk(q, k, v, do, causal, scale):
+    """dK of kv head 0 under each scheme (fp32 accumulations modelled as
+    exact; the output rounded to bf16).  q, do: [g, N, d]; k, v: [N, d]."""
+    g, n, d = q.shape
+    mask = np.arange(n)[None, :] > np.arange(n)[:, None]
+    acc = {s: np.zeros((n, d)) for s in SCHEMES}
+    for h in range(g):
+        s = scale * (q[h] @ k.T)
+        if causal:
+            s = np.where(mask, -np.inf, s)
+        e = np.exp(s - s.max(axis=1, keepdims=True))
+        p = e / e.sum(axis=1, keepdims=True)
+        et = bf(e)
+        o_f = (et @ v) / et.sum(axis=1, keepdims=True)            # forward, bf16 P
+        o_hilo = (et + bf(e - et)) @ v / e.sum(axis=1, keepdims=True)   # recompute, P hi + lo
+        dp = do[h] @ v.T
+        d_of = {"plain": bf(o_f), "split_only": bf(o_f), "residual_bf16p": bf(o_f) + bf(o_f - bf(o_f)),
+                "residual": bf(o_hilo) + bf(o_hilo - bf(o_hilo)), "recompute": o_hilo}
+        for sch in SCHEMES:
+            ds = p * (dp - (d_of[sch] * do[h]).sum(axis=1, keepdims=True))
+            hi = bf(ds)
+            ds_in = hi if sch == "plain" else hi + bf(ds - hi)
+            acc[sch] += scale * (ds_in.T @ q[h])
+    return {sch: bf(a) for sch, a in acc.items()}
+
+
+def excess(got, ref, tol=2e-2):
+    """Largest amount by which an element exceeds the per-element bound
+    (negative: every element within it)."""
+    b, _ = bound(ref, tol)
+    return float((np.abs(got - ref) - b).max())
+
+
+def run(Hq, Hkv, N, d, causal, seed, qmul=1.0):
+    wl = Workload("model", 1, Hq, Hkv, N, N, d, causal, seed)
+    q, k, v, do = (to64(t) for t in make_inputs(wl))
+    q = q * qmul                                   # exact in bf16 for powers of two
+    g = Hq // Hkv
+    ref = oracle.attention_backward(q, k, v, do, causal, wl.scale, heads=[(0, 0)])[1][0, 0]
+    got = model_dk(q[0, :g], k[0, 0], v[0, 0], do[0, :g], causal, wl.scale)
+    return {sch: excess(x, ref) for sch, x in got.items()}
+
+
+@pytest.fixture(scope="module")
+def mqa():
+    """32 query heads on one kv head, causal, N = 1024: the GPU test
+    test_mqa_wide_group's inputs."""
+    return run(32, 1, 1024, 128, True, seed=3)
+
+
+def test_mqa_plain_scheme_breaks_the_bar(mqa):
+    """D from the bf16 output and a bf16 dS: dK misses 2e-2 by about 1.6e-2."""
+    assert mqa["plain"] > 5e-3
+
+
+def test_mqa_splitting_ds_alone_is_not_enough(mqa):
+    """dS as hi + lo with D still from the bf16 output: still above the bar."""
+    assert mqa["split_only"] > 2e-3
+
+
+def test_mqa_split_ds_with_exact_d_meets_the_bar(mqa):
+    """dS as hi + lo and D from the residual output or the recomputation,
+    both with P as hi + lo: within the bound with room to spare.  A residual
+    of a forward with a bf16 P would only just make it, which is why the
+    residual forward splits P too."""
+    assert mqa["residual"] < -2e-3
+    assert mqa["recompute"] < -2e-3
+    assert -2e-3 < mqa["residual_bf16p"] < 0
+
+
+def test_narrow_groups_meet_the_bar_without_either():
+    """Four query heads per kv head (the long GQA workload's structure): the
+    plain scheme already holds dK within the bound."""
+    r = run(8, 2, 1024, 128, True, seed=4)
+    assert r["plain"] < 0
+
+
+def test_peaky_stress_input_misses_the_bar():
+    """Q x 4 (a stress input outside the named workloads, one query head
+    per kv head): the plain scheme, which the backward uses for such a
+    group, leaves dK above the per-element bound; D from the bf16 output is
+    the larger part (the split alone does not fix it).  The parity tests
+    hold dK to the Frobenius bar there."""
+    r = run(2, 2, 512, 64, True, seed=9, qmul=4.0)
+    assert r["plain"] > 0 and r["split_only"] > 0 and r["recompute"] < 0

@@ -69,6 +69,16 @@ def test_random_masks(d, causal, hq, hkv):
 
 
 @pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+def test_mqa_wide_group(d, causal):
+    """32 query heads on one kv head with a block mask that also empties a
+    query block: the backward's exact D is recomputed by the block-sparse
+    forward with the D epilogue, which leaves the empty rows' D at 0."""
+    wl = W(1, 32, 1, 700, 700, d, causal, seed=50 + d)
+    full_check(wl, make_block_mask(700, 700, 0.5, seed=d, empty_rows=(2,)))
+
+
+@pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("nq,nk", [(333, 700), (700, 333), (129, 1000)])
 def test_unequal_lengths(nq, nk, causal):
     wl = W(1, 2, 2, nq, nk, 128, causal, seed=nq + nk)

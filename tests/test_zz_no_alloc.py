@@ -4,12 +4,15 @@ allocation, or a latency-critical path where cudaMalloc, which may
 synchronise the device, is not allowed).  Its scratch is the library's
 built-in device array instead of a caller workspace.
 
-The test calls it twice in a row through the C ABI, on two different
+The test calls it several times in a row through the C ABI, on different
 problems, and checks each result against fa_bwd's on the same inputs, within
-the gradient tolerance the parity tests use (2e-2 max-abs).  The second call
-finds the first call's data still in the shared array, so it also shows that
-each call re-initialises what it reads.  The file is named to be collected
-last, and it passes alone in a fresh process as well as after the others.
+the gradient tolerance the parity tests use (2e-2 max-abs).  Each call finds
+the previous call's data still in the shared array, so it also shows that
+each call re-initialises what it reads: a GQA problem whose dK / dV partial
+sums live in the array follows an MHA one of another shape, and a wide
+group (32 query heads on one kv head, whose exact D is recomputed into the
+array) follows both.  The file is named to be collected last, and it passes
+alone in a fresh process as well as after the others.
 """
 import numpy as np
 import pytest
@@ -39,8 +42,9 @@ def _noalloc(wl, q, k, v, do, o, lse):
 
 
 @pytest.mark.gpu
-def test_noalloc_matches_fa_bwd_on_two_calls_in_a_row():
-    problems = [(2, 8, 2, 1024, 128, True, 31), (1, 4, 4, 640, 64, False, 32)]
+def test_noalloc_matches_fa_bwd_on_calls_in_a_row():
+    problems = [(2, 8, 2, 1024, 128, True, 31), (1, 4, 4, 640, 64, False, 32),
+                (1, 8, 2, 384, 64, False, 33), (1, 32, 1, 512, 128, True, 34)]
     for args in problems:
         wl, q, k, v, do, o, lse = _problem(*args)
         ref = fa.backward(q, k, v, o, lse, do, wl.causal, wl.scale)
