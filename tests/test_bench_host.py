@@ -108,10 +108,30 @@ def test_launches_per_step():
     from exact_io_aware_71_b200.inputs import workloads
     w = workloads()
     assert bench.launches_per_step(w["train_b8h16n2048d128_full"], 148) == 4
-    # 32 query heads on one kv head, 128 key blocks: split, plus the dK/dV convert
-    assert bench.launches_per_step(w["long_gqa_hkv1_n16384_d128_causal"], 148) == 5
+    # 32 query heads on one kv head, 128 key blocks: split, plus the dK/dV
+    # convert, plus the forward pass that recomputes D for the wide group
+    assert bench.launches_per_step(w["long_gqa_hkv1_n16384_d128_causal"], 148) == 6
     # 8 kv heads x 128 key blocks = 1024 CTAs: no split
     assert bench.launches_per_step(w["long_gqa_hkv8_n16384_d128_causal"], 148) == 4
+
+
+def test_roofline_picks_the_bound_by_arithmetic_intensity():
+    from exact_io_aware_71_b200.inputs import workloads
+    peaks = {"hbm_gbs": 6529.4, "bf16_tflops": 1674.6, "bf16_tflops_sustained": 1388.6}
+    w = workloads()
+    for name, bound in (("long_gqa_hkv8_n16384_d128_causal", "tensor"),
+                        ("sweep_n512_d64_full", "hbm")):
+        wl = w[name]
+        fb, bb = bench.algorithmic_bytes(wl)
+        # forward bytes: Q, K, V, O in bf16 plus the fp32 LSE
+        q = wl.B * wl.Hq * wl.Nq * wl.d
+        kv = wl.B * wl.Hkv * wl.Nk * wl.d
+        assert fb == 2 * (2 * q + 2 * kv) + 4 * wl.B * wl.Hq * wl.Nq
+        r = bench.roofline("k", wl.fwd_flops(), fb, 1.0, peaks, "measured")
+        assert r["bound"] == bound
+        assert r["tensor"]["tflops"] == pytest.approx(wl.fwd_flops() / 1e-3 / 1e12, rel=1e-3)
+        assert r["hbm"]["gbs"] == pytest.approx(fb / 1e-3 / 1e9, rel=1e-3)
+        assert r["frac"] == (r["hbm"]["frac"] if bound == "hbm" else r["tensor"]["frac"])
 
 
 def test_varlen_lengths_and_flops():
