@@ -217,11 +217,11 @@ def algorithmic_bytes(wl, frac: float = 1.0):
     return fwd, bwd
 
 
-def peak_clock_mhz():
-    """Median SM clock of the measured bf16 peak, if MEASURED_PEAKS.json
-    records one (else None)."""
+def peak_clock_mhz(path=None):
+    """Median SM clock of the measured bf16 peak, if the peaks file
+    (MEASURED_PEAKS.json by default) records one (else None)."""
     try:
-        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+        with open(path or os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             pk = json.load(f)
     except (OSError, ValueError):
         return None
@@ -233,7 +233,10 @@ def peak_clock_mhz():
         elif isinstance(x, (int, float)) and not isinstance(x, bool):
             yield path, float(x)
     cands = [(p, v) for p, v in walk(pk) if ("mhz" in p or "clock" in p) and "max" not in p
-             and ("bf16" in p or "gemm" in p or "tflops" in p) and 300 < v < 3000]
+             and 300 < v < 3000]
+    # prefer a clock recorded with the GEMM (bf16) measurement, then any SM clock
+    cands.sort(key=lambda c: (not any(t in c[0] for t in ("bf16", "gemm", "tflops")),
+                              "sm" not in c[0]))
     return cands[0][1] if cands else None
 
 
@@ -291,10 +294,32 @@ def kept_fraction(wl, mask) -> float:
     return float(kept / dense)
 
 
-def time_oracle(wl, seconds: float, max_groups=None, mask=None):
-    """fp64 oracle forward + backward on whole (batch, kv-head) groups of the
-    workload, as many as fit in about `seconds`; returns (TFLOP/s, cores,
-    sample description).  Work is exact per group, so the rate scales."""
+ORACLE_ROWS = 2048      # query rows per oracle timing sample
+
+
+def oracle_samples(wl):
+    """Timing samples of the fp64 oracle for a workload: blocks of up to
+    ORACLE_ROWS query rows of one (batch, query head), each against all of
+    that head's keys, in an order that spreads over batches, heads and rows
+    (last rows first).  Returns a list of (b, h, r0, r1)."""
+    rows = min(wl.Nq, ORACLE_ROWS)
+    blocks = [(r0, min(wl.Nq, r0 + rows)) for r0 in range(0, wl.Nq, rows)][::-1]
+    heads = [(b, h) for b in range(wl.B) for h in range(wl.Hq)]
+    order = []
+    for i in range(len(heads) * len(blocks)):
+        b, h = heads[(i * 7919) % len(heads)] if len(heads) > 1 else heads[0]
+        order.append((b, h) + blocks[(i // len(heads)) % len(blocks)])
+    return order
+
+
+def time_oracle(wl, seconds: float, max_samples=None, mask=None):
+    """fp64 oracle forward + backward on samples of the workload (see
+    oracle_samples), as many as fit in about `seconds`; returns (TFLOP/s,
+    cores, sample description, seconds, FLOPs).  The oracle forms every
+    query row's full row of scores (masked entries included), so its work
+    per row is the same for every row of a head: the time for the whole
+    workload is exactly the number of rows over the sampled rows times the
+    sampled time, and the rate is the workload's nominal FLOPs over that."""
     from threadpoolctl import threadpool_limits
 
     import oracle
@@ -306,30 +331,35 @@ def time_oracle(wl, seconds: float, max_groups=None, mask=None):
         _INPUT_CACHE[wl.name] = make_inputs(wl)
     q, k, v, do = _INPUT_CACHE[wl.name]
     g = wl.Hq // wl.Hkv
-    groups = [(b, j) for b in range(wl.B) for j in range(wl.Hkv)]
-    per_group_flops = 3.5 * wl.fwd_flops() * kept_fraction(wl, mask) / len(groups)
-    done, t_total = 0, 0.0
+    total_rows = wl.B * wl.Hq * wl.Nq
+    nominal = 3.5 * wl.fwd_flops() * kept_fraction(wl, mask)
+    done_rows, t_total, n = 0, 0.0, 0
     with threadpool_limits(limits=cores):
-        for (b, j) in groups:
-            if max_groups is not None and done >= max_groups:
+        for (b, h, r0, r1) in oracle_samples(wl):
+            if max_samples is not None and n >= max_samples:
                 break
-            qs = q[b:b + 1, j * g:(j + 1) * g].double().numpy()
-            dos = do[b:b + 1, j * g:(j + 1) * g].double().numpy()
+            j = h // g
+            qs = q[b:b + 1, h:h + 1, r0:r1].double().numpy()
+            dos = do[b:b + 1, h:h + 1, r0:r1].double().numpy()
             ks = k[b:b + 1, j:j + 1].double().numpy()
             vs = v[b:b + 1, j:j + 1].double().numpy()
+            m = None if mask is None else mask.numpy()[r0 // 128:(r1 + 127) // 128]
             t0 = time.perf_counter()
             oracle.attention_backward(qs, ks, vs, dos, wl.causal, wl.scale, return_aux=True,
-                                      block_mask=None if mask is None else mask.numpy())
+                                      block_mask=m)
             t_total += time.perf_counter() - t0
-            done += 1
-            if max_groups is None and t_total >= seconds and done >= 2:
+            done_rows += r1 - r0
+            n += 1
+            if max_samples is None and t_total >= seconds and n >= 2:
                 break
-    tflops = done * per_group_flops / t_total / 1e12
-    sample = (f"fp64 NumPy oracle fwd+bwd on {done} of {len(groups)} (batch, kv-head) groups "
-              f"({g} query head(s) each) of {wl.name}"
-              f"{'' if mask is None else ' with the same block mask'}; {t_total:.1f} s of CPU "
-              f"work; rate scaled exactly by FLOPs")
-    return tflops, cores, sample, t_total, done * per_group_flops
+    flops = nominal * done_rows / total_rows
+    tflops = flops / t_total / 1e12
+    sample = (f"fp64 NumPy oracle fwd+bwd on {n} sample(s) of up to {ORACLE_ROWS} query rows of one "
+              f"(batch, query head) against all its keys, {done_rows} of {total_rows} query rows "
+              f"of {wl.name}{'' if mask is None else ' with the same block mask'}; "
+              f"{t_total:.1f} s of CPU work; rate scaled by rows (the oracle's work per row is "
+              f"uniform)")
+    return tflops, cores, sample, t_total, flops
 
 
 # ----------------------------------------------------------------- packed batches
@@ -871,7 +901,7 @@ def run_reference(args):
     def sample_step():
         if lengths is not None:
             return time_oracle_varlen(wl, lengths, 0.0, max_seqs=1)
-        return time_oracle(wl, 0.0, max_groups=1, mask=mask)
+        return time_oracle(wl, 0.0, max_samples=1, mask=mask)
     for _ in range(args.warmup):
         sample_step()
     t_all, f_all = 0.0, 0.0
@@ -892,7 +922,8 @@ def run_reference(args):
                    + (f"_varlen{args.varlen}" if lengths is not None else ""),
                    "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "Nq": wl.Nq,
                    "Nk": wl.Nk, "d": wl.d, "causal": wl.causal,
-                   "step": "oracle fwd+bwd on one (batch, kv-head) group of the workload"},
+                   "step": "oracle fwd+bwd on one sample of the workload (up to 2048 query "
+                           "rows of one head against all its keys)"},
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,

@@ -134,6 +134,21 @@ def test_roofline_picks_the_bound_by_arithmetic_intensity():
         assert r["frac"] == (r["hbm"]["frac"] if bound == "hbm" else r["tensor"]["frac"])
 
 
+def test_peak_clock_lookup(tmp_path):
+    """The clock the measured peak was taken at is found in the peaks file
+    whatever its nesting; a clock recorded with the GEMM is preferred."""
+    import json
+    f = tmp_path / "peaks.json"
+    f.write_text(json.dumps({"bf16_tflops": 1674.6, "clocks": {"median_sm_mhz": 1327,
+                                                               "max_sm_mhz": 1965}}))
+    assert bench.peak_clock_mhz(str(f)) == 1327
+    f.write_text(json.dumps({"hbm": {"sm_clock_mhz": 1800}, "bf16": {"sm_clock_mhz": 1330}}))
+    assert bench.peak_clock_mhz(str(f)) == 1330
+    f.write_text(json.dumps({"bf16_tflops": 1674.6}))
+    assert bench.peak_clock_mhz(str(f)) is None
+    assert bench.peak_clock_mhz(str(tmp_path / "absent.json")) is None
+
+
 def test_varlen_lengths_and_flops():
     from exact_io_aware_71_b200.inputs import workloads
     wl = workloads()["train_b8h16n2048d128_causal"]
