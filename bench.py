@@ -121,8 +121,30 @@ def aggregate(local_ms: float, local_units: float, world: int, reduce_max=None):
     return t, local_units * world / (t / 1e3)
 
 
+# NVML clock-event reason bits (nvmlClocksEventReason*) reported in `clocks`
+NVML_REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                    "hw_thermal_slowdown": 0x40}
+
+
+def summarise_clock_samples(samples, t0: float, t1: float, max_mhz):
+    """Clock summary of the samples taken inside the timed window [t0, t1]
+    (host perf_counter seconds).  samples: (t, sm_mhz, power_w, reason_bits).
+    A reason counts if any window sample has it."""
+    win = [x for x in samples if t0 <= x[0] <= t1]
+    if not win:
+        return {"sm_mhz": None, "sm_max_mhz": max_mhz, "reasons": ["no samples"]}
+    reasons = sorted(n for n, bit in NVML_REASON_BITS.items() if any(x[3] & bit for x in win))
+    return {"sm_mhz": statistics.median(x[1] for x in win), "sm_max_mhz": max_mhz,
+            "reasons": reasons, "samples": len(win), "power_w_max": max(x[2] for x in win),
+            "source": "nvml, 5 ms polling inside the timed region"}
+
+
 class ClockSampler:
-    """nvidia-smi clock/throttle samples during the timed region."""
+    """SM clock, power and clock-event reasons during the timed region.
+    NVML is polled from a thread every 5 ms and only the samples between
+    start() and stop() (called right around the synchronised timed region)
+    are kept; without NVML, nvidia-smi samples at 100 ms instead.  Reads
+    only: no setting of the GPU is changed."""
 
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -132,8 +154,47 @@ class ClockSampler:
         self.index = index
         self.proc = None
         self.path = None
+        self.nvml = None
+        self.handle = None
+        self.samples = []
+        self.running = False
+        self.thread = None
+        self.t0 = self.t1 = 0.0
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(self.index).uuid)
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID("GPU-" + uuid)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.index)
+
+    def _poll(self):
+        nv, h = self.nvml, self.handle
+        while self.running:
+            try:
+                self.samples.append((time.perf_counter(),
+                                     float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                                     nv.nvmlDeviceGetPowerUsage(h) / 1000.0,
+                                     int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))))
+            except Exception:
+                pass
+            time.sleep(0.005)
 
     def start(self):
+        try:
+            import threading
+            self.nvml, self.handle = self._nvml_handle()
+            self.running = True
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            time.sleep(0.02)
+            self.t0 = time.perf_counter()
+            return
+        except Exception:
+            self.nvml = None
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
         try:
@@ -146,6 +207,15 @@ class ClockSampler:
             self.proc = None
 
     def stop(self):
+        if self.nvml is not None:
+            self.t1 = time.perf_counter()
+            self.running = False
+            self.thread.join()
+            try:
+                mx = float(self.nvml.nvmlDeviceGetMaxClockInfo(self.handle, self.nvml.NVML_CLOCK_SM))
+            except Exception:
+                mx = None
+            return summarise_clock_samples(self.samples, self.t0, self.t1, mx)
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         time.sleep(0.15)

@@ -61,6 +61,20 @@ def test_parse_clock_samples():
     assert bench.parse_clock_samples("")["sm_mhz"] is None
 
 
+def test_nvml_samples_outside_the_timed_window_are_dropped():
+    """Only samples between start() and stop() count: idle samples before
+    and after the timed region (at max clock, no reason) must not move the
+    median or hide a reason seen under load."""
+    cap, hw = bench.NVML_REASON_BITS["sw_power_cap"], bench.NVML_REASON_BITS["hw_slowdown"]
+    samples = [(0.0, 1965.0, 90.0, 0), (0.9, 1965.0, 95.0, hw),          # before the window
+               (1.0, 1800.0, 900.0, cap), (1.1, 1820.0, 950.0, cap), (1.2, 1850.0, 980.0, 0),
+               (2.5, 1965.0, 100.0, 0)]                                  # after it
+    c = bench.summarise_clock_samples(samples, 1.0, 1.2, 1965.0)
+    assert c["samples"] == 3 and c["sm_mhz"] == 1820.0 and c["sm_max_mhz"] == 1965.0
+    assert c["reasons"] == ["sw_power_cap"] and c["power_w_max"] == 980.0
+    assert bench.summarise_clock_samples(samples, 3.0, 4.0, 1965.0)["reasons"] == ["no samples"]
+
+
 def test_traffic_is_reported_only_for_current_sources(tmp_path, monkeypatch):
     prof = tmp_path / "profiles"
     prof.mkdir()
