@@ -259,17 +259,20 @@ DATASHEET_BF16_TFLOPS = 2250.0   # NVIDIA B200 dense BF16 (the sparse figure hal
 
 def launches_per_step(wl, sms: int) -> int:
     """Kernels one step launches: the forward kernel, the backward's
-    preprocess, main and dQ-convert kernels, the dK/dV convert kernel when a
-    GQA group's query heads are split over CTAs (the library splits when one
-    CTA per (batch, kv head, key block) would give fewer than two CTAs per
-    SM), and the D-recomputing forward pass for groups of 16 or more."""
+    preprocess, main and dQ-convert kernels; the fp16 copy of dO and V when
+    dP and dV take fp16 operands (GQA / MQA groups and d = 256, the library's
+    rule); the dK/dV convert kernel when a GQA group's query heads are split
+    over CTAs (the library splits when one CTA per (batch, kv head, key
+    block) would give fewer than two CTAs per SM); and the D-recomputing
+    forward pass for groups of 16 or more (any GQA group at d = 256)."""
     g = wl.Hq // wl.Hkv
+    f16 = g > 1 or wl.d == 256
     if g == 1:
-        return 4
+        return 4 + (1 if f16 else 0)
     base = ((wl.Nk + 127) // 128) * wl.B * wl.Hkv * (2 if wl.d == 256 else 1)
     gsplit = next((s_ for s_ in range(1, g + 1) if g % s_ == 0 and base * s_ >= 2 * sms), g)
     exact = g >= EXACT_GROUP or (wl.d == 256 and g > 1)
-    return 4 + (1 if gsplit > 1 else 0) + (1 if exact else 0)
+    return 4 + 1 + (1 if gsplit > 1 else 0) + (1 if exact else 0)
 
 
 def algorithmic_bytes(wl, frac: float = 1.0):

@@ -15,8 +15,8 @@
 //                   the diagonal ("step" t):
 //                     S^T  = K_j Q_i^T           (TMEM, lanes = keys)
 //                     P^T  = exp2(S^T * scale*log2e - LSE_i*log2e)
-//                     dV_j += P^T dO_i           (P^T from TMEM; bf16 hi + lo for GQA, d=256)
-//                     dP^T = V_j dO_i^T
+//                     dV_j += P^T dO_i           (P^T from TMEM; fp16 P and dO for GQA, d=256)
+//                     dP^T = V_j dO_i^T          (fp16 V and dO with them)
 //                     dS^T = P^T o (dP^T - D_i)
 //                     dK_j += dS^T Q_i           (dS^T read from TMEM)
 //                     dQ_i^T = K_j^T dS^T  -> fp32 reduce-add into dQacc
@@ -89,12 +89,29 @@ inline int round_up(int x, int m) { return (x + m - 1) / m * m; }
 constexpr int kExactGroup = 16;
 inline bool exact_dk(int group, int d) { return group >= kExactGroup || (d == 256 && group > 1); }
 
+// Problems whose dP^T and dV products take fp16 operands (scaled copies of
+// dO and V, and P as fp16): where a bf16 P rounds too coarsely for dV.  A
+// GQA / MQA group adds that rounding up over every query head of the group,
+// and at d = 256 |dV| is large enough that the output rounding leaves no
+// room.  MHA at d <= 128 keeps bf16 operands and skips the fp16 copies.
+inline bool bwd_f16(int Hq, int Hkv, int d) { return Hq > Hkv || d == 256; }
+
 // Workspace: dQacc fp32 [B*Hq, Nq, d] | Dpad fp32 [B*Hq, Nq_pad] |
 // Lpad fp32 [B*Hq, Nq_pad] | (GQA/MQA only) dKacc, dVacc fp32 [B*Hkv, Nk, d]
-// for the partial sums of a kv group split across CTAs.
+// for the partial sums of a kv group split across CTAs | (bwd_f16 only)
+// dO16 fp16 [B*Hq, Nq, d] and V16 fp16 [B*Hkv, Nk, d]: dO and V scaled by
+// powers of two (the operands of the dP^T and dV products) | amax: two
+// words, the largest |dO| and |V| (float bits) that choose those powers.
 struct BwdWorkspace {
-  size_t dq_off, d_off, l_off, kv_off, kv_elems, total;
+  size_t dq_off, d_off, l_off, kv_off, kv_elems, do16_off, v16_off, amax_off, total;
 };
+inline void bwd_workspace_tail(BwdWorkspace& w, size_t do_elems, size_t v_elems) {
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  w.do16_off = w.kv_off + up(2 * w.kv_elems * 4);
+  w.v16_off = w.do16_off + up(do_elems * 2);
+  w.amax_off = w.v16_off + up(v_elems * 2);
+  w.total = w.amax_off + 256;
+}
 inline BwdWorkspace bwd_workspace_layout(int B, int Hq, int Hkv, int Nq, int Nk, int d) {
   const size_t bh = size_t(B) * Hq;
   const size_t nq_pad = size_t(round_up(Nq, 128));
@@ -105,7 +122,8 @@ inline BwdWorkspace bwd_workspace_layout(int B, int Hq, int Hkv, int Nq, int Nk,
   w.l_off = w.d_off + up(bh * nq_pad * 4);
   w.kv_off = w.l_off + up(bh * nq_pad * 4);
   w.kv_elems = (Hq > Hkv) ? size_t(B) * Hkv * Nk * d : 0;   // per tensor
-  w.total = w.kv_off + up(2 * w.kv_elems * 4);
+  const bool f16 = bwd_f16(Hq, Hkv, d);
+  bwd_workspace_tail(w, f16 ? bh * Nq * d : 0, f16 ? size_t(B) * Hkv * Nk * d : 0);
   return w;
 }
 inline size_t bwd_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d) {
@@ -115,7 +133,8 @@ inline size_t bwd_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d)
 // Packed variable-length batch of B sequences: dQacc fp32 [Hq, total_q, d] |
 // Dpad, Lpad fp32 [Hq, ld] with ld = round_up(total_q, 4) + 256 (B + 1),
 // each sequence's rows starting at varlen_pad_start | (GQA/MQA only)
-// dKacc, dVacc fp32 [Hkv, total_k, d].
+// dKacc, dVacc fp32 [Hkv, total_k, d] | dO16 fp16 [Hq, total_q, d] |
+// V16 fp16 [Hkv, total_k, d] | amax.
 inline long long varlen_lpad_ld(int B, int total_q) {
   return (long long)((total_q + 3) & ~3) + 256LL * (B + 1);
 }
@@ -129,7 +148,8 @@ inline BwdWorkspace bwd_workspace_layout_varlen(int B, int Hq, int Hkv, int tota
   w.l_off = w.d_off + up(size_t(Hq) * ld * 4);
   w.kv_off = w.l_off + up(size_t(Hq) * ld * 4);
   w.kv_elems = (Hq > Hkv) ? size_t(Hkv) * total_k * d : 0;
-  w.total = w.kv_off + up(2 * w.kv_elems * 4);
+  const bool f16 = bwd_f16(Hq, Hkv, d);
+  bwd_workspace_tail(w, f16 ? size_t(Hq) * total_q * d : 0, f16 ? size_t(Hkv) * total_k * d : 0);
   return w;
 }
 
@@ -152,18 +172,121 @@ __device__ __forceinline__ void varlen_rows(const int* cu, int b, int total, int
 
 // ores (optional, at o's strides): the forward's residual bf16(O - bf16(O));
 // D then uses o + ores, the fp32 output to 16 bits.
+// ---- fp16 operands of the dP^T and dV products.  dO and V are copied once
+// into fp16, each scaled by a power of two 2^e chosen from its largest
+// magnitude m (m * 2^e in [2^14, 2^15), below fp16's largest finite value),
+// so the copies are exact for every element within 2^24 of m (smaller ones
+// keep an absolute error below m * 2^-25).  P then goes into dV as fp16
+// (relative rounding 2^-11 instead of bf16's 2^-8), which keeps dV within
+// the parity bound without a second (lo) product; the kernels multiply
+// dP^T by 2^-(e_dO + e_V) and dV by 2^-e_dO, exactly.
+__host__ __device__ __forceinline__ int f16_exp(unsigned amax_bits) {
+  const int ex = int((amax_bits >> 23) & 0xFFu);   // biased exponent of m (m >= 0)
+  if (ex == 255 || amax_bits == 0u) return 0;      // inf / NaN, or all zero: no scaling
+  if (ex == 0) return 60;                          // m below the normal range
+  const int k = ex - 126;                          // m = f * 2^k with f in [0.5, 1)
+  const int e = 15 - k;
+  return e < -60 ? -60 : (e > 60 ? 60 : e);
+}
+
+// Largest |x| over one thread's 8 bf16 elements.
+__device__ __forceinline__ float absmax8(uint4 v) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+  float m = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+  }
+  return m;
+}
+
+// Block-wide max of m (256 threads; NaN is ignored by fmaxf) merged into
+// *dst as float bits, which order like the values for m >= 0.
+__device__ __forceinline__ void block_max_to(float m, unsigned* dst) {
+  __shared__ float red[8];
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float r = red[0];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) r = fmaxf(r, red[i]);
+    if (r > 0.f) atomicMax(dst, __float_as_uint(r));
+  }
+  __syncthreads();
+}
+
+// Largest |V| of a [batch, heads, rows, D] view (element strides sv), into
+// amax[1]; the caller's block has already merged its |dO| maximum.
+template <int D>
+__device__ __forceinline__ void v_absmax(const __nv_bfloat16* __restrict__ v, Strides sv, int batch,
+                                         int heads, int rows, unsigned* amax) {
+  constexpr int PR = D / 8;                        // 8-element pieces per row
+  const long long n = (long long)batch * heads * rows * PR;
+  float m = 0.f;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long row = i / PR;
+    const int sb = int(i - row * PR);
+    const long long r = row % rows, bh = row / rows, hh = bh % heads, bb = bh / heads;
+    m = fmaxf(m, absmax8(*reinterpret_cast<const uint4*>(v + bb * sv.b + hh * sv.h + r * sv.n +
+                                                        sb * 8)));
+  }
+  block_max_to(m, amax + 1);
+}
+
+// dO16 = fp16(dO * 2^e_dO) and V16 = fp16(V * 2^e_V), contiguous
+// [batch * heads, rows, D] (packed batches: batch 1, rows = the total),
+// after the preprocess kernel has left the largest magnitudes in amax.
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_f16_kernel(
+    const __nv_bfloat16* __restrict__ dO, Strides sdo, int bq, int Hq, int rows_q,
+    const __nv_bfloat16* __restrict__ v, Strides sv, int bk, int Hkv, int rows_k,
+    __half* __restrict__ do16, __half* __restrict__ v16, const unsigned* __restrict__ amax) {
+  constexpr int PR = D / 8;
+  const float s_do = ldexpf(1.f, f16_exp(amax[0])), s_v = ldexpf(1.f, f16_exp(amax[1]));
+  const long long n_do = (long long)bq * Hq * rows_q * PR;
+  const long long n_all = n_do + (long long)bk * Hkv * rows_k * PR;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n_all;
+       i += (long long)gridDim.x * blockDim.x) {
+    const bool isv = i >= n_do;
+    const long long j = isv ? i - n_do : i;
+    const int heads = isv ? Hkv : Hq, rows = isv ? rows_k : rows_q;
+    const Strides st = isv ? sv : sdo;
+    const float sc = isv ? s_v : s_do;
+    const long long row = j / PR;
+    const int sb = int(j - row * PR);
+    const long long r = row % rows, bh = row / rows, hh = bh % heads, bb = bh / heads;
+    const uint4 x = *reinterpret_cast<const uint4*>((isv ? v : dO) + bb * st.b + hh * st.h +
+                                                    r * st.n + sb * 8);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&x);
+    uint4 y;
+    uint32_t* yw = reinterpret_cast<uint32_t*>(&y);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 f = __bfloat1622float2(h[k]);
+      yw[k] = pack_f16(f.x * sc, f.y * sc);
+    }
+    *reinterpret_cast<uint4*>((isv ? v16 : do16) + row * D + sb * 8) = y;
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(
     const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ ores,
     const __nv_bfloat16* __restrict__ dO,
     const float* __restrict__ lse, float* __restrict__ dqacc, float* __restrict__ Dpad,
     float* __restrict__ Lpad, int rows_bh, int Hq, int Nq, int Nq_pad, Strides so, Strides sdo,
-    float* __restrict__ kvacc, long long kv_n4) {
+    float* __restrict__ kvacc, long long kv_n4, const __nv_bfloat16* __restrict__ v, Strides sv,
+    int B, int Hkv, int Nk, unsigned* __restrict__ amax) {
   constexpr int TPR = D / 8;                       // threads per row
   constexpr int RPB = 256 / TPR;                   // rows per block pass
   const int sub = threadIdx.x % TPR;
   const int rlocal = threadIdx.x / TPR;
   const long long total = (long long)rows_bh * Nq_pad;
+  float mdo = 0.f;                                 // largest |dO| seen by this thread
   for (long long r = (long long)blockIdx.x * RPB + rlocal; r < total;
        r += (long long)gridDim.x * RPB) {
     const long long bh = r / Nq_pad;
@@ -188,6 +311,7 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(
         const float2 b = __bfloat1622float2(d2[i]);
         acc = fmaf(a.x + r.x, b.x, acc);
         acc = fmaf(a.y + r.y, b.y, acc);
+        mdo = fmaxf(mdo, fmaxf(fabsf(b.x), fabsf(b.y)));
       }
       float4* z = reinterpret_cast<float4*>(dqacc + e);
       z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -205,6 +329,10 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < kv_n4;
        i += (long long)gridDim.x * blockDim.x)
     reinterpret_cast<float4*>(kvacc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (amax) {                                      // the fp16 operand scales (bwd_f16)
+    block_max_to(mdo, amax);
+    v_absmax<D>(v, sv, B, Hkv, Nk, amax);
+  }
 }
 
 // The same for a packed variable-length batch: o and dO are [total_q, Hq, d]
@@ -219,7 +347,9 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_varlen_kernel(
     const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
     const float* __restrict__ lse, float* __restrict__ dqacc, float* __restrict__ Dpad,
     float* __restrict__ Lpad, const int* __restrict__ cu_q, int B, int Hq, int total_q,
-    long long ld, Strides so, Strides sdo, float* __restrict__ kvacc, long long kv_n4) {
+    long long ld, Strides so, Strides sdo, float* __restrict__ kvacc, long long kv_n4,
+    const __nv_bfloat16* __restrict__ v, Strides sv, int Hkv, int total_k,
+    unsigned* __restrict__ amax) {
   constexpr int TPR = D / 8;
   constexpr int RPB = 256 / TPR;
   const int sub = threadIdx.x % TPR;
@@ -229,6 +359,7 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_varlen_kernel(
   // shuffles with all lanes; rows past the end only do nothing.
   const long long total = (long long)Hq * total_q;
   const long long total_pad = (total + RPB - 1) / RPB * RPB;
+  float mdo = 0.f;                                 // largest |dO| seen by this thread
   for (long long r = (long long)blockIdx.x * RPB + rlocal; r < total_pad;
        r += (long long)gridDim.x * RPB) {
     const bool valid = r < total;
@@ -256,6 +387,7 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_varlen_kernel(
         const float2 b2 = __bfloat1622float2(d2[i]);
         acc = fmaf(a.x, b2.x, acc);
         acc = fmaf(a.y, b2.y, acc);
+        mdo = fmaxf(mdo, fmaxf(fabsf(b2.x), fabsf(b2.y)));
       }
       float4* z = reinterpret_cast<float4*>(dqacc + ((size_t)h * total_q + n) * D + sub * 8);
       z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -287,6 +419,10 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_varlen_kernel(
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < kv_n4;
        i += (long long)gridDim.x * blockDim.x)
     reinterpret_cast<float4*>(kvacc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (amax) {                                      // the fp16 operand scales (bwd_f16)
+    block_max_to(mdo, amax);
+    v_absmax<D>(v, sv, 1, Hkv, total_k, amax);
+  }
 }
 
 // dk, dv = bf16 of the fp32 partial-sum accumulators (dK already scaled).
@@ -348,7 +484,7 @@ struct BwdParams {
   const float* Dpad;
   const float* Lpad;
   float* dqacc;
-  int split_p;        // dV uses P as bf16 hi + lo (1) or bf16 P alone (0)
+  const unsigned* amax;  // workspace words: largest |dO|, |V| (their fp16 scales, f16_exp)
   int gsplit;         // CTAs sharing one kv group's query heads (1 = none)
   int hps;            // query heads per CTA: group / gsplit
   float* dkacc;       // fp32 dK / dV partial sums when gsplit > 1
@@ -387,7 +523,7 @@ __device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_
 
 // Block-sparse (SPARSE): a key block visits only the query blocks whose mask
 // entry for it is set, in the same cyclic order for every role.
-template <int D, bool CAUSAL, int MODE, bool SPLIT_DS>
+template <int D, bool CAUSAL, int MODE, bool SPLIT_DS, bool F16>
 __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
@@ -575,8 +711,12 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && n_steps > 0) {
-      constexpr uint32_t ID_S = idesc_bf16_f32(128, BR, 0, 0);    // S^T, dP^T: K-major both
-      constexpr uint32_t ID_KV = idesc_bf16_f32(128, DH, 0, 1);   // dV, dK: B MN-major
+      constexpr uint32_t ID_S = idesc_bf16_f32(128, BR, 0, 0);    // S^T: K-major both
+      constexpr uint32_t ID_DP = F16 ? idesc_f16_f32(128, BR, 0, 0)   // dP^T: fp16 V, dO
+                                        : idesc_bf16_f32(128, BR, 0, 0);
+      constexpr uint32_t ID_KV = idesc_bf16_f32(128, DH, 0, 1);   // dK: B MN-major
+      constexpr uint32_t ID_V = F16 ? idesc_f16_f32(128, DH, 0, 1)    // dV: fp16 P, dO
+                                       : idesc_bf16_f32(128, DH, 0, 1);
       constexpr uint32_t ID_DQ = idesc_bf16_f32(128, BR, 1, 1);   // dQ^T: A, B MN-major
       // Descriptor low words: K-major (S^T, dP^T operands) and MN-major (the
       // B operands of dV, dK and both operands of dQ^T).
@@ -590,18 +730,18 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
       // A-operand column (within a P^T / dS^T buffer) of k-step kk: compute
       // group kk/2 wrote queries [32(kk/2), +32) packed into its own columns.
       auto pcol = [](int kk) { return uint32_t((kk >> 1) * 32 + (kk & 1) * 8); };
-      auto mma_sdp = [&](uint32_t d_tm, uint32_t a_lo, uint32_t b_lo) {
+      auto mma_sdp = [&](uint32_t d_tm, uint32_t a_lo, uint32_t b_lo, uint32_t idesc) {
 #pragma unroll (D == 256 ? 4 : D / 16)
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ko = ((kk >> 2) * BC * 128 + (kk & 3) * 32) >> 4;
           const uint32_t qo = ((kk >> 2) * BR * 128 + (kk & 3) * 32) >> 4;
-          umma_ss_lo(d_tm, a_lo + ko, b_lo + qo, ID_S, kk > 0);
+          umma_ss_lo(d_tm, a_lo + ko, b_lo + qo, idesc, kk > 0);
         }
       };
       auto kst = [&](int t) { return kS0 + uint32_t(t % QS) * STG; };   // Q of step t, K-major
       auto mst = [&](int t) { return mS0 + uint32_t(t % QS) * STG; };   // Q of step t, MN-major
       // S^T of step t into buffer t mod 2
-      auto mma_s = [&](int t) { mma_sdp(tmem + C::TM_S + (t & 1) * BR, kK, kst(t)); };
+      auto mma_s = [&](int t) { mma_sdp(tmem + C::TM_S + (t & 1) * BR, kK, kst(t), ID_S); };
       // start of this CTA's share of d (DH columns, whole 64-column chunks) in
       // the MN-major operands
       const uint32_t dq_off = uint32_t((dcol0 / 64) * BR * 128) >> 4;
@@ -612,21 +752,20 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
       if (ok) {
         mma_s(0);
         umma_commit(bar_s + 0);
-        mma_sdp(tmem + C::TM_DP, kV, kst(0) + QT);
+        mma_sdp(tmem + C::TM_DP, kV, kst(0) + QT, ID_DP);
         umma_commit(bar_dp);
       }
       for (int t = 0; t < n_steps && ok; ++t) {
         const int st = t % QS;
         const uint32_t mQ = mst(t) + dq_off, mdO = mQ + QT;
         const uint32_t tS = tmem + C::TM_S + (t & 1) * BR;
-        // dV += P^T dO  (hi then lo half of P)
+        // dV += P^T dO  (fp16 P and dO)
         if (!(ok = mbar_wait(bar_p, t & 1, abort_flag, p.status, WB_P))) break;
         tc_fence_after();
-        for (int half = 0; half < 1 + p.split_p; ++half)
 #pragma unroll
-          for (int kk = 0; kk < BR / 16; ++kk)
-            umma_ts_lo(tmem + C::TM_DV, tS + pcol(kk) + half * 16, mdO + kk * 128, ID_KV,
-                       (t > 0 || kk > 0 || half > 0) ? 1u : 0u);
+        for (int kk = 0; kk < BR / 16; ++kk)
+          umma_ts_lo(tmem + C::TM_DV, tS + pcol(kk), mdO + kk * 128, ID_V,
+                     (t > 0 || kk > 0) ? 1u : 0u);
         // S^T of the next step into the other buffer.  With one Q/dO stage
         // the next Q only arrives after this step's dK releases the stage,
         // so S^T_{t+1} then waits until after dQ_t (below).
@@ -663,7 +802,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
         if (QS == 1 && !(ok = next_s())) break;
         // dP^T of the next step (overwrites dS^T_t, read by dK_t above)
         if (t + 1 < n_steps) {
-          mma_sdp(tmem + C::TM_DP, kV, kst(t + 1) + QT);
+          mma_sdp(tmem + C::TM_DP, kV, kst(t + 1) + QT, ID_DP);
           umma_commit(bar_dp);
         }
       }
@@ -731,6 +870,15 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
     const uint32_t tl = tmem + (uint32_t(w * 32) << 16);
     const int key = key0 + r;
     const float sl2 = p.scale_log2;
+    // F16: dP^T and dV come from fp16 operands scaled by powers of two
+    // (f16_exp): dP = dP^T * 2^-(e_dO + e_V), dV = acc * 2^-e_dO, exactly
+    int e_do = 0, e_v = 0;
+    if constexpr (F16) {
+      e_do = f16_exp(__ldg(p.amax));
+      e_v = f16_exp(__ldg(p.amax + 1));
+    }
+    const float inv_do = ldexpf(1.f, -e_do);
+    const float2 inv_vd2 = make_float2(ldexpf(1.f, -e_do - e_v), ldexpf(1.f, -e_do - e_v));
     bool ok = true;
 
     Seq sq;
@@ -759,10 +907,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
            mbar_wait(bar_s + (t & 1), (t >> 1) & 1, abort_flag, p.status, WB_S);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
-      // ---- P^T for this key row and the group's 32 queries: hi = bf16(P)
-      // over columns [0,16) of the group's S^T columns and, when split_p,
-      // lo = bf16(P - hi) over [16,32); dV then accumulates both, so rounding
-      // P to bf16 does not pile up over the query rows of a whole GQA group.
+      // ---- P^T for this key row and the group's 32 queries: fp16 P over
+      // columns [0,16) of the group's S^T columns, the A operand of dV (fp16
+      // rounding keeps dV within the bound over the query rows of a whole
+      // GQA group, where bf16 would not).
       float P[32];
       {
         uint32_t u[32];
@@ -784,21 +932,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) P[i] = (i < cstart) ? 0.f : P[i];
         }
-        uint32_t hi[16];
+        uint32_t ph[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) hi[i] = pack_bf16(P[2 * i], P[2 * i + 1]);
-        FA_TMEM_ST16(tS, hi);
-        if (p.split_p) {
-          uint32_t lo[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float2 rem = fadd2(make_float2(P[2 * i], P[2 * i + 1]),
-                                     make_float2(-__uint_as_float(hi[i] << 16),
-                                                 -__uint_as_float(hi[i] & 0xFFFF0000u)));
-            lo[i] = pack_bf16(rem.x, rem.y);
-          }
-          FA_TMEM_ST16(tS + 16, lo);
-        }
+        for (int i = 0; i < 16; ++i)
+          ph[i] = F16 ? pack_f16(P[2 * i], P[2 * i + 1]) : pack_bf16(P[2 * i], P[2 * i + 1]);
+        FA_TMEM_ST16(tS, ph);
         tmem_wait_st();
       }
       tc_fence_before();
@@ -819,9 +957,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
         uint32_t pk[16], lo[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float2 x = fadd2(make_float2(__uint_as_float(u[2 * i]),
-                                             __uint_as_float(u[2 * i + 1])),
-                                 make_float2(-dd[2 * i], -dd[2 * i + 1]));
+          // dP^T came from the scaled fp16 operands: dP = dP^T_scaled * 2^-(e_dO + e_V)
+          const float2 dp2 = make_float2(__uint_as_float(u[2 * i]), __uint_as_float(u[2 * i + 1]));
+          const float2 nd = make_float2(-dd[2 * i], -dd[2 * i + 1]);
+          const float2 x = F16 ? ffma2(dp2, inv_vd2, nd) : fadd2(dp2, nd);
           const float2 y = fmul2(make_float2(P[2 * i], P[2 * i + 1]), x);
           pk[i] = pack_bf16(y.x, y.y);
           if constexpr (SPLIT_DS)
@@ -859,7 +998,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
       // (all lanes load from TMEM together; rows past Nk add nothing).
       if (n_steps > 0) {
         const int tcol = g == 0 ? C::TM_DK : C::TM_DV;
-        const float mul = g == 0 ? p.scale : 1.f;
+        const float mul = g == 0 ? p.scale : inv_do;
         float* dst = (g == 0 ? p.dkacc : p.dvacc) +
                      (VARLEN ? size_t(hkv) * p.total_k + koff + key : size_t(bkv) * p.Nk + key) *
                          D + dcol0;
@@ -882,7 +1021,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
       }
     } else if (ok) {
       const int tcol = g == 0 ? C::TM_DK : C::TM_DV;
-      const float mul = g == 0 ? p.scale : 1.f;
+      const float mul = g == 0 ? p.scale : inv_do;
       uint8_t* stage = sStage + g * (BC * DH * 2);
       // Packed batches: a warp whose 32 key rows run past the sequence's
       // end stores its rows directly (a TMA box would reach the next one).
@@ -974,6 +1113,9 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
   float* Dpad = reinterpret_cast<float*>(ws + w.d_off);
   float* Lpad = reinterpret_cast<float*>(ws + w.l_off);
   float* kvacc = reinterpret_cast<float*>(ws + w.kv_off);
+  __half* do16 = reinterpret_cast<__half*>(ws + w.do16_off);
+  __half* v16 = reinterpret_cast<__half*>(ws + w.v16_off);
+  unsigned* amax = reinterpret_cast<unsigned*>(ws + w.amax_off);
   const int Nq_pad = round_up(Nq, 128);
   const int bhq = B * Hq;
   const int group = Hq / Hkv;
@@ -1002,10 +1144,16 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
   // general one with 64-query steps.
   constexpr bool STEP128 = D <= 128;
   constexpr int BRK = STEP128 ? 128 : C::BR;
+  // V and dO reach the main kernel as the preprocess stage's contiguous
+  // fp16 copies (TMA moves the 16-bit elements unchanged; the map's element
+  // type only matters for a NaN out-of-bounds fill, which is not used).
+  const bool f16 = bwd_f16(Hq, Hkv, D);
+  const Strides s_v16{(long long)Hkv * rows_k * D, (long long)rows_k * D, D};
+  const Strides s_do16{(long long)Hq * rows_q * D, (long long)rows_q * D, D};
   if ((stages & 2) && (!make_map_bf16(&mq, q, D, rows_q, Hq, map_b, st[0], BRK) ||
       !make_map_bf16(&mk, k, D, rows_k, Hkv, map_b, st[1], C::BC) ||
-      !make_map_bf16(&mv, v, D, rows_k, Hkv, map_b, st[2], C::BC) ||
-      !make_map_bf16(&mdo, dO, D, rows_q, Hq, map_b, st[4], BRK) ||
+      !make_map_bf16(&mv, f16 ? v16 : v, D, rows_k, Hkv, map_b, f16 ? s_v16 : st[2], C::BC) ||
+      !make_map_bf16(&mdo, f16 ? do16 : dO, D, rows_q, Hq, map_b, f16 ? s_do16 : st[4], BRK) ||
       !make_map_bf16(&mdk, dk, D, rows_k, Hkv, map_b, st[6], 32) ||
       !make_map_bf16(&mdv, dv, D, rows_k, Hkv, map_b, st[7], 32)))
     return 5;
@@ -1013,6 +1161,7 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
 
   if (stages & 1) {
     constexpr int RPB = 256 / (D / 8);
+    if (f16 && cudaMemsetAsync(amax, 0, 2 * sizeof(unsigned), stream) != cudaSuccess) return 5;
     if (vl) {
       const long long rows = (long long)Hq * vl->total_q;
       const long long blocks = std::max<long long>(
@@ -1020,14 +1169,25 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
       fa_bwd_pre_varlen_kernel<D><<<unsigned(blocks), 256, 0, stream>>>(
           static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, dqacc,
           Dpad, Lpad, vl->cu_q, B, Hq, vl->total_q, varlen_lpad_ld(B, vl->total_q), st[3], st[4],
-          kvacc, kv_n4);
+          kvacc, kv_n4, static_cast<const __nv_bfloat16*>(v), st[2], Hkv, vl->total_k,
+          f16 ? amax : nullptr);
     } else {
       const long long rows = (long long)bhq * Nq_pad;
       const long long blocks = std::min<long long>((rows + RPB - 1) / RPB, 148LL * 16);
       fa_bwd_pre_kernel<D><<<unsigned(blocks), 256, 0, stream>>>(
           static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(ores),
           static_cast<const __nv_bfloat16*>(dO), lse, dqacc,
-          Dpad, Lpad, bhq, Hq, Nq, Nq_pad, st[3], st[4], kvacc, kv_n4);
+          Dpad, Lpad, bhq, Hq, Nq, Nq_pad, st[3], st[4], kvacc, kv_n4,
+          static_cast<const __nv_bfloat16*>(v), st[2], B, Hkv, Nk, f16 ? amax : nullptr);
+    }
+    if (f16) {
+      const long long pieces = ((long long)map_b * Hq * rows_q + (long long)map_b * Hkv * rows_k) *
+                               (D / 8);
+      const long long blocks = std::max<long long>(1, std::min<long long>((pieces + 255) / 256,
+                                                                          148LL * 16));
+      fa_bwd_f16_kernel<D><<<unsigned(blocks), 256, 0, stream>>>(
+          static_cast<const __nv_bfloat16*>(dO), st[4], map_b, Hq, rows_q,
+          static_cast<const __nv_bfloat16*>(v), st[2], map_b, Hkv, rows_k, do16, v16, amax);
     }
     if (cudaGetLastError() != cudaSuccess) return 5;
   }
@@ -1037,18 +1197,23 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
     // rounding dS to bf16 alone moves dK by about 2e-2 (causal, N = 4096),
     // so dS also goes in as hi + lo there (exact_dk).
     const bool split_ds = exact_dk(group, D);
-    auto pick = [&](auto split_tag) {
-      constexpr bool S = decltype(split_tag)::value;
+    // instances: (fp16 dP / dV, dS split) = (no, no) for MHA at d <= 128,
+    // (yes, exact_dk) otherwise; d = 256 is always fp16 (bwd_f16)
+    auto pick = [&](auto split_tag, auto f16_tag) {
+      constexpr bool S = decltype(split_tag)::value, F = decltype(f16_tag)::value;
       if constexpr (STEP128)
-        return vl ? fa_bwd_main128_kernel<D, CAUSAL, BMODE_VARLEN, S>
-               : mask ? fa_bwd_main128_kernel<D, CAUSAL, BMODE_SPARSE, S>
-                      : fa_bwd_main128_kernel<D, CAUSAL, BMODE_DENSE, S>;
+        return vl ? fa_bwd_main128_kernel<D, CAUSAL, BMODE_VARLEN, S, F>
+               : mask ? fa_bwd_main128_kernel<D, CAUSAL, BMODE_SPARSE, S, F>
+                      : fa_bwd_main128_kernel<D, CAUSAL, BMODE_DENSE, S, F>;
       else
-        return vl ? fa_bwd_main_kernel<D, CAUSAL, BMODE_VARLEN, S>
-               : mask ? fa_bwd_main_kernel<D, CAUSAL, BMODE_SPARSE, S>
-                      : fa_bwd_main_kernel<D, CAUSAL, BMODE_DENSE, S>;
+        return static_cast<void>(F),   // d = 256 always takes fp16 operands
+               vl ? fa_bwd_main_kernel<D, CAUSAL, BMODE_VARLEN, S, true>
+               : mask ? fa_bwd_main_kernel<D, CAUSAL, BMODE_SPARSE, S, true>
+                      : fa_bwd_main_kernel<D, CAUSAL, BMODE_DENSE, S, true>;
     };
-    auto kern = split_ds ? pick(std::true_type{}) : pick(std::false_type{});
+    auto kern = !f16    ? pick(std::false_type{}, std::false_type{})
+                : split_ds ? pick(std::true_type{}, std::true_type{})
+                           : pick(std::false_type{}, std::true_type{});
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C2::SMEM_BYTES) !=
         cudaSuccess)
       return 5;
@@ -1061,11 +1226,7 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
     p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Nq = Nq; p.Nk = Nk; p.Nq_pad = Nq_pad;
     p.group = group;
     p.n_kblocks = n_kblocks;
-    // dV's rounding error from a bf16 P grows with the number of query rows
-    // that weigh heavily on one key: with a GQA group it is multiplied by the
-    // group size, and at d = 256 |dV| is large enough that the output
-    // rounding leaves no room.  There P goes in as hi + lo (one more MMA).
-    p.split_p = (group > 1 || D == 256) ? 1 : 0;
+    p.amax = f16 ? amax : nullptr;
     p.gsplit = gsplit;
     p.hps = group / gsplit;
     p.dkacc = kvacc;

@@ -67,7 +67,7 @@ struct Bwd128Cfg {
   static_assert(QS * STAGE_BYTES >= 2 * BC * DH * 2, "dK/dV staging fits in the Q/dO stages");
 };
 
-template <int D, bool CAUSAL, int MODE, bool SPLIT_DS>
+template <int D, bool CAUSAL, int MODE, bool SPLIT_DS, bool F16>
 __global__ void __launch_bounds__(Bwd128Cfg<D>::NTHREADS, 1)
     fa_bwd_main128_kernel(const __grid_constant__ CUtensorMap tmQ,
                           const __grid_constant__ CUtensorMap tmK,
@@ -238,8 +238,12 @@ __global__ void __launch_bounds__(Bwd128Cfg<D>::NTHREADS, 1)
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && n_steps > 0) {
-      constexpr uint32_t ID_S = idesc_bf16_f32(128, BR, 0, 0);    // S^T, dP^T: K-major both
-      constexpr uint32_t ID_KV = idesc_bf16_f32(128, DH, 0, 1);   // dV, dK: B MN-major
+      constexpr uint32_t ID_S = idesc_bf16_f32(128, BR, 0, 0);    // S^T: K-major both
+      constexpr uint32_t ID_DP = F16 ? idesc_f16_f32(128, BR, 0, 0)   // dP^T: fp16 V, dO
+                                        : idesc_bf16_f32(128, BR, 0, 0);
+      constexpr uint32_t ID_KV = idesc_bf16_f32(128, DH, 0, 1);   // dK: B MN-major
+      constexpr uint32_t ID_V = F16 ? idesc_f16_f32(128, DH, 0, 1)    // dV: fp16 P, dO
+                                       : idesc_bf16_f32(128, DH, 0, 1);
       constexpr uint32_t ID_DQ = idesc_bf16_f32(128, BR, 1, 1);   // dQ^T: A, B MN-major
       // Descriptor low words: K-major (S^T, dP^T operands) and MN-major (the
       // B operands of dV, dK and both operands of dQ^T).
@@ -252,45 +256,45 @@ __global__ void __launch_bounds__(Bwd128Cfg<D>::NTHREADS, 1)
       constexpr uint32_t STG = C::STAGE_BYTES >> 4, QT = C::QT_BYTES >> 4;
       // A-operand column of k-step kk (16 queries) within a P^T / dS^T
       // region: each 32-query chunk (32 columns of S^T / dP^T) holds its
-      // queries' bf16 pairs in its first 16 columns (P lo in the next 16).
+      // queries' fp16 P / bf16 dS pairs in its first 16 columns (dS lo in
+      // the next 16).
       auto pcol = [](int kk) { return uint32_t((kk >> 1) * 32 + (kk & 1) * 8); };
       auto kst = [&](int t) { return kS0 + uint32_t(t % QS) * STG; };   // Q of step t, K-major
       auto mst = [&](int t) { return mS0 + uint32_t(t % QS) * STG; };   // Q of step t, MN-major
-      auto mma_kq = [&](uint32_t d_tm, uint32_t a_lo, uint32_t b_lo) {
+      auto mma_kq = [&](uint32_t d_tm, uint32_t a_lo, uint32_t b_lo, uint32_t idesc) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ko = ((kk >> 2) * BC * 128 + (kk & 3) * 32) >> 4;
           const uint32_t qo = ((kk >> 2) * BR * 128 + (kk & 3) * 32) >> 4;
-          umma_ss_lo(d_tm, a_lo + ko, b_lo + qo, ID_S, kk > 0);
+          umma_ss_lo(d_tm, a_lo + ko, b_lo + qo, idesc, kk > 0);
         }
       };
       bool ok = mbar_wait(bar_kv, 0, abort_flag, p.status, WB_KV) &&
                 mbar_wait(bar_qfull + 0, 0, abort_flag, p.status, WB_QFULL);
       tc_fence_after();
       if (ok) {
-        mma_kq(tmem + C::TM_SP, kK, kst(0));
+        mma_kq(tmem + C::TM_SP, kK, kst(0), ID_S);
         umma_commit(bar_s);
-        mma_kq(tmem + C::TM_DP, kV, kst(0) + QT);
+        mma_kq(tmem + C::TM_DP, kV, kst(0) + QT, ID_DP);
         umma_commit(bar_dp);
       }
       for (int t = 0; t < n_steps && ok; ++t) {
         const int st = t % QS;
         const uint32_t mQ = mst(t), mdO = mQ + QT;
-        // dV += P^T dO  (hi, then lo when the precision rule asks for it)
+        // dV += P^T dO  (fp16 P and dO)
         if (!(ok = mbar_wait(bar_p, t & 1, abort_flag, p.status, WB_P))) break;
         tc_fence_after();
-        for (int half = 0; half < 1 + p.split_p; ++half)
 #pragma unroll
-          for (int kk = 0; kk < BR / 16; ++kk)
-            umma_ts_lo(tmem + C::TM_DV, tmem + C::TM_SP + pcol(kk) + half * 16, mdO + kk * 128,
-                       ID_KV, (t > 0 || kk > 0 || half > 0) ? 1u : 0u);
+        for (int kk = 0; kk < BR / 16; ++kk)
+          umma_ts_lo(tmem + C::TM_DV, tmem + C::TM_SP + pcol(kk), mdO + kk * 128, ID_V,
+                     (t > 0 || kk > 0) ? 1u : 0u);
         // S^T of the next step (SP is free once dV_t has read P_t)
         if (t + 1 < n_steps) {
           if (!(ok = mbar_wait(bar_qfull + (t + 1) % QS, ((t + 1) / QS) & 1, abort_flag,
                                p.status, WB_QFULL)))
             break;
           tc_fence_after();
-          mma_kq(tmem + C::TM_SP, kK, kst(t + 1));
+          mma_kq(tmem + C::TM_SP, kK, kst(t + 1), ID_S);
           umma_commit(bar_s);
         }
         // dK += dS^T Q
@@ -323,7 +327,7 @@ __global__ void __launch_bounds__(Bwd128Cfg<D>::NTHREADS, 1)
             if (!(ok = mbar_wait(bar_dqempty, t & 1, abort_flag, p.status, WB_DQEMPTY))) break;
             tc_fence_after();
           }
-          mma_kq(tmem + C::TM_DP, kV, kst(t + 1) + QT);
+          mma_kq(tmem + C::TM_DP, kV, kst(t + 1) + QT, ID_DP);
           umma_commit(bar_dp);
         }
       }
@@ -383,6 +387,15 @@ __global__ void __launch_bounds__(Bwd128Cfg<D>::NTHREADS, 1)
     const uint32_t tl = tmem + (uint32_t(w * 32) << 16);
     const int key = key0 + r;
     const float sl2 = p.scale_log2;
+    // F16: dP^T and dV come from fp16 operands scaled by powers of two
+    // (f16_exp): dP = dP^T * 2^-(e_dO + e_V), dV = acc * 2^-e_dO, exactly
+    int e_do = 0, e_v = 0;
+    if constexpr (F16) {
+      e_do = f16_exp(__ldg(p.amax));
+      e_v = f16_exp(__ldg(p.amax + 1));
+    }
+    const float inv_do = ldexpf(1.f, -e_do);
+    const float2 inv_vd2 = make_float2(ldexpf(1.f, -e_do - e_v), ldexpf(1.f, -e_do - e_v));
     bool ok = true;
     Seq sq;
     if constexpr (SPARSE) seq_begin(sq);
@@ -395,13 +408,13 @@ __global__ void __launch_bounds__(Bwd128Cfg<D>::NTHREADS, 1)
       const uint32_t tSP = tl + C::TM_SP + g * 64;
       const uint32_t tDP = tl + C::TM_DP + g * 64;
       // ---- P^T for this key row and the group's 64 queries, 32 at a time:
-      // hi = bf16(P) over the chunk's first 16 S^T columns and lo =
-      // bf16(P - hi) over the next 16 (each chunk is read before written).
+      // fp16(P) over the chunk's first 16 S^T columns (each chunk is read
+      // before written): the A operand of dV, whose fp16 rounding keeps dV
+      // within the bound over the query rows of a whole GQA group.
       ok = mbar_wait(bar_s, t & 1, abort_flag, p.status, WB_S);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
       float pf[64];                                 // P (fp32), kept for dS
-      const bool split = p.split_p != 0;
       const float2 sl22 = make_float2(sl2, sl2);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
@@ -427,27 +440,19 @@ __global__ void __launch_bounds__(Bwd128Cfg<D>::NTHREADS, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) pf[c * 32 + i + e] = pv[e];
         }
-        uint32_t hi[16];
+        uint32_t ph[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) hi[i] = pack_bf16(pf[c * 32 + 2 * i], pf[c * 32 + 2 * i + 1]);
-        FA_TMEM_ST16(tSP + c * 32, hi);
-        if (split) {                                 // lo = P - hi, for dV of GQA/MQA groups
-          uint32_t lo[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float2 rem = fadd2(make_float2(pf[c * 32 + 2 * i], pf[c * 32 + 2 * i + 1]),
-                                     make_float2(-__uint_as_float(hi[i] << 16),
-                                                 -__uint_as_float(hi[i] & 0xFFFF0000u)));
-            lo[i] = pack_bf16(rem.x, rem.y);
-          }
-          FA_TMEM_ST16(tSP + c * 32 + 16, lo);
-        }
+        for (int i = 0; i < 16; ++i)
+          ph[i] = F16 ? pack_f16(pf[c * 32 + 2 * i], pf[c * 32 + 2 * i + 1])
+                      : pack_bf16(pf[c * 32 + 2 * i], pf[c * 32 + 2 * i + 1]);
+        FA_TMEM_ST16(tSP + c * 32, ph);
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar_p);
 
-      // ---- dS^T = P^T o (dP^T - D), 16 columns at a time; P = hi + lo.
+      // ---- dS^T = P^T o (dP - D), 16 columns at a time (dP unscaled from
+      // the fp16 product).
       ok = mbar_wait(bar_dp, t & 1, abort_flag, p.status, WB_DP);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
@@ -468,9 +473,10 @@ __global__ void __launch_bounds__(Bwd128Cfg<D>::NTHREADS, 1)
             for (int e = 0; e < 2; ++e) {
               const float2 pp =
                   make_float2(pf[c * 16 + 2 * (i + e)], pf[c * 16 + 2 * (i + e) + 1]);
-              const float2 x = fadd2(make_float2(__uint_as_float(dpv[2 * (i + e)]),
-                                                 __uint_as_float(dpv[2 * (i + e) + 1])),
-                                     make_float2(-dsub[2 * e], -dsub[2 * e + 1]));
+              const float2 dp2 = make_float2(__uint_as_float(dpv[2 * (i + e)]),
+                                             __uint_as_float(dpv[2 * (i + e) + 1]));
+              const float2 nd = make_float2(-dsub[2 * e], -dsub[2 * e + 1]);
+              const float2 x = F16 ? ffma2(dp2, inv_vd2, nd) : fadd2(dp2, nd);
               const float2 y = fmul2(pp, x);
               pk[i + e] = pack_bf16(y.x, y.y);
               if constexpr (SPLIT)
@@ -517,7 +523,7 @@ __global__ void __launch_bounds__(Bwd128Cfg<D>::NTHREADS, 1)
     if (ok && p.gsplit > 1) {
       if (n_steps > 0) {
         const int tcol = g == 0 ? C::TM_DK : C::TM_DV;
-        const float mul = g == 0 ? p.scale : 1.f;
+        const float mul = g == 0 ? p.scale : inv_do;
         float* dst = (g == 0 ? p.dkacc : p.dvacc) +
                      (VARLEN ? size_t(hkv) * p.total_k + koff + key : size_t(bkv) * p.Nk + key) *
                          D;
@@ -540,7 +546,7 @@ __global__ void __launch_bounds__(Bwd128Cfg<D>::NTHREADS, 1)
       }
     } else if (ok) {
       const int tcol = g == 0 ? C::TM_DK : C::TM_DV;
-      const float mul = g == 0 ? p.scale : 1.f;
+      const float mul = g == 0 ? p.scale : inv_do;
       uint8_t* stage = sStage + g * (BC * DH * 2);
       const bool direct = VARLEN && (key0 + w * 32 + 32 > nk);
 #pragma unroll

@@ -5,6 +5,7 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #ifndef FA_WAIT_LIMIT_NS
 // A single wait longer than this means the pipeline is broken; the kernel then
@@ -260,6 +261,12 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, in
          | (uint32_t(M >> 4) << 24);    // M / 16
 }
 
+// The same for fp16 A and B (format field 0); A and B of one product always
+// have the same type.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, int a_mn, int b_mn) {
+  return idesc_bf16_f32(M, N, a_mn, b_mn) & ~((7u << 7) | (7u << 10));
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version bits.
 // lbo/sbo in bytes.
 __host__ __device__ __forceinline__ constexpr uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo,
@@ -418,6 +425,10 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
 }
 

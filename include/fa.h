@@ -88,7 +88,9 @@ int fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* 
 /*
  * Bytes of caller-owned device workspace fa_bwd needs for these sizes: the
  * fp32 dQ accumulator [B, Hq, Nq, d] and two fp32 row vectors (D =
- * rowsum(dO * O) and LSE * log2 e) padded to 128 rows per head.
+ * rowsum(dO * O) and LSE * log2 e) padded to 128 rows per head; for GQA /
+ * MQA groups also fp32 dK / dV partial sums [B, Hkv, Nk, d], and for GQA /
+ * MQA groups and d = 256 fp16 copies of dO and V (see fa_bwd).
  * Returns 0 for invalid sizes.
  */
 size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal);
@@ -105,6 +107,13 @@ size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int 
  * from the fp32 output with one more forward pass (about the forward's
  * time).  fa_fwd_residual / fa_bwd_residual give the same precision
  * without it.
+ * GQA / MQA groups and d = 256: dV = P^T dO and dP = dO V^T take fp16
+ * operands (P rounded to fp16, 8x finer than bf16, which dV sums over every
+ * query row of the group).  The preprocess copies dO and V into the
+ * workspace as fp16, each scaled by one power of two chosen from its
+ * largest magnitude, so the copy is exact for every element within a factor
+ * 2^24 of that magnitude; smaller elements keep an absolute error below
+ * 2^-25 of it.  Non-finite dO or V give non-finite results, as in bf16.
  */
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
            const void* dO, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nk,
@@ -225,7 +234,8 @@ int fa_bwd_residual(const void* q, const void* k, const void* v, const void* o,
 typedef enum {
   FA_BWD_ALL = 0,   /* the whole backward pass (same as fa_bwd) */
   FA_BWD_PRE = 1,   /* D = rowsum(dO * O), LSE copy, dQ accumulator := 0 (in the workspace);
-                       for wide groups also the forward pass that recomputes D (see fa_bwd) */
+                       GQA / MQA and d = 256: the fp16 copies of dO and V; wide groups:
+                       the forward pass that recomputes D (see fa_bwd) */
   FA_BWD_MAIN = 2,  /* dK, dV written; dQ accumulated into the workspace */
   FA_BWD_DQ = 3     /* dq = scale * dQ accumulator, as bf16 */
 } fa_bwd_stage_t;

@@ -122,11 +122,13 @@ def test_launches_per_step():
     from exact_io_aware_71_b200.inputs import workloads
     w = workloads()
     assert bench.launches_per_step(w["train_b8h16n2048d128_full"], 148) == 4
-    # 32 query heads on one kv head, 128 key blocks: split, plus the dK/dV
-    # convert, plus the forward pass that recomputes D for the wide group
-    assert bench.launches_per_step(w["long_gqa_hkv1_n16384_d128_causal"], 148) == 6
-    # 8 kv heads x 128 key blocks = 1024 CTAs: no split
-    assert bench.launches_per_step(w["long_gqa_hkv8_n16384_d128_causal"], 148) == 4
+    # d = 256: the fp16 copy of dO and V
+    assert bench.launches_per_step(w["large_b4h8n4096d256_full"], 148) == 5
+    # 32 query heads on one kv head, 128 key blocks: the fp16 copy, the split
+    # and its dK/dV convert, and the forward pass that recomputes D
+    assert bench.launches_per_step(w["long_gqa_hkv1_n16384_d128_causal"], 148) == 7
+    # 8 kv heads x 128 key blocks = 1024 CTAs: no split; the fp16 copy
+    assert bench.launches_per_step(w["long_gqa_hkv8_n16384_d128_causal"], 148) == 5
 
 
 def test_roofline_picks_the_bound_by_arithmetic_intensity():

@@ -1,5 +1,5 @@
-"""An exact-arithmetic model of the backward pass's bf16 rounding points, and
-what it says about dK for wide GQA / MQA groups.  CPU only.
+"""An exact-arithmetic model of the backward pass's rounding points, and what
+it says about dK and dV for wide GQA / MQA groups.  CPU only.
 
 dK_j = scale * sum_h sum_i dS_ij q_i sums over every query row of every
 query head that shares the kv head, so per-element rounding that is harmless
@@ -127,3 +127,55 @@ def test_peaky_stress_input_misses_the_bar():
     hold dK to the Frobenius bar there."""
     r = run(2, 2, 512, 64, True, seed=9, qmul=4.0)
     assert r["plain"] > 0 and r["split_only"] > 0 and r["recompute"] < 0
+
+
+# ---- dV: P rounded to bf16, to bf16 hi + lo, or to fp16 ----------------------
+# dV_j = sum_h sum_i P_ij dO_i also sums over every query row of every query
+# head of the group.  The kernels give dV (and dP) fp16 operands for GQA / MQA
+# groups and d = 256: dO and V exactly (scaled by a power of two), P rounded
+# to fp16.  The model below compares that with bf16 P and with the bf16
+# hi + lo split it replaces, per element against the parity bound.
+
+def model_dv(q, k, v, do, causal, scale):
+    """dV of kv head 0 (stored as bf16) under the three P roundings."""
+    g, n, d = q.shape
+    mask = np.arange(n)[None, :] > np.arange(n)[:, None]
+    acc = {s: np.zeros((n, d)) for s in ("bf16", "hilo", "f16")}
+    for h in range(g):
+        s = scale * (q[h] @ k.T)
+        if causal:
+            s = np.where(mask, -np.inf, s)
+        e = np.exp(s - s.max(axis=1, keepdims=True))
+        p = e / e.sum(axis=1, keepdims=True)
+        hb = bf(p)
+        acc["bf16"] += hb.T @ do[h]
+        acc["hilo"] += (hb + bf(p - hb)).T @ do[h]
+        acc["f16"] += f16(p).T @ do[h]
+    return {sch: bf(a) for sch, a in acc.items()}
+
+
+def f16(x):
+    """Round fp64 values to fp16 (round to nearest even), back to fp64."""
+    return torch.from_numpy(np.ascontiguousarray(x)).to(torch.float16).to(torch.float64).numpy()
+
+
+def run_dv(Hq, Hkv, N, d, causal, seed):
+    wl = Workload("model", 1, Hq, Hkv, N, N, d, causal, seed)
+    q, k, v, do = (to64(t) for t in make_inputs(wl))
+    g = Hq // Hkv
+    ref = oracle.attention_backward(q, k, v, do, causal, wl.scale, heads=[(0, 0)])[2][0, 0]
+    got = model_dv(q[0, :g], k[0, 0], v[0, 0], do[0, :g], causal, wl.scale)
+    return {sch: excess(x, ref) for sch, x in got.items()}
+
+
+@pytest.mark.parametrize("Hq,Hkv,N,d,seed", [(32, 1, 1024, 128, 3), (4, 1, 1024, 256, 6)],
+                         ids=["mqa_d128", "gqa4_d256"])
+def test_dv_fp16_p_meets_the_bar_where_bf16_p_does_not(Hq, Hkv, N, d, seed):
+    """Causal, 32 query heads on one kv head at d = 128, and 4 on one at
+    d = 256: bf16 P leaves dV above the per-element bound, while fp16 P
+    stays within it with about the margin of the hi + lo split (the
+    excesses printed by the model: bf16 +1.4e-2 / +1.5e-3, hi + lo
+    -4.4e-3 / -4.6e-3, fp16 -3.9e-3 / -4.1e-3)."""
+    r = run_dv(Hq, Hkv, N, d, True, seed)
+    assert r["bf16"] > 0
+    assert r["f16"] < -2e-3 and r["hilo"] < -2e-3
