@@ -131,12 +131,19 @@ def summarise_clock_samples(samples, t0: float, t1: float, max_mhz):
     (host perf_counter seconds).  samples: (t, sm_mhz, power_w, reason_bits).
     A reason counts if any window sample has it."""
     win = [x for x in samples if t0 <= x[0] <= t1]
+    source = "nvml, 5 ms polling inside the timed region"
+    if not win:
+        # a region shorter than the polling interval: the sample nearest to it,
+        # if one was taken within 10 ms
+        near = sorted(samples, key=lambda x: max(t0 - x[0], x[0] - t1))[:1]
+        win = [x for x in near if max(t0 - x[0], x[0] - t1) <= 0.010]
+        source = "nvml, nearest sample to a timed region shorter than the 5 ms polling"
     if not win:
         return {"sm_mhz": None, "sm_max_mhz": max_mhz, "reasons": ["no samples"]}
     reasons = sorted(n for n, bit in NVML_REASON_BITS.items() if any(x[3] & bit for x in win))
     return {"sm_mhz": statistics.median(x[1] for x in win), "sm_max_mhz": max_mhz,
             "reasons": reasons, "samples": len(win), "power_w_max": max(x[2] for x in win),
-            "source": "nvml, 5 ms polling inside the timed region"}
+            "source": source}
 
 
 class ClockSampler:

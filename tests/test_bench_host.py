@@ -73,6 +73,9 @@ def test_nvml_samples_outside_the_timed_window_are_dropped():
     assert c["samples"] == 3 and c["sm_mhz"] == 1820.0 and c["sm_max_mhz"] == 1965.0
     assert c["reasons"] == ["sw_power_cap"] and c["power_w_max"] == 980.0
     assert bench.summarise_clock_samples(samples, 3.0, 4.0, 1965.0)["reasons"] == ["no samples"]
+    # a region shorter than the polling interval takes the nearest sample (within 10 ms)
+    c = bench.summarise_clock_samples(samples, 1.203, 1.204, 1965.0)
+    assert c["samples"] == 1 and c["sm_mhz"] == 1850.0 and "nearest" in c["source"]
 
 
 def test_traffic_is_reported_only_for_current_sources(tmp_path, monkeypatch):
