@@ -270,8 +270,9 @@ def launches_per_step(wl, sms: int) -> int:
     dP and dV take fp16 operands (GQA / MQA groups and d = 256, the library's
     rule); the dK/dV convert kernel when a GQA group's query heads are split
     over CTAs (the library splits when one CTA per (batch, kv head, key
-    block) would give fewer than two CTAs per SM); and the D-recomputing
-    forward pass for groups of 16 or more (any GQA group at d = 256)."""
+    block) would give fewer than two CTAs per SM); and for groups of 16 or
+    more (any GQA group at d = 256) the fp16 copy of Q and K and the
+    D-recomputing forward pass."""
     g = wl.Hq // wl.Hkv
     f16 = g > 1 or wl.d == 256
     if g == 1:
@@ -279,7 +280,8 @@ def launches_per_step(wl, sms: int) -> int:
     base = ((wl.Nk + 127) // 128) * wl.B * wl.Hkv * (2 if wl.d == 256 else 1)
     gsplit = next((s_ for s_ in range(1, g + 1) if g % s_ == 0 and base * s_ >= 2 * sms), g)
     exact = g >= EXACT_GROUP or (wl.d == 256 and g > 1)
-    return 4 + 1 + (1 if gsplit > 1 else 0) + (1 if exact else 0)
+    # exact: also the fp16 copy of Q and K, and the D-recomputing forward pass
+    return 4 + 1 + (1 if gsplit > 1 else 0) + (2 if exact else 0)
 
 
 def algorithmic_bytes(wl, frac: float = 1.0):

@@ -18,7 +18,8 @@
 //                     dV_j += P^T dO_i           (P^T from TMEM; fp16 P and dO for GQA, d=256)
 //                     dP^T = V_j dO_i^T          (fp16 V and dO with them)
 //                     dS^T = P^T o (dP^T - D_i)
-//                     dK_j += dS^T Q_i           (dS^T read from TMEM)
+//                     dK_j += dS^T Q_i           (dS^T read from TMEM; fp16 dS and Q, and
+//                                                 fp16 S^T and dQ^T, for wide groups)
 //                     dQ_i^T = K_j^T dS^T  -> fp32 reduce-add into dQacc
 //                   then dK_j * scale and dV_j are written as bf16
 //   fa_bwd_dq       dq = bf16(scale * dQacc)              (HBM-bound)
@@ -79,10 +80,11 @@ struct BwdCfg {
 
 inline int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
-// Groups whose dK the backward computes from dS as bf16 hi + lo and from an
-// exact D (the forward's residual output, or D recomputed by a forward pass
-// with the D epilogue): the errors of a bf16 dS and of D from the bf16 O add
-// up over every query row of the group.  From 16 query heads per kv head
+// Groups whose dK the backward computes from dS rounded to fp16 (every
+// product then takes fp16 operands: op_scales) and from an exact D (the
+// forward's residual output, or D recomputed by a forward pass with the D
+// epilogue): the errors of a bf16 dS and of D from the bf16 O add up over
+// every query row of the group.  From 16 query heads per kv head
 // on at d <= 128; at d = 256, whose dK carries more of that error (measured
 // 2.1e-2 on a packed batch with 4 query heads per kv head), for every GQA /
 // MQA group.
@@ -100,16 +102,23 @@ inline bool bwd_f16(int Hq, int Hkv, int d) { return Hq > Hkv || d == 256; }
 // Lpad fp32 [B*Hq, Nq_pad] | (GQA/MQA only) dKacc, dVacc fp32 [B*Hkv, Nk, d]
 // for the partial sums of a kv group split across CTAs | (bwd_f16 only)
 // dO16 fp16 [B*Hq, Nq, d] and V16 fp16 [B*Hkv, Nk, d]: dO and V scaled by
-// powers of two (the operands of the dP^T and dV products) | amax: two
-// words, the largest |dO| and |V| (float bits) that choose those powers.
+// powers of two (the operands of the dP^T and dV products) | (exact_dk
+// only) Q16, K16 likewise | amax: four words, the largest |dO|, |V|, |Q|,
+// |K| (float bits) that choose those powers.
 struct BwdWorkspace {
-  size_t dq_off, d_off, l_off, kv_off, kv_elems, do16_off, v16_off, amax_off, total;
+  size_t dq_off, d_off, l_off, kv_off, kv_elems, do16_off, v16_off, q16_off, k16_off, amax_off,
+      total;
 };
-inline void bwd_workspace_tail(BwdWorkspace& w, size_t do_elems, size_t v_elems) {
+// The fp16 copies: dO and V (bwd_f16), and Q and K as well (exact_dk, where
+// dS and every product that reads it are fp16 too); sizes in elements.
+inline void bwd_workspace_tail(BwdWorkspace& w, size_t do_elems, size_t v_elems, size_t q_elems,
+                               size_t k_elems) {
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   w.do16_off = w.kv_off + up(2 * w.kv_elems * 4);
   w.v16_off = w.do16_off + up(do_elems * 2);
-  w.amax_off = w.v16_off + up(v_elems * 2);
+  w.q16_off = w.v16_off + up(v_elems * 2);
+  w.k16_off = w.q16_off + up(q_elems * 2);
+  w.amax_off = w.k16_off + up(k_elems * 2);
   w.total = w.amax_off + 256;
 }
 inline BwdWorkspace bwd_workspace_layout(int B, int Hq, int Hkv, int Nq, int Nk, int d) {
@@ -122,8 +131,9 @@ inline BwdWorkspace bwd_workspace_layout(int B, int Hq, int Hkv, int Nq, int Nk,
   w.l_off = w.d_off + up(bh * nq_pad * 4);
   w.kv_off = w.l_off + up(bh * nq_pad * 4);
   w.kv_elems = (Hq > Hkv) ? size_t(B) * Hkv * Nk * d : 0;   // per tensor
-  const bool f16 = bwd_f16(Hq, Hkv, d);
-  bwd_workspace_tail(w, f16 ? bh * Nq * d : 0, f16 ? size_t(B) * Hkv * Nk * d : 0);
+  const bool f16 = bwd_f16(Hq, Hkv, d), all16 = exact_dk(Hq / Hkv, d);
+  bwd_workspace_tail(w, f16 ? bh * Nq * d : 0, f16 ? size_t(B) * Hkv * Nk * d : 0,
+                     all16 ? bh * Nq * d : 0, all16 ? size_t(B) * Hkv * Nk * d : 0);
   return w;
 }
 inline size_t bwd_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d) {
@@ -134,7 +144,7 @@ inline size_t bwd_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d)
 // Dpad, Lpad fp32 [Hq, ld] with ld = round_up(total_q, 4) + 256 (B + 1),
 // each sequence's rows starting at varlen_pad_start | (GQA/MQA only)
 // dKacc, dVacc fp32 [Hkv, total_k, d] | dO16 fp16 [Hq, total_q, d] |
-// V16 fp16 [Hkv, total_k, d] | amax.
+// V16 fp16 [Hkv, total_k, d] | Q16, K16 | amax.
 inline long long varlen_lpad_ld(int B, int total_q) {
   return (long long)((total_q + 3) & ~3) + 256LL * (B + 1);
 }
@@ -148,8 +158,9 @@ inline BwdWorkspace bwd_workspace_layout_varlen(int B, int Hq, int Hkv, int tota
   w.l_off = w.d_off + up(size_t(Hq) * ld * 4);
   w.kv_off = w.l_off + up(size_t(Hq) * ld * 4);
   w.kv_elems = (Hq > Hkv) ? size_t(Hkv) * total_k * d : 0;
-  const bool f16 = bwd_f16(Hq, Hkv, d);
-  bwd_workspace_tail(w, f16 ? size_t(Hq) * total_q * d : 0, f16 ? size_t(Hkv) * total_k * d : 0);
+  const bool f16 = bwd_f16(Hq, Hkv, d), all16 = exact_dk(Hq / Hkv, d);
+  bwd_workspace_tail(w, f16 ? size_t(Hq) * total_q * d : 0, f16 ? size_t(Hkv) * total_k * d : 0,
+                     all16 ? size_t(Hq) * total_q * d : 0, all16 ? size_t(Hkv) * total_k * d : 0);
   return w;
 }
 
@@ -218,11 +229,11 @@ __device__ __forceinline__ void block_max_to(float m, unsigned* dst) {
   __syncthreads();
 }
 
-// Largest |V| of a [batch, heads, rows, D] view (element strides sv), into
-// amax[1]; the caller's block has already merged its |dO| maximum.
+// Largest |x| of a [batch, heads, rows, D] view (element strides sv),
+// merged into *dst.
 template <int D>
-__device__ __forceinline__ void v_absmax(const __nv_bfloat16* __restrict__ v, Strides sv, int batch,
-                                         int heads, int rows, unsigned* amax) {
+__device__ __forceinline__ void absmax_scan(const __nv_bfloat16* __restrict__ v, Strides sv,
+                                            int batch, int heads, int rows, unsigned* dst) {
   constexpr int PR = D / 8;                        // 8-element pieces per row
   const long long n = (long long)batch * heads * rows * PR;
   float m = 0.f;
@@ -234,19 +245,22 @@ __device__ __forceinline__ void v_absmax(const __nv_bfloat16* __restrict__ v, St
     m = fmaxf(m, absmax8(*reinterpret_cast<const uint4*>(v + bb * sv.b + hh * sv.h + r * sv.n +
                                                         sb * 8)));
   }
-  block_max_to(m, amax + 1);
+  block_max_to(m, dst);
 }
 
-// dO16 = fp16(dO * 2^e_dO) and V16 = fp16(V * 2^e_V), contiguous
-// [batch * heads, rows, D] (packed batches: batch 1, rows = the total),
-// after the preprocess kernel has left the largest magnitudes in amax.
+// Two fp16 copies in one launch: A16 = fp16(A * 2^e_A) for a query-side
+// tensor A (dO, or Q) and B16 = fp16(B * 2^e_B) for a key-side tensor B (V,
+// or K), contiguous [batch * heads, rows, D] (packed batches: batch 1, rows
+// = the total), after the preprocess kernel has left their largest
+// magnitudes in amax_a, amax_b.
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_f16_kernel(
     const __nv_bfloat16* __restrict__ dO, Strides sdo, int bq, int Hq, int rows_q,
     const __nv_bfloat16* __restrict__ v, Strides sv, int bk, int Hkv, int rows_k,
-    __half* __restrict__ do16, __half* __restrict__ v16, const unsigned* __restrict__ amax) {
+    __half* __restrict__ do16, __half* __restrict__ v16, const unsigned* __restrict__ amax_a,
+    const unsigned* __restrict__ amax_b) {
   constexpr int PR = D / 8;
-  const float s_do = ldexpf(1.f, f16_exp(amax[0])), s_v = ldexpf(1.f, f16_exp(amax[1]));
+  const float s_do = ldexpf(1.f, f16_exp(*amax_a)), s_v = ldexpf(1.f, f16_exp(*amax_b));
   const long long n_do = (long long)bq * Hq * rows_q * PR;
   const long long n_all = n_do + (long long)bk * Hkv * rows_k * PR;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n_all;
@@ -280,7 +294,8 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(
     const float* __restrict__ lse, float* __restrict__ dqacc, float* __restrict__ Dpad,
     float* __restrict__ Lpad, int rows_bh, int Hq, int Nq, int Nq_pad, Strides so, Strides sdo,
     float* __restrict__ kvacc, long long kv_n4, const __nv_bfloat16* __restrict__ v, Strides sv,
-    int B, int Hkv, int Nk, unsigned* __restrict__ amax) {
+    int B, int Hkv, int Nk, unsigned* __restrict__ amax, const __nv_bfloat16* __restrict__ qin,
+    Strides sq, const __nv_bfloat16* __restrict__ kin, Strides sk) {
   constexpr int TPR = D / 8;                       // threads per row
   constexpr int RPB = 256 / TPR;                   // rows per block pass
   const int sub = threadIdx.x % TPR;
@@ -331,7 +346,11 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(
     reinterpret_cast<float4*>(kvacc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   if (amax) {                                      // the fp16 operand scales (bwd_f16)
     block_max_to(mdo, amax);
-    v_absmax<D>(v, sv, B, Hkv, Nk, amax);
+    absmax_scan<D>(v, sv, B, Hkv, Nk, amax + 1);
+    if (qin) {                                     // and Q, K (exact_dk)
+      absmax_scan<D>(qin, sq, B, Hq, Nq, amax + 2);
+      absmax_scan<D>(kin, sk, B, Hkv, Nk, amax + 3);
+    }
   }
 }
 
@@ -349,7 +368,8 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_varlen_kernel(
     float* __restrict__ Lpad, const int* __restrict__ cu_q, int B, int Hq, int total_q,
     long long ld, Strides so, Strides sdo, float* __restrict__ kvacc, long long kv_n4,
     const __nv_bfloat16* __restrict__ v, Strides sv, int Hkv, int total_k,
-    unsigned* __restrict__ amax) {
+    unsigned* __restrict__ amax, const __nv_bfloat16* __restrict__ qin, Strides sq,
+    const __nv_bfloat16* __restrict__ kin, Strides sk) {
   constexpr int TPR = D / 8;
   constexpr int RPB = 256 / TPR;
   const int sub = threadIdx.x % TPR;
@@ -421,7 +441,11 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_varlen_kernel(
     reinterpret_cast<float4*>(kvacc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   if (amax) {                                      // the fp16 operand scales (bwd_f16)
     block_max_to(mdo, amax);
-    v_absmax<D>(v, sv, 1, Hkv, total_k, amax);
+    absmax_scan<D>(v, sv, 1, Hkv, total_k, amax + 1);
+    if (qin) {                                     // and Q, K (exact_dk)
+      absmax_scan<D>(qin, sq, 1, Hq, total_q, amax + 2);
+      absmax_scan<D>(kin, sk, 1, Hkv, total_k, amax + 3);
+    }
   }
 }
 
@@ -521,9 +545,45 @@ __device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_
       : "memory");
 }
 
+// Scale factors of the fp16 operands (f16_exp), per launch.
+//  F16 (bwd_f16): dP^T = 2^(e_dO + e_V) dP and dV_acc = 2^e_dO dV.
+//  ALL16 (exact_dk): also S^T = 2^(e_Q + e_K) S from the fp16 copies of Q
+//  and K, and dS goes in as fp16(dS * 2^e_dS), with 2^e_dS chosen from the
+//  bound |dS| <= |dP - D| <= 2 max|dP| <= 2 d max|dO| max|V| (P <= 1, D a
+//  P-weighted mean of the row's dP), so dK_acc = 2^(e_dS + e_Q) dK and the
+//  dQ^T product gives 2^(e_dS + e_K) dQ.  Every factor is a power of two.
+struct OpScales {
+  float sl2;      // multiplies S^T (scale * log2 e, unscaled)
+  float inv_vd;   // multiplies dP^T
+  float s_ds;     // multiplies dS before fp16 rounding
+  float mul_dk;   // multiplies the dK accumulator (includes the softmax scale)
+  float mul_dv;   // multiplies the dV accumulator
+  float mul_dq;   // multiplies dQ^T before its fp32 reduce-adds
+};
+template <int D, bool F16, bool ALL16>
+__device__ __forceinline__ OpScales op_scales(const unsigned* amax, float scale, float scale_log2) {
+  OpScales o{scale_log2, 1.f, 1.f, scale, 1.f, 1.f};
+  if constexpr (F16) {
+    const int e_do = f16_exp(__ldg(amax)), e_v = f16_exp(__ldg(amax + 1));
+    o.inv_vd = ldexpf(1.f, -e_do - e_v);
+    o.mul_dv = ldexpf(1.f, -e_do);
+    if constexpr (ALL16) {
+      const int e_q = f16_exp(__ldg(amax + 2)), e_k = f16_exp(__ldg(amax + 3));
+      const float bound = 2.f * float(D) * __uint_as_float(__ldg(amax)) *
+                          __uint_as_float(__ldg(amax + 1));
+      const int e_ds = f16_exp(__float_as_uint(bound));
+      o.sl2 = scale_log2 * ldexpf(1.f, -e_q - e_k);
+      o.s_ds = ldexpf(1.f, e_ds);
+      o.mul_dk = scale * ldexpf(1.f, -e_ds - e_q);
+      o.mul_dq = ldexpf(1.f, -e_ds - e_k);
+    }
+  }
+  return o;
+}
+
 // Block-sparse (SPARSE): a key block visits only the query blocks whose mask
 // entry for it is set, in the same cyclic order for every role.
-template <int D, bool CAUSAL, int MODE, bool SPLIT_DS, bool F16>
+template <int D, bool CAUSAL, int MODE, bool ALL16, bool F16>
 __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
@@ -711,13 +771,16 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && n_steps > 0) {
-      constexpr uint32_t ID_S = idesc_bf16_f32(128, BR, 0, 0);    // S^T: K-major both
+      constexpr uint32_t ID_S = ALL16 ? idesc_f16_f32(128, BR, 0, 0)   // S^T: K-major both
+                                      : idesc_bf16_f32(128, BR, 0, 0);
       constexpr uint32_t ID_DP = F16 ? idesc_f16_f32(128, BR, 0, 0)   // dP^T: fp16 V, dO
                                         : idesc_bf16_f32(128, BR, 0, 0);
-      constexpr uint32_t ID_KV = idesc_bf16_f32(128, DH, 0, 1);   // dK: B MN-major
+      constexpr uint32_t ID_KV = ALL16 ? idesc_f16_f32(128, DH, 0, 1)  // dK: B MN-major
+                                       : idesc_bf16_f32(128, DH, 0, 1);
       constexpr uint32_t ID_V = F16 ? idesc_f16_f32(128, DH, 0, 1)    // dV: fp16 P, dO
                                        : idesc_bf16_f32(128, DH, 0, 1);
-      constexpr uint32_t ID_DQ = idesc_bf16_f32(128, BR, 1, 1);   // dQ^T: A, B MN-major
+      constexpr uint32_t ID_DQ = ALL16 ? idesc_f16_f32(128, BR, 1, 1)  // dQ^T: A, B MN-major
+                                       : idesc_bf16_f32(128, BR, 1, 1);
       // Descriptor low words: K-major (S^T, dP^T operands) and MN-major (the
       // B operands of dV, dK and both operands of dQ^T).
       const uint32_t kK = sdesc_sw128_lo(smem_u32(sK), 16);
@@ -784,11 +847,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
         if (!(ok = mbar_wait(bar_ds, t & 1, abort_flag, p.status, WB_DS))) break;
         tc_fence_after();
 #pragma unroll
-        for (int half = 0; half < 1 + int(SPLIT_DS); ++half)
-#pragma unroll
-          for (int kk = 0; kk < BR / 16; ++kk)
-            umma_ts_lo(tmem + C::TM_DK, tmem + C::TM_DP + pcol(kk) + half * 16, mQ + kk * 128,
-                       ID_KV, (t > 0 || kk > 0 || half > 0) ? 1u : 0u);
+        for (int kk = 0; kk < BR / 16; ++kk)
+          umma_ts_lo(tmem + C::TM_DK, tmem + C::TM_DP + pcol(kk), mQ + kk * 128, ID_KV,
+                     (t > 0 || kk > 0) ? 1u : 0u);
         umma_commit(bar_qempty + st);
         // dQ^T = K^T dS^T  (M = 128 rows of d, N = BR queries, K = 128 keys).
         // For d = 64 the upper 64 rows of M read the V tile and are ignored.
@@ -822,6 +883,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
     const int w = warp - 12;
     const int r = w * 32 + lane;                   // d row
     const uint32_t tl = tmem + (uint32_t(w * 32) << 16);
+    // ALL16: dQ^T came from fp16 K and dS, scaled by 2^(e_dS + e_K)
+    const float mul_dq = op_scales<D, F16, ALL16>(p.amax, p.scale, p.scale_log2).mul_dq;
+    auto dqv = [&](uint32_t x) { return ALL16 ? __uint_as_float(x) * mul_dq : __uint_as_float(x); };
     Seq sq;
     if constexpr (SPARSE) seq_begin(sq);
     for (int u = 0; u < n_steps; ++u) {
@@ -849,12 +913,12 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
                                        : (size_t(bh) * p.Nq + q0) * D) + dcol0 + r;
         if (q0 + BR <= nq) {
 #pragma unroll
-          for (int i = 0; i < BR; ++i) atomicAdd(dst + i * D, __uint_as_float(v[i]));
+          for (int i = 0; i < BR; ++i) atomicAdd(dst + i * D, dqv(v[i]));
         } else {
           const int nvalid = nq - q0;
 #pragma unroll
           for (int i = 0; i < BR; ++i)
-            if (i < nvalid) atomicAdd(dst + i * D, __uint_as_float(v[i]));
+            if (i < nvalid) atomicAdd(dst + i * D, dqv(v[i]));
         }
       } else {
         tc_fence_before();
@@ -869,16 +933,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
     const int r = w * 32 + lane;                   // key row == TMEM lane (also d row for dQ^T)
     const uint32_t tl = tmem + (uint32_t(w * 32) << 16);
     const int key = key0 + r;
-    const float sl2 = p.scale_log2;
-    // F16: dP^T and dV come from fp16 operands scaled by powers of two
-    // (f16_exp): dP = dP^T * 2^-(e_dO + e_V), dV = acc * 2^-e_dO, exactly
-    int e_do = 0, e_v = 0;
-    if constexpr (F16) {
-      e_do = f16_exp(__ldg(p.amax));
-      e_v = f16_exp(__ldg(p.amax + 1));
-    }
-    const float inv_do = ldexpf(1.f, -e_do);
-    const float2 inv_vd2 = make_float2(ldexpf(1.f, -e_do - e_v), ldexpf(1.f, -e_do - e_v));
+    // fp16 operands (F16, ALL16) come scaled by powers of two (op_scales)
+    const OpScales os = op_scales<D, F16, ALL16>(p.amax, p.scale, p.scale_log2);
+    const float sl2 = os.sl2;
+    const float2 inv_vd2 = make_float2(os.inv_vd, os.inv_vd);
+    const float2 s_ds2 = make_float2(os.s_ds, os.s_ds);
     bool ok = true;
 
     Seq sq;
@@ -954,7 +1013,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
         for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4*>(dd + i) =
             *reinterpret_cast<const float4*>(sd + i);
         tmem_wait_ld();
-        uint32_t pk[16], lo[16];
+        uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           // dP^T came from the scaled fp16 operands: dP = dP^T_scaled * 2^-(e_dO + e_V)
@@ -962,14 +1021,14 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
           const float2 nd = make_float2(-dd[2 * i], -dd[2 * i + 1]);
           const float2 x = F16 ? ffma2(dp2, inv_vd2, nd) : fadd2(dp2, nd);
           const float2 y = fmul2(make_float2(P[2 * i], P[2 * i + 1]), x);
-          pk[i] = pack_bf16(y.x, y.y);
-          if constexpr (SPLIT_DS)
-            lo[i] = pack_bf16(y.x - __uint_as_float(pk[i] << 16),
-                              y.y - __uint_as_float(pk[i] & 0xFFFF0000u));
+          if constexpr (ALL16) {                 // fp16(dS * 2^e_dS)
+            const float2 z = fmul2(y, s_ds2);
+            pk[i] = pack_f16(z.x, z.y);
+          } else {
+            pk[i] = pack_bf16(y.x, y.y);
+          }
         }
         FA_TMEM_ST16(tDP, pk);
-        // dS lo over the group's other 16 columns (all 32 were read above)
-        if constexpr (SPLIT_DS) FA_TMEM_ST16(tDP + 16, lo);
         // dS^T row r, queries 32g..32g+31: half of a 128-byte swizzled row
         uint8_t* row = sdS + r * 128;
 #pragma unroll
@@ -998,7 +1057,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
       // (all lanes load from TMEM together; rows past Nk add nothing).
       if (n_steps > 0) {
         const int tcol = g == 0 ? C::TM_DK : C::TM_DV;
-        const float mul = g == 0 ? p.scale : inv_do;
+        const float mul = g == 0 ? os.mul_dk : os.mul_dv;
         float* dst = (g == 0 ? p.dkacc : p.dvacc) +
                      (VARLEN ? size_t(hkv) * p.total_k + koff + key : size_t(bkv) * p.Nk + key) *
                          D + dcol0;
@@ -1021,7 +1080,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
       }
     } else if (ok) {
       const int tcol = g == 0 ? C::TM_DK : C::TM_DV;
-      const float mul = g == 0 ? p.scale : inv_do;
+      const float mul = g == 0 ? os.mul_dk : os.mul_dv;
       uint8_t* stage = sStage + g * (BC * DH * 2);
       // Packed batches: a warp whose 32 key rows run past the sequence's
       // end stores its rows directly (a TMA box would reach the next one).
@@ -1115,6 +1174,8 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
   float* kvacc = reinterpret_cast<float*>(ws + w.kv_off);
   __half* do16 = reinterpret_cast<__half*>(ws + w.do16_off);
   __half* v16 = reinterpret_cast<__half*>(ws + w.v16_off);
+  __half* q16 = reinterpret_cast<__half*>(ws + w.q16_off);
+  __half* k16 = reinterpret_cast<__half*>(ws + w.k16_off);
   unsigned* amax = reinterpret_cast<unsigned*>(ws + w.amax_off);
   const int Nq_pad = round_up(Nq, 128);
   const int bhq = B * Hq;
@@ -1148,10 +1209,13 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
   // fp16 copies (TMA moves the 16-bit elements unchanged; the map's element
   // type only matters for a NaN out-of-bounds fill, which is not used).
   const bool f16 = bwd_f16(Hq, Hkv, D);
+  // exact_dk: dS, and with it S^T, dK and dQ^T, take fp16 operands as well
+  const bool all16 = exact_dk(group, D);
   const Strides s_v16{(long long)Hkv * rows_k * D, (long long)rows_k * D, D};
   const Strides s_do16{(long long)Hq * rows_q * D, (long long)rows_q * D, D};
-  if ((stages & 2) && (!make_map_bf16(&mq, q, D, rows_q, Hq, map_b, st[0], BRK) ||
-      !make_map_bf16(&mk, k, D, rows_k, Hkv, map_b, st[1], C::BC) ||
+  if ((stages & 2) &&
+      (!make_map_bf16(&mq, all16 ? q16 : q, D, rows_q, Hq, map_b, all16 ? s_do16 : st[0], BRK) ||
+       !make_map_bf16(&mk, all16 ? k16 : k, D, rows_k, Hkv, map_b, all16 ? s_v16 : st[1], C::BC) ||
       !make_map_bf16(&mv, f16 ? v16 : v, D, rows_k, Hkv, map_b, f16 ? s_v16 : st[2], C::BC) ||
       !make_map_bf16(&mdo, f16 ? do16 : dO, D, rows_q, Hq, map_b, f16 ? s_do16 : st[4], BRK) ||
       !make_map_bf16(&mdk, dk, D, rows_k, Hkv, map_b, st[6], 32) ||
@@ -1161,7 +1225,7 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
 
   if (stages & 1) {
     constexpr int RPB = 256 / (D / 8);
-    if (f16 && cudaMemsetAsync(amax, 0, 2 * sizeof(unsigned), stream) != cudaSuccess) return 5;
+    if (f16 && cudaMemsetAsync(amax, 0, 4 * sizeof(unsigned), stream) != cudaSuccess) return 5;
     if (vl) {
       const long long rows = (long long)Hq * vl->total_q;
       const long long blocks = std::max<long long>(
@@ -1170,7 +1234,8 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
           static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, dqacc,
           Dpad, Lpad, vl->cu_q, B, Hq, vl->total_q, varlen_lpad_ld(B, vl->total_q), st[3], st[4],
           kvacc, kv_n4, static_cast<const __nv_bfloat16*>(v), st[2], Hkv, vl->total_k,
-          f16 ? amax : nullptr);
+          f16 ? amax : nullptr, all16 ? static_cast<const __nv_bfloat16*>(q) : nullptr, st[0],
+          static_cast<const __nv_bfloat16*>(k), st[1]);
     } else {
       const long long rows = (long long)bhq * Nq_pad;
       const long long blocks = std::min<long long>((rows + RPB - 1) / RPB, 148LL * 16);
@@ -1178,7 +1243,9 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
           static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(ores),
           static_cast<const __nv_bfloat16*>(dO), lse, dqacc,
           Dpad, Lpad, bhq, Hq, Nq, Nq_pad, st[3], st[4], kvacc, kv_n4,
-          static_cast<const __nv_bfloat16*>(v), st[2], B, Hkv, Nk, f16 ? amax : nullptr);
+          static_cast<const __nv_bfloat16*>(v), st[2], B, Hkv, Nk, f16 ? amax : nullptr,
+          all16 ? static_cast<const __nv_bfloat16*>(q) : nullptr, st[0],
+          static_cast<const __nv_bfloat16*>(k), st[1]);
     }
     if (f16) {
       const long long pieces = ((long long)map_b * Hq * rows_q + (long long)map_b * Hkv * rows_k) *
@@ -1187,7 +1254,13 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
                                                                           148LL * 16));
       fa_bwd_f16_kernel<D><<<unsigned(blocks), 256, 0, stream>>>(
           static_cast<const __nv_bfloat16*>(dO), st[4], map_b, Hq, rows_q,
-          static_cast<const __nv_bfloat16*>(v), st[2], map_b, Hkv, rows_k, do16, v16, amax);
+          static_cast<const __nv_bfloat16*>(v), st[2], map_b, Hkv, rows_k, do16, v16, amax,
+          amax + 1);
+      if (all16)
+        fa_bwd_f16_kernel<D><<<unsigned(blocks), 256, 0, stream>>>(
+            static_cast<const __nv_bfloat16*>(q), st[0], map_b, Hq, rows_q,
+            static_cast<const __nv_bfloat16*>(k), st[1], map_b, Hkv, rows_k, q16, k16, amax + 2,
+            amax + 3);
     }
     if (cudaGetLastError() != cudaSuccess) return 5;
   }
@@ -1195,9 +1268,8 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
     using C2 = typename std::conditional<STEP128, Bwd128Cfg<(D <= 128 ? D : 128)>, C>::type;
     // dK sums dS^T Q over every query row of the kv group: for wide groups
     // rounding dS to bf16 alone moves dK by about 2e-2 (causal, N = 4096),
-    // so dS also goes in as hi + lo there (exact_dk).
-    const bool split_ds = exact_dk(group, D);
-    // instances: (fp16 dP / dV, dS split) = (no, no) for MHA at d <= 128,
+    // so dS goes in as fp16 there (exact_dk: all16).
+    // instances: (fp16 dP / dV, fp16 dS) = (no, no) for MHA at d <= 128,
     // (yes, exact_dk) otherwise; d = 256 is always fp16 (bwd_f16)
     auto pick = [&](auto split_tag, auto f16_tag) {
       constexpr bool S = decltype(split_tag)::value, F = decltype(f16_tag)::value;
@@ -1212,8 +1284,8 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
                       : fa_bwd_main_kernel<D, CAUSAL, BMODE_DENSE, S, true>;
     };
     auto kern = !f16    ? pick(std::false_type{}, std::false_type{})
-                : split_ds ? pick(std::true_type{}, std::true_type{})
-                           : pick(std::false_type{}, std::true_type{});
+                : all16 ? pick(std::true_type{}, std::true_type{})
+                        : pick(std::false_type{}, std::true_type{});
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C2::SMEM_BYTES) !=
         cudaSuccess)
       return 5;

@@ -8,8 +8,8 @@
 //
 // At d = 128, TMEM (512 columns) cannot hold S^T, dP^T, dQ^T, dK and dV of
 // a 128-query step side by side, so regions are reused within a step:
-//   SP  [0, 128)    S^T (fp32)  -> P^T as bf16 hi | lo pairs (per group)
-//   DP  [128, 256)  dP^T (fp32) -> dS^T as bf16 pairs -> dQ^T (fp32)
+//   SP  [0, 128)    S^T (fp32)  -> P^T as 16-bit pairs (per group)
+//   DP  [128, 256)  dP^T (fp32) -> dS^T as 16-bit pairs -> dQ^T (fp32)
 //   DK  [256, 256 + d), DV [256 + d, 256 + 2d)
 // At d = 64, dQ^T has its own columns [384, 512).
 // MMA order per step t (one issuing thread; tcgen05 MMAs run in issue
@@ -23,10 +23,11 @@
 // frees DP for dP_{t+1}.  Waiting for dP_t also proves that dQ_{t-1}, which
 // reads the shared dS^T tile, has finished before dS_t overwrites it.
 //
-// P goes to TMEM as bf16 hi (plus lo = P - hi when the precision rule asks
-// for it: GQA/MQA groups) for dV, and stays in the thread's registers in
-// fp32 for dS, because S^T_{t+1} overwrites the P^T columns while dS_t is
-// being formed.  The LSE
+// P goes to TMEM rounded once for dV (bf16; fp16 with the F16 operands of
+// GQA / MQA groups) and stays in the thread's registers in fp32 for dS,
+// because S^T_{t+1} overwrites the P^T columns while dS_t is being formed.
+// With ALL16 (wide groups) every product takes fp16 operands and dS goes
+// in as fp16 (op_scales, fa_bwd.cuh).  The LSE
 // and D rows are read straight from the workspace (L1-resident broadcast
 // loads) rather than staged, which keeps shared memory within 227 KB.
 #pragma once
@@ -67,7 +68,7 @@ struct Bwd128Cfg {
   static_assert(QS * STAGE_BYTES >= 2 * BC * DH * 2, "dK/dV staging fits in the Q/dO stages");
 };
 
-template <int D, bool CAUSAL, int MODE, bool SPLIT_DS, bool F16>
+template <int D, bool CAUSAL, int MODE, bool ALL16, bool F16>
 __global__ void __launch_bounds__(Bwd128Cfg<D>::NTHREADS, 1)
     fa_bwd_main128_kernel(const __grid_constant__ CUtensorMap tmQ,
                           const __grid_constant__ CUtensorMap tmK,
@@ -238,13 +239,16 @@ __global__ void __launch_bounds__(Bwd128Cfg<D>::NTHREADS, 1)
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && n_steps > 0) {
-      constexpr uint32_t ID_S = idesc_bf16_f32(128, BR, 0, 0);    // S^T: K-major both
+      constexpr uint32_t ID_S = ALL16 ? idesc_f16_f32(128, BR, 0, 0)   // S^T: K-major both
+                                      : idesc_bf16_f32(128, BR, 0, 0);
       constexpr uint32_t ID_DP = F16 ? idesc_f16_f32(128, BR, 0, 0)   // dP^T: fp16 V, dO
                                         : idesc_bf16_f32(128, BR, 0, 0);
-      constexpr uint32_t ID_KV = idesc_bf16_f32(128, DH, 0, 1);   // dK: B MN-major
+      constexpr uint32_t ID_KV = ALL16 ? idesc_f16_f32(128, DH, 0, 1)  // dK: B MN-major
+                                       : idesc_bf16_f32(128, DH, 0, 1);
       constexpr uint32_t ID_V = F16 ? idesc_f16_f32(128, DH, 0, 1)    // dV: fp16 P, dO
                                        : idesc_bf16_f32(128, DH, 0, 1);
-      constexpr uint32_t ID_DQ = idesc_bf16_f32(128, BR, 1, 1);   // dQ^T: A, B MN-major
+      constexpr uint32_t ID_DQ = ALL16 ? idesc_f16_f32(128, BR, 1, 1)  // dQ^T: A, B MN-major
+                                       : idesc_bf16_f32(128, BR, 1, 1);
       // Descriptor low words: K-major (S^T, dP^T operands) and MN-major (the
       // B operands of dV, dK and both operands of dQ^T).
       const uint32_t kK = sdesc_sw128_lo(smem_u32(sK), 16);
@@ -301,11 +305,9 @@ __global__ void __launch_bounds__(Bwd128Cfg<D>::NTHREADS, 1)
         if (!(ok = mbar_wait(bar_ds, t & 1, abort_flag, p.status, WB_DS))) break;
         tc_fence_after();
 #pragma unroll
-        for (int half = 0; half < 1 + int(SPLIT_DS); ++half)
-#pragma unroll
-          for (int kk = 0; kk < BR / 16; ++kk)
-            umma_ts_lo(tmem + C::TM_DK, tmem + C::TM_DP + pcol(kk) + half * 16, mQ + kk * 128,
-                       ID_KV, (t > 0 || kk > 0 || half > 0) ? 1u : 0u);
+        for (int kk = 0; kk < BR / 16; ++kk)
+          umma_ts_lo(tmem + C::TM_DK, tmem + C::TM_DP + pcol(kk), mQ + kk * 128, ID_KV,
+                     (t > 0 || kk > 0) ? 1u : 0u);
         umma_commit(bar_qempty + st);
         // dQ^T = K^T dS^T (M = 128 rows of d, N = 128 queries, K = 128 keys);
         // for d = 64 the upper 64 rows of M read the V tile and are ignored.
@@ -346,6 +348,9 @@ __global__ void __launch_bounds__(Bwd128Cfg<D>::NTHREADS, 1)
     const int w = warp - 12;
     const int r = w * 32 + lane;                   // d row
     const uint32_t tl = tmem + (uint32_t(w * 32) << 16);
+    // ALL16: dQ^T came from fp16 K and dS, scaled by 2^(e_dS + e_K)
+    const float mul_dq = op_scales<D, F16, ALL16>(p.amax, p.scale, p.scale_log2).mul_dq;
+    auto dqv = [&](uint32_t x) { return ALL16 ? __uint_as_float(x) * mul_dq : __uint_as_float(x); };
     Seq sq;
     if constexpr (SPARSE) seq_begin(sq);
     for (int u = 0; u < n_steps; ++u) {
@@ -369,12 +374,12 @@ __global__ void __launch_bounds__(Bwd128Cfg<D>::NTHREADS, 1)
                              : (size_t(b * p.Hq + head0 + hh) * p.Nq + q0) * D) + r;
         if (q0 + BR <= nq) {
 #pragma unroll
-          for (int i = 0; i < BR; ++i) atomicAdd(dst + i * D, __uint_as_float(v[i]));
+          for (int i = 0; i < BR; ++i) atomicAdd(dst + i * D, dqv(v[i]));
         } else {
           const int nvalid = nq - q0;
 #pragma unroll
           for (int i = 0; i < BR; ++i)
-            if (i < nvalid) atomicAdd(dst + i * D, __uint_as_float(v[i]));
+            if (i < nvalid) atomicAdd(dst + i * D, dqv(v[i]));
         }
       }
     }
@@ -386,16 +391,11 @@ __global__ void __launch_bounds__(Bwd128Cfg<D>::NTHREADS, 1)
     const int r = w * 32 + lane;                   // key row == TMEM lane
     const uint32_t tl = tmem + (uint32_t(w * 32) << 16);
     const int key = key0 + r;
-    const float sl2 = p.scale_log2;
-    // F16: dP^T and dV come from fp16 operands scaled by powers of two
-    // (f16_exp): dP = dP^T * 2^-(e_dO + e_V), dV = acc * 2^-e_dO, exactly
-    int e_do = 0, e_v = 0;
-    if constexpr (F16) {
-      e_do = f16_exp(__ldg(p.amax));
-      e_v = f16_exp(__ldg(p.amax + 1));
-    }
-    const float inv_do = ldexpf(1.f, -e_do);
-    const float2 inv_vd2 = make_float2(ldexpf(1.f, -e_do - e_v), ldexpf(1.f, -e_do - e_v));
+    // fp16 operands (F16, ALL16) come scaled by powers of two (op_scales)
+    const OpScales os = op_scales<D, F16, ALL16>(p.amax, p.scale, p.scale_log2);
+    const float sl2 = os.sl2;
+    const float2 inv_vd2 = make_float2(os.inv_vd, os.inv_vd);
+    const float2 s_ds2 = make_float2(os.s_ds, os.s_ds);
     bool ok = true;
     Seq sq;
     if constexpr (SPARSE) seq_begin(sq);
@@ -457,14 +457,12 @@ __global__ void __launch_bounds__(Bwd128Cfg<D>::NTHREADS, 1)
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
       {
-        constexpr bool SPLIT = SPLIT_DS;
-        uint32_t lo_even[8];                        // dS lo of a chunk's first 16 queries
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t dpv[16];
           FA_TMEM_LD16(tDP + c * 16, dpv);
           tmem_wait_ld();
-          uint32_t pk[8], lo[8];
+          uint32_t pk[8];
 #pragma unroll
           for (int i = 0; i < 8; i += 2) {
             const float4 d4 = __ldg(dd4 + (c * 16 + 2 * i) / 4);
@@ -477,27 +475,18 @@ __global__ void __launch_bounds__(Bwd128Cfg<D>::NTHREADS, 1)
                                              __uint_as_float(dpv[2 * (i + e) + 1]));
               const float2 nd = make_float2(-dsub[2 * e], -dsub[2 * e + 1]);
               const float2 x = F16 ? ffma2(dp2, inv_vd2, nd) : fadd2(dp2, nd);
-              const float2 y = fmul2(pp, x);
-              pk[i + e] = pack_bf16(y.x, y.y);
-              if constexpr (SPLIT)
-                lo[i + e] = pack_bf16(y.x - __uint_as_float(pk[i + e] << 16),
-                                      y.y - __uint_as_float(pk[i + e] & 0xFFFF0000u));
+              if constexpr (ALL16) {             // fp16(dS * 2^e_dS)
+                const float2 y = fmul2(fmul2(pp, x), s_ds2);
+                pk[i + e] = pack_f16(y.x, y.y);
+              } else {
+                const float2 y = fmul2(pp, x);
+                pk[i + e] = pack_bf16(y.x, y.y);
+              }
             }
           }
           // dS^T pairs over already read dP^T columns of this 32-query chunk
           // (the chunk's first 16 columns, 8 per 16 queries) ...
           FA_TMEM_ST8(tDP + (c >> 1) * 32 + (c & 1) * 8, pk);
-          // ... when split, the lo pairs over the chunk's last 16 columns,
-          // which are all read only once the chunk's second half is ...
-          if constexpr (SPLIT) {
-            if ((c & 1) == 0) {
-#pragma unroll
-              for (int i = 0; i < 8; ++i) lo_even[i] = lo[i];
-            } else {
-              FA_TMEM_ST8(tDP + (c >> 1) * 32 + 16, lo_even);
-              FA_TMEM_ST8(tDP + (c >> 1) * 32 + 24, lo);
-            }
-          }
           // ... and into the shared tile for dQ: row r, queries [64g + 16c, +16)
           uint8_t* rowp = sdS + g * (BC * 128) + r * 128;
 #pragma unroll
@@ -523,7 +512,7 @@ __global__ void __launch_bounds__(Bwd128Cfg<D>::NTHREADS, 1)
     if (ok && p.gsplit > 1) {
       if (n_steps > 0) {
         const int tcol = g == 0 ? C::TM_DK : C::TM_DV;
-        const float mul = g == 0 ? p.scale : inv_do;
+        const float mul = g == 0 ? os.mul_dk : os.mul_dv;
         float* dst = (g == 0 ? p.dkacc : p.dvacc) +
                      (VARLEN ? size_t(hkv) * p.total_k + koff + key : size_t(bkv) * p.Nk + key) *
                          D;
@@ -546,7 +535,7 @@ __global__ void __launch_bounds__(Bwd128Cfg<D>::NTHREADS, 1)
       }
     } else if (ok) {
       const int tcol = g == 0 ? C::TM_DK : C::TM_DV;
-      const float mul = g == 0 ? p.scale : inv_do;
+      const float mul = g == 0 ? os.mul_dk : os.mul_dv;
       uint8_t* stage = sStage + g * (BC * DH * 2);
       const bool direct = VARLEN && (key0 + w * 32 + 32 > nk);
 #pragma unroll

@@ -90,7 +90,8 @@ int fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* 
  * fp32 dQ accumulator [B, Hq, Nq, d] and two fp32 row vectors (D =
  * rowsum(dO * O) and LSE * log2 e) padded to 128 rows per head; for GQA /
  * MQA groups also fp32 dK / dV partial sums [B, Hkv, Nk, d], and for GQA /
- * MQA groups and d = 256 fp16 copies of dO and V (see fa_bwd).
+ * MQA groups and d = 256 fp16 copies of dO and V, for wide groups also of
+ * Q and K (see fa_bwd).
  * Returns 0 for invalid sizes.
  */
 size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal);
@@ -106,7 +107,9 @@ size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int 
  * D = rowsum(dO * O) from the bf16 o adds up; the pass then recomputes D
  * from the fp32 output with one more forward pass (about the forward's
  * time).  fa_fwd_residual / fa_bwd_residual give the same precision
- * without it.
+ * without it.  For these groups every product takes fp16 operands (q and
+ * k are copied like dO and v below) and dS goes in rounded to fp16, scaled
+ * by a power of two chosen from the bound |dS| <= 2 d max|dO| max|v|.
  * GQA / MQA groups and d = 256: dV = P^T dO and dP = dO V^T take fp16
  * operands (P rounded to fp16, 8x finer than bf16, which dV sums over every
  * query row of the group).  The preprocess copies dO and V into the
@@ -235,7 +238,7 @@ typedef enum {
   FA_BWD_ALL = 0,   /* the whole backward pass (same as fa_bwd) */
   FA_BWD_PRE = 1,   /* D = rowsum(dO * O), LSE copy, dQ accumulator := 0 (in the workspace);
                        GQA / MQA and d = 256: the fp16 copies of dO and V; wide groups:
-                       the forward pass that recomputes D (see fa_bwd) */
+                       those of Q and K and the forward pass that recomputes D (see fa_bwd) */
   FA_BWD_MAIN = 2,  /* dK, dV written; dQ accumulated into the workspace */
   FA_BWD_DQ = 3     /* dq = scale * dQ accumulator, as bf16 */
 } fa_bwd_stage_t;

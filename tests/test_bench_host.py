@@ -127,9 +127,10 @@ def test_launches_per_step():
     assert bench.launches_per_step(w["train_b8h16n2048d128_full"], 148) == 4
     # d = 256: the fp16 copy of dO and V
     assert bench.launches_per_step(w["large_b4h8n4096d256_full"], 148) == 5
-    # 32 query heads on one kv head, 128 key blocks: the fp16 copy, the split
-    # and its dK/dV convert, and the forward pass that recomputes D
-    assert bench.launches_per_step(w["long_gqa_hkv1_n16384_d128_causal"], 148) == 7
+    # 32 query heads on one kv head, 128 key blocks: the fp16 copies (dO, V;
+    # Q, K), the split and its dK/dV convert, and the forward pass that
+    # recomputes D
+    assert bench.launches_per_step(w["long_gqa_hkv1_n16384_d128_causal"], 148) == 8
     # 8 kv heads x 128 key blocks = 1024 CTAs: no split; the fp16 copy
     assert bench.launches_per_step(w["long_gqa_hkv8_n16384_d128_causal"], 148) == 5
 
