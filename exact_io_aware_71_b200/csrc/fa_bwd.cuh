@@ -852,7 +852,6 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
                      (t > 0 || kk > 0) ? 1u : 0u);
         umma_commit(bar_qempty + st);
         // dQ^T = K^T dS^T  (M = 128 rows of d, N = BR queries, K = 128 keys).
-        // For d = 64 the upper 64 rows of M read the V tile and are ignored.
         if (t > 0 && !(ok = mbar_wait(bar_dqempty, (t - 1) & 1, abort_flag, p.status, WB_DQEMPTY)))
           break;
         tc_fence_after();

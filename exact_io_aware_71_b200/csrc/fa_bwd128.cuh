@@ -310,7 +310,8 @@ __global__ void __launch_bounds__(Bwd128Cfg<D>::NTHREADS, 1)
                      (t > 0 || kk > 0) ? 1u : 0u);
         umma_commit(bar_qempty + st);
         // dQ^T = K^T dS^T (M = 128 rows of d, N = 128 queries, K = 128 keys);
-        // for d = 64 the upper 64 rows of M read the V tile and are ignored.
+        // for d = 64 the upper 64 rows of M read the V tile's 16-bit elements (whatever
+        // their type) and are ignored.
         // In its own columns it only waits for the read-out of dQ^T_{t-1}.
         if constexpr (C::DQ_OWN) {
           if (t > 0 &&

@@ -268,9 +268,10 @@ int fa_bwd_stage(int stage, const void* q, const void* k, const void* v, const v
  * application that owns every device allocation, or code on a
  * latency-critical path where cudaMalloc (which may synchronise the device)
  * is not acceptable.  Same arguments and results as fa_bwd without the
- * workspace: its scratch (the fp32 dQ accumulator and the two fp32 row
- * vectors) lives in the library's built-in array of FA_NOALLOC_SCRATCH_BYTES
- * instead.  The call allocates nothing and calls no allocating routine.
+ * workspace: its scratch (the fp32 dQ accumulator, the two fp32 row vectors
+ * and, for GQA / MQA groups and d = 256, the fp16 operand copies; all that
+ * fa_bwd_workspace_size() counts) lives in the library's built-in array of
+ * FA_NOALLOC_SCRATCH_BYTES instead.  The call allocates nothing and calls no allocating routine.
  *  - Problems whose fa_bwd_workspace_size() exceeds FA_NOALLOC_SCRATCH_BYTES
  *    are rejected with FA_ERR_TOO_LARGE before anything is launched.
  *  - Every call looks up the array's device address in the caller's current

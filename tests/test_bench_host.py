@@ -92,6 +92,10 @@ def test_traffic_is_reported_only_for_current_sources(tmp_path, monkeypatch):
     (prof / "traffic.json").write_text(json.dumps(rec))
     assert bench.recorded_traffic("k", "w") == 123
     assert bench.recorded_traffic("k", "other") is None
+    # a comment-only edit keeps the record; a code edit drops it
+    (tmp_path / bench.KERNEL_SOURCES[0]).write_text("kernel  " + bench.KERNEL_SOURCES[0] +
+                                                    "  // note\n/* block */")
+    assert bench.recorded_traffic("k", "w") == 123
     (tmp_path / bench.KERNEL_SOURCES[0]).write_text("changed")
     assert bench.recorded_traffic("k", "w") is None
 
