@@ -116,7 +116,9 @@ size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int 
  * workspace as fp16, each scaled by one power of two chosen from its
  * largest magnitude, so the copy is exact for every element within a factor
  * 2^24 of that magnitude; smaller elements keep an absolute error below
- * 2^-25 of it.  Non-finite dO or V give non-finite results, as in bf16.
+ * 2^-25 of it.  (The scale stops at 2^60 and 2^-60: a largest magnitude
+ * below 2^-46 or above 2^75 keeps less precision.)  Non-finite dO or V give
+ * non-finite results, as in bf16.
  */
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
            const void* dO, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nk,

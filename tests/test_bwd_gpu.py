@@ -179,3 +179,39 @@ def kv_rows_parallel(wl, q, k, v, do, dk, dv, keys):
         ref_k[b, j] += pk
         ref_v[b, j] += pv
     return dk[:, :, keys], dv[:, :, keys], ref_k, ref_v
+
+
+def _grads_with_do_scaled(wl, k):
+    """fa.forward + fa.backward with dO multiplied by 2^k (exact in bf16)."""
+    q, kk, v, do = (t.to(DEV) for t in make_inputs(wl))
+    do = (do.float() * 2.0 ** k).to(torch.bfloat16)
+    o, lse = fa.forward(q, kk, v, wl.causal, wl.scale)
+    grads = fa.backward(q, kk, v, o, lse, do, wl.causal, wl.scale)
+    torch.cuda.synchronize()
+    st, where = fa.fa_device_status(None)
+    assert st == 0, f"device status {st} at wait {where}"
+    return [g.float().cpu().double().numpy() for g in grads]
+
+
+@pytest.mark.parametrize("wl", [W(1, 8, 2, 640, 640, 128, True),     # GQA: fp16 dP, dV
+                                W(1, 16, 1, 512, 512, 128, False),    # MQA: every product fp16
+                                W(1, 2, 2, 384, 384, 256, False)],    # d = 256: fp16 dP, dV
+                         ids=lambda w: w.name)
+@pytest.mark.parametrize("k", [-24, 16])
+def test_fp16_operand_scales_follow_a_power_of_two(wl, k):
+    """The fp16 operands carry scales chosen from the largest |dO|, |V| (and
+    |Q|, |K|, and the bound on |dS| for wide groups).  Multiplying dO by 2^k
+    must multiply every gradient by exactly 2^k: the kernels' powers of two
+    absorb k (including max |dO| near 2^18, beyond fp16's range, for
+    k = 16).  The only difference allowed is the order of the fp32
+    reduce-adds of dQ and of split dK / dV, at most one bf16 ulp.  With the
+    parity tests at k = 0 this covers dO at any scale."""
+    base = _grads_with_do_scaled(wl, 0)
+    scaled = _grads_with_do_scaled(wl, k)
+    for name, g0, gk in zip(("dQ", "dK", "dV"), base, scaled):
+        assert np.isfinite(gk).all(), name
+        back = gk * 2.0 ** -k
+        ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(g0), 1e-300))) - 7)
+        diff = np.abs(back - g0)
+        assert (diff[g0 == 0] == 0).all(), name
+        assert (diff <= ulp + 1e-300).all(), f"{name}: max ulp {float((diff / ulp).max())}"
