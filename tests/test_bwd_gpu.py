@@ -72,10 +72,10 @@ def test_unequal_lengths(nq, nk, causal):
 @pytest.mark.parametrize("causal", [False, True])
 def test_mqa_wide_group(causal, d, residual):
     """32 query heads on one kv head (N=1024): the per-CTA loop over the
-    group.  Wide groups take dS as bf16 hi + lo in dK and an exact D: from
-    the forward's residual output, or recomputed by a forward pass.  Strict
-    bar on all three gradients (tests/test_precision_model.py shows why both
-    are needed)."""
+    group.  Wide groups take an exact D (from the forward's residual output,
+    or recomputed by a forward pass) and dS rounded to fp16, with every
+    product on fp16 operands.  Strict bar on all three gradients
+    (tests/test_precision_model.py shows why both are needed)."""
     full_check(W(1, 32, 1, 1024, 1024, d, causal, seed=3), residual=residual)
 
 
@@ -91,10 +91,10 @@ def test_long_gqa_shape_full_oracle(hkv, residual):
 def test_large_magnitude_scores(qmul):
     """Peaky softmax (stress inputs Q x 2 and Q x 4, outside the named
     workloads); dK held to the Frobenius bar.  With one query head per kv
-    head neither the dS split nor the exact D applies, and even both would
-    leave Q x 4 above the per-element bar: the exact-arithmetic model in
-    tests/test_precision_model.py puts the remaining error in the forward's
-    bf16 P, which sets the fp32 output that D is formed from."""
+    head the backward takes D from the bf16 output and dS as bf16 (the
+    exact D and the fp16 dS are for wide groups); the exact-arithmetic model
+    in tests/test_precision_model.py shows dK above the per-element bound
+    there, mostly from D, and within it once D is exact."""
     full_check(W(1, 2, 2, 512, 512, 64, True, seed=9), qmul=qmul, frobenius_only=("dK",))
 
 
