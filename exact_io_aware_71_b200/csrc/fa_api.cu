@@ -325,14 +325,21 @@ int recompute_d(const void* q, const void* k, const void* v, const void* o, cons
   const int rows_q = vl ? vl->total_q : Nq, rows_k = vl ? vl->total_k : Nk;
   const int map_b = vl ? 1 : B;
   const int bc = (d == 256) ? 64 : 128;
+  const BwdWorkspace w = vl ? bwd_workspace_layout_varlen(B, Hq, Hkv, vl->total_q, vl->total_k, d)
+                            : bwd_workspace_layout(B, Hq, Hkv, Nq, Nk, d);
+  // d <= 128: the tile-pair kernel multiplies P (as fp16) by the preprocess
+  // stage's fp16 copy of V (these groups always have one); d = 256 keeps
+  // bf16 V with P as hi + lo.
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const bool v16 = d <= 128;
+  const Strides s_v16{(long long)Hkv * rows_k * d, (long long)rows_k * d, d};
   CUtensorMap mq, mk, mv, mo;
   if (!make_map_bf16(&mq, q, d, rows_q, Hq, map_b, st[0], 128) ||
       !make_map_bf16(&mk, k, d, rows_k, Hkv, map_b, st[1], bc) ||
-      !make_map_bf16(&mv, v, d, rows_k, Hkv, map_b, st[2], bc) ||
+      !make_map_bf16(&mv, v16 ? static_cast<const void*>(ws + w.v16_off) : v, d, rows_k, Hkv,
+                     map_b, v16 ? s_v16 : st[2], bc) ||
       !make_map_bf16(&mo, o, d, rows_q, Hq, map_b, st[3], 32))
     return FA_ERR_CUDA;
-  const BwdWorkspace w = vl ? bwd_workspace_layout_varlen(B, Hq, Hkv, vl->total_q, vl->total_k, d)
-                            : bwd_workspace_layout(B, Hq, Hkv, Nq, Nk, d);
   FwdParams p;
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Nq = Nq; p.Nk = Nk;
   p.group = Hq / Hkv;
@@ -350,10 +357,11 @@ int recompute_d(const void* q, const void* k, const void* v, const void* o, cons
   p.total_q = rows_q;
   p.total_k = rows_k;
   p.o_res = nullptr;
-  p.d_out = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.d_off);
+  p.d_out = reinterpret_cast<float*>(ws + w.d_off);
   p.d_ld = vl ? varlen_lpad_ld(B, vl->total_q) : (long long)round_up(Nq, 128);
   p.dO = static_cast<const __nv_bfloat16*>(dO);
   p.do_sb = st[4].b; p.do_sh = st[4].h; p.do_sn = st[4].n;
+  p.v_amax = v16 ? reinterpret_cast<const unsigned*>(ws + w.amax_off) + 1 : nullptr;
   return launch_fwd_any(mq, mk, mv, mo, p, d, causal, stream);
 }
 

@@ -191,14 +191,7 @@ __device__ __forceinline__ void varlen_rows(const int* cu, int b, int total, int
 // (relative rounding 2^-11 instead of bf16's 2^-8), which keeps dV within
 // the parity bound without a second (lo) product; the kernels multiply
 // dP^T by 2^-(e_dO + e_V) and dV by 2^-e_dO, exactly.
-__host__ __device__ __forceinline__ int f16_exp(unsigned amax_bits) {
-  const int ex = int((amax_bits >> 23) & 0xFFu);   // biased exponent of m (m >= 0)
-  if (ex == 255 || amax_bits == 0u) return 0;      // inf / NaN, or all zero: no scaling
-  if (ex == 0) return 60;                          // m below the normal range
-  const int k = ex - 126;                          // m = f * 2^k with f in [0.5, 1)
-  const int e = 15 - k;
-  return e < -60 ? -60 : (e > 60 ? 60 : e);
-}
+// (f16_exp, the exponent rule, is in fa_rows.cuh.)
 
 // Largest |x| over one thread's 8 bf16 elements.
 __device__ __forceinline__ float absmax8(uint4 v) {

@@ -77,6 +77,10 @@ struct FwdParams {
   long long d_ld;
   const __nv_bfloat16* dO;
   long long do_sb, do_sh, do_sn;
+  // D epilogue of the tile-pair kernel: V is the backward workspace's fp16
+  // copy, scaled by 2^f16_exp(*v_amax) (the largest |V|), and P V is one
+  // fp16 product.  Null elsewhere.
+  const unsigned* v_amax = nullptr;
 };
 
 // Kernel variants: fixed-length batch, block-sparse, variable-length batch.
@@ -189,7 +193,8 @@ struct RowState {
 // HALVES: once the first half of the block's keys has its P in TMEM, the
 // thread arrives on p_half (the MMA issuer starts that half's P V); the
 // caller arrives on the block's P-full barrier after the function returns.
-template <int BC, int D, bool CAUSAL, bool SPLIT_P = false, bool HALVES = false>
+template <int BC, int D, bool CAUSAL, bool SPLIT_P = false, bool HALVES = false,
+          bool F16P = false>
 __device__ __forceinline__ bool softmax_block(RowState& st, uint32_t tS, uint32_t tO, int j,
                                               bool first, int gj, int q_tile, int grow, int Nk,
                                               float sl2,
@@ -267,6 +272,10 @@ __device__ __forceinline__ bool softmax_block(RowState& st, uint32_t tS, uint32_
       const float2 t = ffma2(make_float2(s[e], s[e + 1]), sl22, neg2);
       const float2 pp = make_float2(ex2(t.x), ex2(t.y));
       al[i & 3] = fadd2(al[i & 3], pp);
+      if constexpr (F16P) {                        // fp16 P (the D epilogue; normalised by l)
+        pk[i] = pack_f16(pp.x, pp.y);
+        continue;
+      }
       const uint32_t pr = pack_bf16(pp.x, pp.y);
       ar[i & 3] = fadd2(ar[i & 3], make_float2(__uint_as_float(pr << 16),
                                                __uint_as_float(pr & 0xFFFF0000u)));
@@ -306,10 +315,11 @@ template <int D, bool VARLEN, int EPI>
 __device__ __forceinline__ void softmax_finish(const RowState& st, uint32_t tO, uint8_t* stage,
                                                int w, int lane, const CUtensorMap* tmO,
                                                int q_tile, const SeqGeo& g, long long o_sn,
-                                               long long do_sn, int H, int grow) {
-  // The residual and D epilogues' P V used P as hi + lo: normalise by the
-  // fp32 sum of P.
-  const float inv = 1.0f / (EPI != EPI_O ? st.l : st.lr);
+                                               long long do_sn, int H, int grow,
+                                               float o_mul = 1.f) {
+  // The residual and D epilogues' P V used P as hi + lo (or as fp16): normalise
+  // by the fp32 sum of P.  o_mul undoes the scale of an fp16 copy of V.
+  const float inv = o_mul / (EPI != EPI_O ? st.l : st.lr);
   if constexpr (EPI == EPI_D) {
     const bool row_ok = grow < g.nq;
     const uint4* dor = reinterpret_cast<const uint4*>(g.dO + (long long)(row_ok ? grow : 0) * do_sn);
@@ -435,6 +445,9 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
   using C = FwdPairCfg<D>;
   constexpr int BR = C::BR, BC = C::BC, NS = C::NS;
   constexpr bool SPARSE = MODE == MODE_SPARSE, VARLEN = MODE == MODE_VARLEN;
+  // The D epilogue reads V as the backward workspace's scaled fp16 copy and
+  // multiplies it by P as fp16 (one product; p.v_amax gives the scale).
+  constexpr bool PV16 = EPI == EPI_D;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -617,7 +630,8 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_bf16_f32(BR, BC, 0, 0);
-      constexpr uint32_t IDESC_O = idesc_bf16_f32(BR, D, 0, 1);
+      constexpr uint32_t IDESC_O =
+          PV16 ? idesc_f16_f32(BR, D, 0, 1) : idesc_bf16_f32(BR, D, 0, 1);
       const uint32_t sQ_addr = smem_u32(sQ);
       const uint32_t sKV_addr = smem_u32(sKV);
       int cnt = 0;                                 // K/V ring position
@@ -670,7 +684,7 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
           return false;
         // the residual and D epilogues also add P_lo V (P_lo in the block's
         // last BC/2 columns)
-        constexpr int NPH = EPI != EPI_O ? 2 : 1;
+        constexpr int NPH = (EPI != EPI_O && !PV16) ? 2 : 1;
         constexpr int NH = C::P_HALVES ? 2 : 1;         // P handed over in NH parts
         constexpr int KH = BC / 16 / NH;                // k-steps per part
         if constexpr (NPH == 1 && NH == 1) {
@@ -821,6 +835,8 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
     const int row = w * 32 + lane;
     const uint32_t tl = tmem + t * C::TM_TILE + (uint32_t(w * 32) << 16);
     uint64_t* o_done = bar_o_done + t * 2;
+    float o_mul = 1.f;                              // undoes the fp16 copy's scale of V
+    if constexpr (PV16) o_mul = ldexpf(1.f, -f16_exp(__ldg(p.v_amax)));
     int gb = 0;                                     // running block count of this tile
     bool ok = true;
     for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
@@ -854,7 +870,7 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
           ok = mbar_wait(bar_s_full + t, (gb + j) & 1, abort_flag, p.status, W_S_FULL);
           if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
           tc_fence_after();
-          ok = softmax_block<BC, D, CAUSAL, EPI != EPI_O, C::P_HALVES>(
+          ok = softmax_block<BC, D, CAUSAL, EPI != EPI_O && !PV16, C::P_HALVES, PV16>(
               st, tl, tl + 128, j, j == 0, gb + j, q_tile, grow, sg.nk, p.scale_log2, o_done,
               abort_flag, p.status, bar_p_half + t);
           if (!ok) break;
@@ -871,7 +887,7 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
           ok = mbar_wait(bar_s_full + t, (gb + l) & 1, abort_flag, p.status, W_S_FULL);
           if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
           tc_fence_after();
-          ok = softmax_block<BC, D, CAUSAL, EPI != EPI_O, C::P_HALVES>(
+          ok = softmax_block<BC, D, CAUSAL, EPI != EPI_O && !PV16, C::P_HALVES, PV16>(
               st, tl, tl + 128, j, l == 0, gb + l, q_tile, grow, sg.nk, p.scale_log2, o_done,
               abort_flag, p.status, bar_p_half + t);
           if (!ok) break;
@@ -884,7 +900,7 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
       softmax_finish<D, VARLEN, EPI>(st, tl + 128, sQ + t * C::Q_BYTES, w, lane, &tmO, q_tile,
-                                     sg, p.o_sn, p.do_sn, p.Hq, grow);
+                                     sg, p.o_sn, p.do_sn, p.Hq, grow, o_mul);
       tc_fence_before();
       mbar_arrive(bar_o_free + t);                  // O has been read out of TMEM
       if (lane == 0) mbar_arrive(bar_q_free + t);   // this warp's staging boxes were read

@@ -105,8 +105,8 @@ size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int 
  * Wide groups (Hq / Hkv >= 16, e.g. MQA; at d = 256 every Hq / Hkv >= 2):
  * dk sums dS^T q over every query row of the group, so the rounding of
  * D = rowsum(dO * O) from the bf16 o adds up; the pass then recomputes D
- * from the fp32 output with one more forward pass (about the forward's
- * time).  fa_fwd_residual / fa_bwd_residual give the same precision
+ * from the fp32 output with one more forward pass (below the forward's
+ * time: at d <= 128 it multiplies P, as fp16, by the fp16 copy of v).  fa_fwd_residual / fa_bwd_residual give the same precision
  * without it.  For these groups every product takes fp16 operands (q and
  * k are copied like dO and v below) and dS goes in rounded to fp16, scaled
  * by a power of two chosen from the bound |dS| <= 2 d max|dO| max|v|.

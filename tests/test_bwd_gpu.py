@@ -204,14 +204,19 @@ def test_fp16_operand_scales_follow_a_power_of_two(wl, k):
     must multiply every gradient by exactly 2^k: the kernels' powers of two
     absorb k (including max |dO| near 2^18, beyond fp16's range, for
     k = 16).  The only difference allowed is the order of the fp32
-    reduce-adds of dQ and of split dK / dV, at most one bf16 ulp.  With the
-    parity tests at k = 0 this covers dO at any scale."""
+    reduce-adds of dQ and of split dK / dV (atomics, in no fixed order):
+    one bf16 ulp, plus fp32 rounding noise on elements whose partial sums
+    cancel (2^-16 of the largest gradient; a wrong power of two would be a
+    factor of 2).  With the parity tests at k = 0 this covers dO at any
+    scale."""
     base = _grads_with_do_scaled(wl, 0)
     scaled = _grads_with_do_scaled(wl, k)
     for name, g0, gk in zip(("dQ", "dK", "dV"), base, scaled):
         assert np.isfinite(gk).all(), name
         back = gk * 2.0 ** -k
         ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(g0), 1e-300))) - 7)
+        tol = ulp + 2.0 ** -16 * np.abs(g0).max()
         diff = np.abs(back - g0)
-        assert (diff[g0 == 0] == 0).all(), name
-        assert (diff <= ulp + 1e-300).all(), f"{name}: max ulp {float((diff / ulp).max())}"
+        assert (diff <= tol).all(), (
+            f"{name}: worst {float((diff / tol).max()):.2f} x the allowance, "
+            f"max |diff| {float(diff.max()):.3e}, max |g| {float(np.abs(g0).max()):.3e}")
