@@ -504,6 +504,7 @@ struct BwdParams {
   const unsigned* amax;  // workspace words: largest |dO|, |V| (their fp16 scales, f16_exp)
   int gsplit;         // CTAs sharing one kv group's query heads (1 = none)
   int hps;            // query heads per CTA: group / gsplit
+  int hg;             // > 0: kv heads per group of the longest-first CTA order (bwd_cta)
   float* dkacc;       // fp32 dK / dV partial sums when gsplit > 1
   float* dvacc;
   DevStatus* status;
@@ -522,6 +523,32 @@ struct BwdParams {
   __nv_bfloat16* dv;
   Strides sdk, sdv;
 };
+
+// CTA order of the main kernels (after the d-half index, which varies
+// fastest in the general kernel).  By default the group share varies
+// fastest, then the key block, then the (batch, kv head): the CTAs running
+// at once work on one or two heads, whose Q, dO and fp32 dQ rows stay in L2.
+// Under the causal mask a key block's walk shrinks as the block moves right,
+// so in that order the last head's longest CTAs start at the end of the grid
+// and run on while the other SMs idle.  With hg > 0 the kv heads go in
+// groups of hg (sized on the host so that a group's rows fit in L2) and,
+// inside a group, key block by key block across the group's heads: the
+// longest walks first, the shortest last.
+__device__ __forceinline__ void bwd_cta(const BwdParams& p, int rest, int& gs, int& kb, int& bkv) {
+  gs = rest % p.gsplit;
+  rest /= p.gsplit;
+  if (p.hg > 0) {
+    const int per = p.hg * p.n_kblocks;              // CTAs of a full group
+    const int grp = rest / per;
+    const int r = rest - grp * per;
+    const int hgt = min(p.hg, p.B * p.Hkv - grp * p.hg);   // the last group may be short
+    kb = r / hgt;
+    bkv = grp * p.hg + (r - kb * hgt);
+  } else {
+    kb = rest % p.n_kblocks;
+    bkv = rest / p.n_kblocks;
+  }
+}
 
 enum : int { BMODE_DENSE = 0, BMODE_SPARSE = 1, BMODE_VARLEN = 2 };
 
@@ -614,16 +641,12 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // Work unit: (batch, kv head, key block, d half).  Key blocks near the
-  // start see the most query blocks under the causal mask; they go first.
+  // Work unit: (batch, kv head, key block, d half), in bwd_cta's order.
   // With a large GQA/MQA group and few key blocks, the group's query heads
   // are split over `gsplit` CTAs that add fp32 partial dK / dV.
   const int split = blockIdx.x % C::NSPLIT;
-  int rest = blockIdx.x / C::NSPLIT;
-  const int gs = rest % p.gsplit;
-  rest /= p.gsplit;
-  const int kb = rest % p.n_kblocks;
-  const int bkv = rest / p.n_kblocks;
+  int gs, kb, bkv;
+  bwd_cta(p, blockIdx.x / C::NSPLIT, gs, kb, bkv);
   const int b = bkv / p.Hkv;
   const int hkv = bkv - b * p.Hkv;
   const int key0 = kb * BC;
@@ -1293,6 +1316,17 @@ int launch_bwd_t(int stages, const void* q, const void* k, const void* v, const 
     p.amax = f16 ? amax : nullptr;
     p.gsplit = gsplit;
     p.hps = group / gsplit;
+    // Longest-first CTA order for the dense causal backward at d = 128, in
+    // groups of kv heads whose Q and dO (2 bytes an element each) and fp32
+    // dQ rows (4 bytes) take at most 16 MiB of L2.  Measured against the
+    // key-block-fastest order: causal N = 4096 +4 %, N = 2048 +4 % (16 MiB
+    // beat 48 and 96); at d = 64 every budget was 1-2 % slower.
+    p.hg = 0;
+    if (CAUSAL && D == 128 && !vl && !mask) {
+      const long long per_head = (long long)group * Nq_pad * D * 8;
+      p.hg = int(std::max<long long>(1, std::min<long long>((16LL << 20) / per_head,
+                                                            (long long)B * Hkv)));
+    }
     p.dkacc = kvacc;
     p.dvacc = kvacc + w.kv_elems;
     p.n_qblocks = (Nq + BRK - 1) / BRK;

@@ -106,11 +106,9 @@ __global__ void __launch_bounds__(Bwd128Cfg<D>::NTHREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // Work unit: (batch, kv head, key block[, group share]) as in the general kernel.
-  const int gs = blockIdx.x % p.gsplit;
-  int rest = blockIdx.x / p.gsplit;
-  const int kb = rest % p.n_kblocks;
-  const int bkv = rest / p.n_kblocks;
+  // Work unit: (batch, kv head, key block[, group share]) in bwd_cta's order.
+  int gs, kb, bkv;
+  bwd_cta(p, blockIdx.x, gs, kb, bkv);
   const int b = bkv / p.Hkv;
   const int hkv = bkv - b * p.Hkv;
   const int key0 = kb * BC;
