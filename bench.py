@@ -132,10 +132,12 @@ NVML_REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdow
                     "hw_thermal_slowdown": 0x40}
 
 
-def summarise_clock_samples(samples, t0: float, t1: float, max_mhz):
+def summarise_clock_samples(samples, t0: float, t1: float, max_mhz, edges=()):
     """Clock summary of the samples taken inside the timed window [t0, t1]
     (host perf_counter seconds).  samples: (t, sm_mhz, power_w, reason_bits).
-    A reason counts if any window sample has it."""
+    A reason counts if any window sample has it.  edges: samples taken by
+    the timing thread itself at t0 and t1, used only when the polling thread
+    left none in or within 10 ms of the window."""
     win = [x for x in samples if t0 <= x[0] <= t1]
     source = "nvml, 5 ms polling inside the timed region"
     if not win:
@@ -144,6 +146,9 @@ def summarise_clock_samples(samples, t0: float, t1: float, max_mhz):
         near = sorted(samples, key=lambda x: max(t0 - x[0], x[0] - t1))[:1]
         win = [x for x in near if max(t0 - x[0], x[0] - t1) <= 0.010]
         source = "nvml, nearest sample to a timed region shorter than the 5 ms polling"
+    if not win and edges:
+        win = list(edges)
+        source = "nvml, samples at the timed region's start and end (none polled inside it)"
     if not win:
         return {"sm_mhz": None, "sm_max_mhz": max_mhz, "reasons": ["no samples"]}
     reasons = sorted(n for n, bit in NVML_REASON_BITS.items() if any(x[3] & bit for x in win))
@@ -170,6 +175,7 @@ class ClockSampler:
         self.nvml = None
         self.handle = None
         self.samples = []
+        self.edges = []
         self.running = False
         self.thread = None
         self.t0 = self.t1 = 0.0
@@ -184,14 +190,22 @@ class ClockSampler:
         except Exception:
             return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.index)
 
-    def _poll(self):
+    def _sample(self):
         nv, h = self.nvml, self.handle
+        return (time.perf_counter(), float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                nv.nvmlDeviceGetPowerUsage(h) / 1000.0,
+                int(nv.nvmlDeviceGetCurrentClocksEventReasons(h)))
+
+    def _edge(self):
+        try:
+            self.edges.append(self._sample())
+        except Exception:
+            pass
+
+    def _poll(self):
         while self.running:
             try:
-                self.samples.append((time.perf_counter(),
-                                     float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
-                                     nv.nvmlDeviceGetPowerUsage(h) / 1000.0,
-                                     int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))))
+                self.samples.append(self._sample())
             except Exception:
                 pass
             time.sleep(0.005)
@@ -204,6 +218,7 @@ class ClockSampler:
             self.thread = threading.Thread(target=self._poll, daemon=True)
             self.thread.start()
             time.sleep(0.02)
+            self._edge()
             self.t0 = time.perf_counter()
             return
         except Exception:
@@ -222,13 +237,14 @@ class ClockSampler:
     def stop(self):
         if self.nvml is not None:
             self.t1 = time.perf_counter()
+            self._edge()
             self.running = False
             self.thread.join()
             try:
                 mx = float(self.nvml.nvmlDeviceGetMaxClockInfo(self.handle, self.nvml.NVML_CLOCK_SM))
             except Exception:
                 mx = None
-            return summarise_clock_samples(self.samples, self.t0, self.t1, mx)
+            return summarise_clock_samples(self.samples, self.t0, self.t1, mx, self.edges)
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         time.sleep(0.15)

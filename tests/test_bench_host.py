@@ -78,6 +78,21 @@ def test_nvml_samples_outside_the_timed_window_are_dropped():
     assert c["samples"] == 1 and c["sm_mhz"] == 1850.0 and "nearest" in c["source"]
 
 
+def test_edge_samples_stand_in_only_when_polling_left_none():
+    """The samples the timing thread takes itself at the region's start and
+    end are used only when the polling thread took none in or near it."""
+    cap = bench.NVML_REASON_BITS["sw_power_cap"]
+    polled = [(0.0, 1965.0, 90.0, 0), (1.1, 1800.0, 900.0, cap), (5.0, 1965.0, 95.0, 0)]
+    edges = [(1.0, 1700.0, 800.0, 0), (2.0, 1750.0, 850.0, cap)]
+    c = bench.summarise_clock_samples(polled, 1.0, 2.0, 1965.0, edges)
+    assert c["samples"] == 1 and c["sm_mhz"] == 1800.0 and "edge" not in c["source"]
+    c = bench.summarise_clock_samples(polled, 2.5, 3.5, 1965.0, [(2.5, 1700.0, 800.0, 0),
+                                                                (3.5, 1750.0, 850.0, cap)])
+    assert c["samples"] == 2 and c["sm_mhz"] == 1725.0 and c["reasons"] == ["sw_power_cap"]
+    assert "start and end" in c["source"]
+    assert bench.summarise_clock_samples(polled, 2.5, 3.5, 1965.0, [])["reasons"] == ["no samples"]
+
+
 def test_traffic_is_reported_only_for_current_sources(tmp_path, monkeypatch):
     prof = tmp_path / "profiles"
     prof.mkdir()
