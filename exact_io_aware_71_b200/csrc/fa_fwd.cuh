@@ -21,7 +21,8 @@
 //    one head and streams K/V once for both.  Warps 0-3 and 4-7 are the two
 //    tiles' softmax warpgroups; in the third warpgroup warp 8 is the TMA
 //    producer, warp 9 the MMA issuer (10, 11 idle).  TMEM holds S and O of
-//    each tile (2 x (128 + d) columns); while one warpgroup exponentiates its
+//    each tile (2 x (128 + d) columns, + 16 at d = 64 where the P V product
+//    also sums the rounded P); while one warpgroup exponentiates its
 //    S, the tensor pipe works on the other tile, and two softmax warps share
 //    each SM sub-partition.  The softmax warpgroups take 208 registers per
 //    thread from the third warpgroup's share (setmaxnreg, 208 / 88).
@@ -168,7 +169,8 @@ enum : unsigned { W_Q = 1, W_KV_EMPTY, W_KV_FULL, W_S_FULL, W_P_FULL, W_O_DONE, 
 // l: fp32 sum of the probabilities (for the log-sum-exp); lr: the same
 // probabilities after rounding to bf16, i.e. the weights that actually
 // multiply V, so that O = sum(p~ v) / sum(p~) stays a convex combination
-// even when one key dominates a row.
+// even when one key dominates a row.  At d = 64 (plain output) the tensor
+// core forms that sum instead, in O's TMEM column d (LR_TC).
 struct RowState {
   float m, l, lr;
 };
@@ -193,8 +195,11 @@ struct RowState {
 // HALVES: once the first half of the block's keys has its P in TMEM, the
 // thread arrives on p_half (the MMA issuer starts that half's P V); the
 // caller arrives on the block's P-full barrier after the function returns.
+// LR_TC: the tensor core forms the sum of the rounded P (the P V product has a
+// column of ones beyond V's d columns, so O's TMEM column D holds it); the
+// thread neither adds it up nor keeps it, but rescales that column with O.
 template <int BC, int D, bool CAUSAL, bool SPLIT_P = false, bool HALVES = false,
-          bool F16P = false>
+          bool F16P = false, bool LR_TC = false>
 __device__ __forceinline__ bool softmax_block(RowState& st, uint32_t tS, uint32_t tO, int j,
                                               bool first, int gj, int q_tile, int grow, int Nk,
                                               float sl2,
@@ -250,6 +255,13 @@ __device__ __forceinline__ bool softmax_block(RowState& st, uint32_t tS, uint32_
         for (int i = 0; i < 16; ++i) r2[i] = fmul2(r2[i], make_float2(alpha, alpha));
         FA_TMEM_ST32(tO + c * 32, r);
       }
+      if constexpr (LR_TC) {
+        uint32_t r;
+        FA_TMEM_LD1(tO + D, r);
+        tmem_wait_ld();
+        r = __float_as_uint(__uint_as_float(r) * alpha);
+        FA_TMEM_ST1(tO + D, r);
+      }
       tmem_wait_st();
       st.l *= alpha;
       st.lr *= alpha;
@@ -277,8 +289,11 @@ __device__ __forceinline__ bool softmax_block(RowState& st, uint32_t tS, uint32_
         continue;
       }
       const uint32_t pr = pack_bf16(pp.x, pp.y);
-      ar[i & 3] = fadd2(ar[i & 3], make_float2(__uint_as_float(pr << 16),
-                                               __uint_as_float(pr & 0xFFFF0000u)));
+      if constexpr (LR_TC) {
+        pk[i] = pr;
+        continue;
+      }
+      ar[i & 3] = make_float2(add_bf16_lo(pr, ar[i & 3].x), add_bf16_hi(pr, ar[i & 3].y));
       pk[i] = pr;
       if constexpr (SPLIT_P)
         lo[i] = pack_bf16(pp.x - __uint_as_float(pr << 16), pp.y - __uint_as_float(pr & 0xFFFF0000u));
@@ -311,7 +326,7 @@ __device__ __forceinline__ bool softmax_block(RowState& st, uint32_t tS, uint32_
 // bf16(O - bf16(O)) is stored directly as well.  In the D epilogue
 // (g.dpad set) the row's fp32 output is only dotted with its row of dO and
 // D is written; O and the LSE are left alone.
-template <int D, bool VARLEN, int EPI>
+template <int D, bool VARLEN, int EPI, bool LR_TC = false>
 __device__ __forceinline__ void softmax_finish(const RowState& st, uint32_t tO, uint8_t* stage,
                                                int w, int lane, const CUtensorMap* tmO,
                                                int q_tile, const SeqGeo& g, long long o_sn,
@@ -319,7 +334,14 @@ __device__ __forceinline__ void softmax_finish(const RowState& st, uint32_t tO, 
                                                float o_mul = 1.f) {
   // The residual and D epilogues' P V used P as hi + lo (or as fp16): normalise
   // by the fp32 sum of P.  o_mul undoes the scale of an fp16 copy of V.
-  const float inv = o_mul / (EPI != EPI_O ? st.l : st.lr);
+  float lr = st.lr;
+  if constexpr (LR_TC) {
+    uint32_t r;
+    FA_TMEM_LD1(tO + D, r);
+    tmem_wait_ld();
+    lr = __uint_as_float(r);
+  }
+  const float inv = o_mul / (EPI != EPI_O ? st.l : lr);
   if constexpr (EPI == EPI_D) {
     const bool row_ok = grow < g.nq;
     const uint4* dor = reinterpret_cast<const uint4*>(g.dO + (long long)(row_ok ? grow : 0) * do_sn);
@@ -416,8 +438,13 @@ struct FwdPairCfg {
   static constexpr int REGS_SOFTMAX = 208;          // per thread, warpgroups 0 and 1
   static constexpr int REGS_OTHER = 88;             // per thread, warpgroup 2
   static constexpr int REGS_NEEDED = 256 * REGS_SOFTMAX + 128 * REGS_OTHER;
-  static constexpr int SMEM_BYTES = 2 * Q_BYTES + NS * KV_BYTES + 1024 + 1024;
-  static_assert(128 + D <= TM_TILE, "TMEM budget");
+  // d = 64: a 128 x 64 bf16 chunk of ones after the K/V ring, the P V
+  // product's extra B columns (its N = d + 16), so that O's column d sums
+  // the rounded P on the tensor core.
+  static constexpr bool LR_TC = D == 64;
+  static constexpr int ONES_BYTES = LR_TC ? BC * 128 : 0;
+  static constexpr int SMEM_BYTES = 2 * Q_BYTES + NS * KV_BYTES + ONES_BYTES + 1024 + 1024;
+  static_assert(128 + D + (LR_TC ? 16 : 0) <= TM_TILE, "TMEM budget");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
@@ -448,13 +475,17 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
   // The D epilogue reads V as the backward workspace's scaled fp16 copy and
   // multiplies it by P as fp16 (one product; p.v_amax gives the scale).
   constexpr bool PV16 = EPI == EPI_D;
+  // The tensor core sums the rounded P (plain output with one bf16 P only).
+  constexpr bool LR_TC = C::LR_TC && EPI == EPI_O;
+  constexpr int NO = D + (LR_TC ? 16 : 0);       // P V product's N
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* sQ = smem;                          // 2 tiles of [KCH][BR][128B]; O staging later
   uint8_t* sKV = smem + 2 * C::Q_BYTES;        // NS slots of [KCH][BC][128B]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + NS * C::KV_BYTES);
+  uint8_t* sOnes = sKV + NS * C::KV_BYTES;     // [BC][128B] bf16 ones (d = 64)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sOnes + C::ONES_BYTES);
   uint64_t* bar_q = bars + 0;                  // [2] Q tile loaded
   uint64_t* bar_kv_full = bars + 2;            // [NS]
   uint64_t* bar_kv_empty = bars + 2 + NS;      // [NS]
@@ -527,6 +558,12 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
   if (warp == 9) {
     tmem_alloc(tmem_holder, C::TMEM_COLS);
     tmem_relinquish();
+  }
+  if constexpr (C::ONES_BYTES > 0) {
+    uint4* o4 = reinterpret_cast<uint4*>(sOnes);
+    for (int i = threadIdx.x; i < C::ONES_BYTES / 16; i += C::NTHREADS)
+      o4[i] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+    fence_proxy_async_smem();                  // the tensor core reads it
   }
   tc_fence_before();
   __syncthreads();
@@ -631,7 +668,7 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_bf16_f32(BR, BC, 0, 0);
       constexpr uint32_t IDESC_O =
-          PV16 ? idesc_f16_f32(BR, D, 0, 1) : idesc_bf16_f32(BR, D, 0, 1);
+          PV16 ? idesc_f16_f32(BR, NO, 0, 1) : idesc_bf16_f32(BR, NO, 0, 1);
       const uint32_t sQ_addr = smem_u32(sQ);
       const uint32_t sKV_addr = smem_u32(sKV);
       int cnt = 0;                                 // K/V ring position
@@ -651,10 +688,23 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
       const uint32_t qlo = sdesc_sw128_lo(sQ_addr, 16);
       const uint32_t klo = sdesc_sw128_lo(sKV_addr, 16);
       const uint32_t vlo = sdesc_sw128_lo(sKV_addr, BC * 128);
+      // V of ring slot `slot` as the P V product's B operand.  With LR_TC its
+      // 64-column chunks step by the leading byte offset to the ones chunk,
+      // which holds the product's columns d .. d + 15.
+      const uint32_t ones_addr = smem_u32(sOnes);
+      auto vdesc = [&](int slot) -> uint32_t {
+        if constexpr (LR_TC) {
+          const uint32_t a = sKV_addr + uint32_t(slot * C::KV_BYTES);
+          return sdesc_sw128_lo(a, ones_addr - a);
+        } else {
+          return vlo + uint32_t(slot * (C::KV_BYTES >> 4));
+        }
+      };
       // At d = 128 the descriptors are built per k-step from the byte
       // address instead: measured about 2% faster there (and 3% slower at
       // d = 64) than adding offsets to precomputed low words.
       constexpr bool LEAN = D != 128;
+      static_assert(LEAN || !LR_TC, "the ones chunk is addressed through the low-word descriptors");
       auto mma_s = [&](int t, int slot) {
         if constexpr (LEAN) {
           const uint32_t a0 = qlo + uint32_t(t * (C::Q_BYTES >> 4));
@@ -692,7 +742,7 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
           tc_fence_after();
           const uint32_t tt = tmem + t * C::TM_TILE;
           if constexpr (LEAN) {
-            const uint32_t b0 = vlo + uint32_t(slot * (C::KV_BYTES >> 4));
+            const uint32_t b0 = vdesc(slot);
 #pragma unroll
             for (int kk = 0; kk < BC / 16; ++kk)
               umma_ts_lo(tt + 128, tt + kk * 8, b0 + kk * 128, IDESC_O,
@@ -714,7 +764,7 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
           if (!mbar_wait(pb, gj & 1, abort_flag, p.status, W_P_FULL)) return false;
           tc_fence_after();
           if constexpr (LEAN) {
-            const uint32_t b0 = vlo + uint32_t(slot * (C::KV_BYTES >> 4));
+            const uint32_t b0 = vdesc(slot);
 #pragma unroll
             for (int ph = 0; ph < NPH; ++ph)
 #pragma unroll
@@ -870,7 +920,7 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
           ok = mbar_wait(bar_s_full + t, (gb + j) & 1, abort_flag, p.status, W_S_FULL);
           if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
           tc_fence_after();
-          ok = softmax_block<BC, D, CAUSAL, EPI != EPI_O && !PV16, C::P_HALVES, PV16>(
+          ok = softmax_block<BC, D, CAUSAL, EPI != EPI_O && !PV16, C::P_HALVES, PV16, LR_TC>(
               st, tl, tl + 128, j, j == 0, gb + j, q_tile, grow, sg.nk, p.scale_log2, o_done,
               abort_flag, p.status, bar_p_half + t);
           if (!ok) break;
@@ -887,7 +937,7 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
           ok = mbar_wait(bar_s_full + t, (gb + l) & 1, abort_flag, p.status, W_S_FULL);
           if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
           tc_fence_after();
-          ok = softmax_block<BC, D, CAUSAL, EPI != EPI_O && !PV16, C::P_HALVES, PV16>(
+          ok = softmax_block<BC, D, CAUSAL, EPI != EPI_O && !PV16, C::P_HALVES, PV16, LR_TC>(
               st, tl, tl + 128, j, l == 0, gb + l, q_tile, grow, sg.nk, p.scale_log2, o_done,
               abort_flag, p.status, bar_p_half + t);
           if (!ok) break;
@@ -899,8 +949,8 @@ __global__ void __launch_bounds__(FwdPairCfg<D>::NTHREADS, 1)
       ok = mbar_wait(o_done + (jl & 1), (jl >> 1) & 1, abort_flag, p.status, W_O_DONE);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
-      softmax_finish<D, VARLEN, EPI>(st, tl + 128, sQ + t * C::Q_BYTES, w, lane, &tmO, q_tile,
-                                     sg, p.o_sn, p.do_sn, p.Hq, grow, o_mul);
+      softmax_finish<D, VARLEN, EPI, LR_TC>(st, tl + 128, sQ + t * C::Q_BYTES, w, lane, &tmO,
+                                            q_tile, sg, p.o_sn, p.do_sn, p.Hq, grow, o_mul);
       tc_fence_before();
       mbar_arrive(bar_o_free + t);                  // O has been read out of TMEM
       if (lane == 0) mbar_arrive(bar_q_free + t);   // this warp's staging boxes were read

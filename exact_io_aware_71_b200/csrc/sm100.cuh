@@ -337,6 +337,13 @@ __device__ __forceinline__ void umma_ts_lo(uint32_t d_tmem, uint32_t a_tmem, uin
         "=r"(r[31])                                                                         \
       : "r"(taddr))
 
+#define FA_TMEM_LD1(taddr, r)                                                               \
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];"                         \
+               : "=r"(r)                                                                    \
+               : "r"(taddr))
+#define FA_TMEM_ST1(taddr, r)                                                               \
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(r)    \
+               : "memory")
 #define FA_TMEM_LD16(taddr, r)                                                              \
   asm volatile(                                                                             \
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 "                                             \
@@ -426,6 +433,21 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
+}
+// c + (the low / high bf16 of a packed pair), one fp32 rounding (sm_100
+// mixed-precision add): the same value as widening the bf16 exactly and
+// adding in fp32, in one instruction instead of two.
+__device__ __forceinline__ float add_bf16_lo(uint32_t pr, float c) {
+  float d;
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\t"
+      "add.rn.f32.bf16 %0, lo, %2;\n\t}" : "=f"(d) : "r"(pr), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float add_bf16_hi(uint32_t pr, float c) {
+  float d;
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\t"
+      "add.rn.f32.bf16 %0, hi, %2;\n\t}" : "=f"(d) : "r"(pr), "f"(c));
+  return d;
 }
 __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   __half2 h = __floats2half2_rn(lo, hi);
