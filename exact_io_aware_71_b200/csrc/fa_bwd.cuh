@@ -524,8 +524,8 @@ struct BwdParams {
   Strides sdk, sdv;
 };
 
-// CTA order of the main kernels (after the d-half index, which varies
-// fastest in the general kernel).  By default the group share varies
+// CTA order of the dense causal d = 128 kernel.  By default (and in every
+// other instance, which decode it inline) the group share varies
 // fastest, then the key block, then the (batch, kv head): the CTAs running
 // at once work on one or two heads, whose Q, dO and fp32 dQ rows stay in L2.
 // Under the causal mask a key block's walk shrinks as the block moves right,
@@ -641,12 +641,17 @@ __global__ void __launch_bounds__(BwdCfg<D>::NTHREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // Work unit: (batch, kv head, key block, d half), in bwd_cta's order.
-  // With a large GQA/MQA group and few key blocks, the group's query heads
-  // are split over `gsplit` CTAs that add fp32 partial dK / dV.
+  // Work unit: (batch, kv head, key block, d half), key block fastest after
+  // the d half and the group share (the longest-first order of bwd_cta is
+  // for d = 128 only).  With a large GQA/MQA group and few key blocks, the
+  // group's query heads are split over `gsplit` CTAs that add fp32 partial
+  // dK / dV.
   const int split = blockIdx.x % C::NSPLIT;
-  int gs, kb, bkv;
-  bwd_cta(p, blockIdx.x / C::NSPLIT, gs, kb, bkv);
+  int rest = blockIdx.x / C::NSPLIT;
+  const int gs = rest % p.gsplit;
+  rest /= p.gsplit;
+  const int kb = rest % p.n_kblocks;
+  const int bkv = rest / p.n_kblocks;
   const int b = bkv / p.Hkv;
   const int hkv = bkv - b * p.Hkv;
   const int key0 = kb * BC;

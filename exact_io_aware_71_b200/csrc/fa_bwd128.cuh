@@ -106,9 +106,19 @@ __global__ void __launch_bounds__(Bwd128Cfg<D>::NTHREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // Work unit: (batch, kv head, key block[, group share]) in bwd_cta's order.
+  // Work unit: (batch, kv head, key block[, group share]).  The dense causal
+  // d = 128 instance takes bwd_cta's longest-first order; the others keep
+  // the plain decode inline (sharing bwd_cta cost the d = 64 causal kernel
+  // 3-4 % through its code generation, although the order is the same).
   int gs, kb, bkv;
-  bwd_cta(p, blockIdx.x, gs, kb, bkv);
+  if constexpr (CAUSAL && D == 128 && MODE == BMODE_DENSE) {
+    bwd_cta(p, blockIdx.x, gs, kb, bkv);
+  } else {
+    gs = blockIdx.x % p.gsplit;
+    const int rest = blockIdx.x / p.gsplit;
+    kb = rest % p.n_kblocks;
+    bkv = rest / p.n_kblocks;
+  }
   const int b = bkv / p.Hkv;
   const int hkv = bkv - b * p.Hkv;
   const int key0 = kb * BC;
