@@ -67,6 +67,16 @@ def test_unequal_lengths(nq, nk, causal):
     full_check(W(1, 2, 1, nq, nk, 128, causal, seed=nq + nk))
 
 
+@pytest.mark.parametrize("b,hq,hkv,n", [(1, 9, 9, 2048), (3, 6, 3, 1500)])
+def test_causal_longest_first_head_groups(b, hq, hkv, n):
+    """The causal d = 128 backward orders its CTAs longest walk first inside
+    groups of kv heads whose Q, dO and fp32 dQ rows take at most 16 MiB.
+    Nine heads at N = 2048 (2 MiB each) form groups of 8 and 1; nine kv
+    heads of two query heads at N = 1500 (3 MiB each) form groups of 5 and
+    4.  Both end on a short group, the decode's edge case."""
+    full_check(W(b, hq, hkv, n, n, 128, True, seed=b * 100 + n))
+
+
 @pytest.mark.parametrize("residual", [False, True])
 @pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("causal", [False, True])
