@@ -54,6 +54,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 KERNEL_SOURCES = ["exact_io_aware_71_b200/csrc/sm100.cuh", "exact_io_aware_71_b200/csrc/fa_fwd.cuh",
                   "exact_io_aware_71_b200/csrc/fa_bwd.cuh", "exact_io_aware_71_b200/csrc/fa_mask.cuh",
                   "exact_io_aware_71_b200/csrc/fa_bwd128.cuh", "exact_io_aware_71_b200/csrc/fa_rows.cuh"]
+# The forward kernels are built from these alone (fa_fwd.cuh includes no
+# backward source); the backward's traffic is keyed on all of them.
+FWD_KERNEL_SOURCES = [r for r in KERNEL_SOURCES if "fa_bwd" not in r]
 METRIC = "attention fwd / fwd+bwd TFLOP/s (bf16, 1×B200) and % of dense BF16 peak"
 
 
@@ -90,12 +93,14 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash():
-    """Hash of the kernel sources' code: comments and whitespace are dropped
-    first, so an edit that only touches comments keeps a traffic record."""
+def kernel_source_hash(kernel: str = ""):
+    """Hash of the code of the sources a kernel is built from (the forward
+    kernels' own for names starting with fa_fwd, else all): comments and
+    whitespace are dropped first, so an edit that only touches comments keeps
+    a traffic record, and so does a backward edit for a forward record."""
     import re
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in (FWD_KERNEL_SOURCES if kernel.startswith("fa_fwd") else KERNEL_SOURCES):
         with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
             text = f.read()
         text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
@@ -115,7 +120,7 @@ def recorded_traffic(kernel: str, workload: str):
         return None
     for r in rec.get("entries", []):
         if (r.get("kernel") == kernel and r.get("workload") == workload
-                and r.get("src_sha") == kernel_source_hash()):
+                and r.get("src_sha") == kernel_source_hash(kernel)):
             return r.get("dram_bytes_per_launch")
     return None
 

@@ -115,6 +115,36 @@ def test_traffic_is_reported_only_for_current_sources(tmp_path, monkeypatch):
     assert bench.recorded_traffic("k", "w") is None
 
 
+def test_forward_traffic_survives_backward_edits(tmp_path, monkeypatch):
+    """A forward kernel's record is keyed on the forward's own sources: an
+    edit of a backward source keeps it and drops the backward's record; an
+    edit of a shared header drops both."""
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    for rel in bench.KERNEL_SOURCES:
+        p = tmp_path / rel
+        p.parent.mkdir(parents=True, exist_ok=True)
+        p.write_text("kernel " + rel)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert set(bench.FWD_KERNEL_SOURCES) < set(bench.KERNEL_SOURCES)
+    assert not any("fa_bwd" in r for r in bench.FWD_KERNEL_SOURCES)
+    rec = {"entries": [
+        {"kernel": "fa_fwd_kernel", "workload": "w", "dram_bytes_per_launch": 1,
+         "src_sha": bench.kernel_source_hash("fa_fwd_kernel")},
+        {"kernel": "fa_bwd_main_kernel", "workload": "w", "dram_bytes_per_launch": 2,
+         "src_sha": bench.kernel_source_hash("fa_bwd_main_kernel")}]}
+    (prof / "traffic.json").write_text(json.dumps(rec))
+    assert bench.recorded_traffic("fa_fwd_kernel", "w") == 1
+    assert bench.recorded_traffic("fa_bwd_main_kernel", "w") == 2
+    bwd = next(r for r in bench.KERNEL_SOURCES if r.endswith("fa_bwd128.cuh"))
+    (tmp_path / bwd).write_text("changed")
+    assert bench.recorded_traffic("fa_fwd_kernel", "w") == 1
+    assert bench.recorded_traffic("fa_bwd_main_kernel", "w") is None
+    shared = next(r for r in bench.KERNEL_SOURCES if r.endswith("sm100.cuh"))
+    (tmp_path / shared).write_text("changed")
+    assert bench.recorded_traffic("fa_fwd_kernel", "w") is None
+
+
 def test_peaks_fallback(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     pk, src = bench.load_peaks()
